@@ -1,0 +1,147 @@
+/*
+ * moe_ffn.h - C ABI of libmoe_ffn.so: forward pass of a mixture-of-experts
+ * feed-forward layer with fine-grained routed experts and an always-on shared
+ * expert, on one NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (one call of moe_forward, T tokens of width d):
+ *
+ *   s[t,e]  = x[t,:] . W_g[e,:] + bias[e]                 router scores
+ *   p[t,:]  = softmax(s[t,:]) over all N_r routed experts
+ *   S_t     = the top_k experts by p, ties to the lower expert index
+ *   g[t,i]  = p[t,i]            (renorm = 0), or
+ *             p[t,i] / sum_{j in S_t} p[t,j]   (renorm = 1), for i in S_t
+ *   out[t]  = FFN_shared(x[t]) + sum_{i in S_t} g[t,i] * FFN_i(x[t])
+ *   FFN(u)  = W2 ( SiLU(W1 u) * (W3 u) ),   SiLU(z) = z / (1 + exp(-z))
+ *
+ * Sources: "Shared Expert (DeepSeek-V3)" (ai-engineer-exhaustive), "How it
+ * works": eq. (12) without its residual term u_t (the caller adds the residual
+ * at block level), the SwiGLU definition, and "Official code" (N_s shared
+ * experts fused into one SwiGLU of inner width N_s*f, computed on the whole
+ * packed batch and added with coefficient 1, never gated, never in the top-k
+ * pool). The router (linear scorer, softmax blend weights, keep the top-k) is
+ * "What is an "expert," really?" (svac-llc), glossary and panel 2; the
+ * selected-set sum is "Shared and fine-grained experts", Researcher "Why
+ * segmentation helps".
+ *
+ * Conventions for every call:
+ *  - Tensor pointers are DEVICE pointers owned by the caller, row-major,
+ *    16-byte aligned. bf16 tensors are passed as uint16_t bit patterns.
+ *  - Layouts: x (T, d); W_g (N_r, d); W1, W3 (N_r, f, d); W2 (N_r, d, f);
+ *    W1s, W3s (N_s*f, d); W2s (d, N_s*f); bias (N_r) fp32; out (T, d).
+ *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy default
+ *    stream. Calls that take a stream only enqueue work: they never
+ *    synchronise the host and never allocate device memory.
+ *  - Every call returns a moe_status (0 = OK). On failure, moe_last_error()
+ *    returns a message for the calling thread.
+ *  - A plan is not thread-safe: do not run two forwards of one plan at the
+ *    same time. Distinct plans are independent.
+ */
+#ifndef MOE_FFN_H
+#define MOE_FFN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16_t;               /* bf16 bit pattern */
+typedef struct moe_plan* moe_plan_t;      /* opaque, owned by the library */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_INVALID_CONFIG = 1,   /* layer shape rejected (see moe_plan_create) */
+  MOE_INVALID_ARG = 2,      /* null or misaligned pointer, negative T, ... */
+  MOE_WORKSPACE_TOO_SMALL = 3,
+  MOE_CUDA_ERROR = 4,       /* a CUDA runtime/driver call or launch failed */
+  MOE_UNSUPPORTED = 5,      /* valid layer the kernels do not cover */
+  MOE_DEVICE_TIMEOUT = 6    /* a kernel gave up a bounded wait (see moe_plan_device_status) */
+} moe_status;
+
+/* Create a plan for one layer shape.
+ * d: model width; f: inner width of one routed expert; n_routed: N_r;
+ * top_k: experts kept per token; n_shared: N_s (shared inner width N_s*f);
+ * renorm: 1 to renormalise the selected probabilities to sum 1, 0 for raw.
+ * Rejected with MOE_INVALID_CONFIG (returns NULL) when any of d, f, N_r, top_k
+ * is below 1, N_s is negative or top_k exceeds N_r - the budget rules of
+ * "MoE：细粒度专家与共享专家（shared expert）" (cooking-agi), budget section.
+ * Returns NULL with MOE_UNSUPPORTED when d or f is not a multiple of 8
+ * (16-byte rows), N_r > 1024, top_k > 32 or N_s*f > 2^24.
+ * The plan is bound to the CUDA device current at creation. */
+moe_plan_t moe_plan_create(int d, int f, int n_routed, int top_k, int n_shared,
+                           int renorm);
+
+/* Status of the last moe_plan_create on this thread (MOE_OK if it succeeded). */
+int moe_last_status(void);
+
+/* Optional per-expert logit bias: device pointer to N_r fp32 values added to
+ * the router scores before the softmax (affects both selection and gates).
+ * NULL removes it. The pointer must stay valid while forwards use it. */
+int moe_plan_set_logit_bias(moe_plan_t plan, const float* bias);
+
+/* Bytes of device workspace one forward over T tokens needs (T >= 0). */
+size_t moe_workspace_bytes(moe_plan_t plan, int64_t T);
+
+/* Hand the plan a caller-owned device workspace (256-byte aligned). The plan
+ * keeps the pointer; forwards over T tokens need moe_workspace_bytes(T).
+ * The workspace also holds the routing of the last forward. */
+int moe_plan_set_workspace(moe_plan_t plan, void* workspace, size_t bytes);
+
+/* Forward over T tokens (T = 0 is a no-op returning MOE_OK). x, W_g, W1, W3,
+ * W2 and out must be non-NULL; W1s, W3s, W2s must be NULL exactly when N_s = 0.
+ * Enqueues the whole layer on `stream`: router GEMM, softmax + top-k, expert
+ * histogram + scan + stable permutation, grouped gate/up + SiLU GEMM, grouped
+ * down GEMM, shared SwiGLU GEMMs, weighted combine. No host synchronisation,
+ * no device allocation. Errors: MOE_INVALID_ARG, MOE_WORKSPACE_TOO_SMALL,
+ * MOE_CUDA_ERROR (launch failures are reported, in-kernel faults surface at the
+ * next synchronising CUDA call). */
+int moe_forward(moe_plan_t plan, int64_t T, const moe_bf16_t* x,
+                const moe_bf16_t* W_g, const moe_bf16_t* W1, const moe_bf16_t* W3,
+                const moe_bf16_t* W2, const moe_bf16_t* W1s,
+                const moe_bf16_t* W3s, const moe_bf16_t* W2s, moe_bf16_t* out,
+                void* stream);
+
+/* Copy the routing of the last forward (device to device, enqueued on
+ * `stream`): idx (T, top_k) int32 expert ids in slot order (descending
+ * probability, ties to the lower index); w (T, top_k) fp32 gates; counts (N_r)
+ * int32 rows per expert; offsets (N_r+1) int32 exclusive prefix of counts.
+ * Any output may be NULL. T must equal the last forward's T. */
+int moe_get_routing(moe_plan_t plan, int64_t T, int32_t* idx, float* w,
+                    int32_t* counts, int32_t* offsets, void* stream);
+
+/* Copy the stable permutation of the last forward (device to device):
+ * perm_src (T*top_k) int32 token of each grouped row (rows of expert e are
+ * offsets[e]..offsets[e+1]-1, in ascending (token, slot) order);
+ * inv_pos (T, top_k) int32 grouped row of each (token, slot). NULL skips. */
+int moe_get_permutation(moe_plan_t plan, int64_t T, int32_t* perm_src,
+                        int32_t* inv_pos, void* stream);
+
+/* Read (synchronously) and clear the plan's device status word: MOE_OK, or
+ * MOE_DEVICE_TIMEOUT if a kernel abandoned a bounded wait since the last
+ * read. Kernels never spin without a bound; a timeout means the forward's
+ * output is invalid. */
+int moe_plan_device_status(moe_plan_t plan);
+
+/* Timing: when enabled, moe_forward records a CUDA event on its stream before
+ * every kernel launch and after the last one. moe_plan_kernel_times waits for
+ * the last forward's final event and writes up to `cap` per-kernel durations
+ * in milliseconds; it returns how many kernels the last forward launched (or a
+ * negative moe_status). moe_plan_kernel_name gives the name of kernel i of the
+ * last forward (static string; NULL when out of range). */
+int moe_plan_enable_timing(moe_plan_t plan, int enable);
+int moe_plan_kernel_times(moe_plan_t plan, float* ms, int cap);
+const char* moe_plan_kernel_name(moe_plan_t plan, int i);
+
+/* Number of kernels the last forward of this plan launched. */
+int moe_plan_last_launch_count(moe_plan_t plan);
+
+void moe_plan_destroy(moe_plan_t plan);
+
+const char* moe_strerror(int status);
+const char* moe_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_FFN_H */

@@ -1,0 +1,365 @@
+// gemm_sm100.cuh - grouped bf16 GEMM engine on the 5th-generation tensor core.
+//
+//   C[r, n] = sum_k A[r, k] * B_g[n, k]      for every row r of group g
+//
+// A is a (rows, K) row-major bf16 matrix whose rows are grouped by expert
+// (group g owns rows offsets[g] .. offsets[g+1]-1; group sizes are known only on
+// the device). B_g is expert g's (N, K) row-major bf16 weight, i.e. K-major, as
+// the layer stores W1/W3 (f, d) and W2 (d, f) ("Shared Expert (DeepSeek-V3)",
+// "How it works", SwiGLU definition). A dense GEMM is the special case of one
+// group holding every row (the shared expert and the router).
+//
+// Design (sm_100a):
+//  * persistent: one CTA per SM walks a linear tile list; tile t maps to
+//    (group, n-block, m-block) through a device prefix of per-group m-tile
+//    counts, so no host synchronisation is needed to learn the group sizes;
+//    within a group the m-blocks are innermost so the CTAs running at the same
+//    time share one weight tile through L2;
+//  * warp 0: TMA producer (128B-swizzled boxes, no cluster multicast), a
+//    kStages-deep shared-memory ring guarded by full/empty mbarriers;
+//  * warp 1: allocates 512 TMEM columns, one thread issues
+//    tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) and commits;
+//  * warps 2..5: epilogue, each owns one 32-lane quarter of TMEM; two
+//    256-column accumulators let the epilogue of tile i overlap the MMAs of
+//    tile i+1;
+//  * epilogues: SwiGLU (the 256 accumulator columns are 128 gate columns from
+//    W1 followed by the same 128 columns of W3; writes SiLU(gate)*up as bf16),
+//    plain bf16, plain fp32. Rows past the group's end and columns past N are
+//    masked, so partial tiles never write outside their group.
+#pragma once
+
+#include "ptx_sm100.cuh"
+
+namespace moe {
+
+constexpr int kBM = 128;                       // tile rows (MMA M)
+constexpr int kBN = 256;                       // accumulator columns (MMA N)
+constexpr int kBK = 64;                        // K per stage: one 128-byte swizzle row
+constexpr int kUK = 16;                        // K per tcgen05.mma (kind::f16)
+constexpr int kStages = 4;
+constexpr int kATileBytes = kBM * kBK * 2;     // 16 KB
+constexpr int kBHalfBytes = 128 * kBK * 2;     // 16 KB (one 128-row TMA box)
+constexpr int kBTileBytes = kBN * kBK * 2;     // 32 KB
+constexpr int kStageBytes = kATileBytes + kBTileBytes;
+constexpr int kNumAcc = 2;
+constexpr int kTmemCols = kNumAcc * kBN;       // 512: the whole TMEM of the SM
+constexpr int kGemmThreads = 192;
+constexpr int kEpiThreads = 128;
+
+enum EpiMode : int { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiF32 = 2 };
+
+// Output columns one tile produces.
+__host__ __device__ constexpr int tile_cols(int mode) { return mode == kEpiSwiGLU ? 128 : 256; }
+
+struct GemmParams {
+  const int* group_offsets;  // device (num_groups+1); nullptr: one dense group of dense_rows
+  const int* group_mtiles;   // device (num_groups+1) exclusive prefix of ceil(n_g / 128)
+  int num_groups;
+  int dense_rows;
+  int K;                     // reduction length (elements)
+  int N;                     // valid output columns
+  int n_tiles;               // ceil(N / tile_cols(mode))
+  void* out;                 // bf16 or fp32, row-major
+  long long ldo;             // elements between output rows
+  int* status;               // device status word (moe_status codes)
+};
+
+// Dynamic shared memory the kernel needs for a given number of groups.
+__host__ __device__ constexpr size_t gemm_smem_bytes(int num_groups) {
+  return 1024 /* alignment slack */ + size_t(kStages) * kStageBytes + 256 /* barriers */ +
+         size_t(2) * (num_groups + 1) * sizeof(int);
+}
+
+struct TileCoord {
+  int group, n_blk, row0, rows;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(int tile, const int* s_off, const int* s_mp,
+                                                 int num_groups, int n_tiles) {
+  // largest g with s_mp[g] * n_tiles <= tile (empty groups share a prefix value,
+  // the largest index among them is the next non-empty group)
+  int lo = 0, hi = num_groups;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s_mp[mid] * n_tiles <= tile) lo = mid; else hi = mid;
+  }
+  const int mt = s_mp[lo + 1] - s_mp[lo];
+  const int local = tile - s_mp[lo] * n_tiles;
+  const int n_blk = local / mt;
+  const int m_blk = local - n_blk * mt;
+  TileCoord c;
+  c.group = lo;
+  c.n_blk = n_blk;
+  c.row0 = s_off[lo] + m_blk * kBM;
+  c.rows = min(kBM, s_off[lo + 1] - c.row0);
+  return c;
+}
+
+__device__ __forceinline__ void raise_timeout(volatile int* s_abort, int* status) {
+  *s_abort = 1;
+  atomicExch(status, 6 /* MOE_DEVICE_TIMEOUT */);
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+template <int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                    const __grid_constant__ CUtensorMap tmB1, const GemmParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(kStages) * kStageBytes);
+  uint64_t* full_bar = bars;                       // [kStages] TMA -> MMA
+  uint64_t* empty_bar = bars + kStages;            // [kStages] MMA -> TMA
+  uint64_t* tfull_bar = bars + 2 * kStages;        // [kNumAcc] MMA -> epilogue
+  uint64_t* tempty_bar = tfull_bar + kNumAcc;      // [kNumAcc] epilogue -> MMA
+  uint64_t* drain_bar = tempty_bar + kNumAcc;      // MMA drain on abort
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  int* s_off = reinterpret_cast<int*>(smem + size_t(kStages) * kStageBytes + 256);
+  const int num_groups = P.group_offsets ? P.num_groups : 1;
+  int* s_mp = s_off + (num_groups + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (P.group_offsets) {
+    for (int i = threadIdx.x; i <= num_groups; i += blockDim.x) {
+      s_off[i] = P.group_offsets[i];
+      s_mp[i] = P.group_mtiles[i];
+    }
+  } else if (threadIdx.x == 0) {
+    s_off[0] = 0;
+    s_off[1] = P.dense_rows;
+    s_mp[0] = 0;
+    s_mp[1] = (P.dense_rows + kBM - 1) / kBM;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    for (int b = 0; b < kNumAcc; ++b) {
+      mbar_init(smem_u32(&tfull_bar[b]), 1);
+      mbar_init(smem_u32(&tempty_bar[b]), kEpiThreads);
+    }
+    mbar_init(smem_u32(drain_bar), 1);
+    *s_abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(s_tmem), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *s_tmem;
+
+  const int total_tiles = s_mp[num_groups] * P.n_tiles;
+  const int num_kb = (P.K + kBK - 1) / kBK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    int s = 0;
+    uint32_t ph = 0;
+    uint32_t issued_mask = 0, issued_par = 0;  // per stage: issued at least once / last parity
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      const TileCoord tc = decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles);
+      const int z = P.group_offsets ? tc.group : 0;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        ok = mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, s_abort);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) {
+          if (lane == 0) raise_timeout(s_abort, P.status);
+          break;
+        }
+        if (lane == 0) {
+          const uint32_t fb = smem_u32(&full_bar[s]);
+          const uint32_t a_dst = smem_u32(smem + size_t(s) * kStageBytes);
+          const uint32_t b_dst = a_dst + kATileBytes;
+          const int k0 = kb * kBK;
+          mbar_arrive_expect_tx(fb, kStageBytes);
+          tma_load_2d(a_dst, &tmA, fb, k0, tc.row0);
+          if (MODE == kEpiSwiGLU) {
+            tma_load_3d(b_dst, &tmB0, fb, k0, tc.n_blk * 128, z);
+            tma_load_3d(b_dst + kBHalfBytes, &tmB1, fb, k0, tc.n_blk * 128, z);
+          } else {
+            tma_load_3d(b_dst, &tmB0, fb, k0, tc.n_blk * 256, z);
+            tma_load_3d(b_dst + kBHalfBytes, &tmB0, fb, k0, tc.n_blk * 256 + 128, z);
+          }
+        }
+        __syncwarp();
+        issued_mask |= 1u << s;
+        issued_par = (issued_par & ~(1u << s)) | (ph << s);
+        if (++s == kStages) { s = 0; ph ^= 1u; }
+      }
+    }
+    if (!ok && lane == 0) {
+      // give the copies already issued a bounded chance to land before teardown
+      for (int i = 0; i < kStages; ++i)
+        if (issued_mask & (1u << i)) {
+          int never = 0;
+          mbar_wait(smem_u32(&full_bar[i]), (issued_par >> i) & 1u, &never);
+        }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN);
+    int s = 0;
+    uint32_t ph = 0;
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      ok = mbar_wait(smem_u32(&tempty_bar[acc]), acc_ph ^ 1u, s_abort);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after_sync();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+      for (int kb = 0; kb < num_kb; ++kb) {
+        ok = mbar_wait(smem_u32(&full_bar[s]), ph, s_abort);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after_sync();
+        if (lane == 0) {
+          const uint32_t a_base = smem_u32(smem + size_t(s) * kStageBytes);
+          const uint32_t b_base = a_base + kATileBytes;
+#pragma unroll
+          for (int k = 0; k < kBK / kUK; ++k) {
+            umma_bf16(d_tmem, sdesc_kmajor_sw128(a_base + k * kUK * 2),
+                      sdesc_kmajor_sw128(b_base + k * kUK * 2), idesc,
+                      (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(smem_u32(&empty_bar[s]));   // frees the stage when these MMAs finish
+        }
+        __syncwarp();
+        if (++s == kStages) { s = 0; ph ^= 1u; }
+      }
+      if (!ok) break;
+      if (lane == 0) umma_commit(smem_u32(&tfull_bar[acc]));  // accumulator ready
+      __syncwarp();
+      if (++acc == kNumAcc) { acc = 0; acc_ph ^= 1u; }
+    }
+    if (!ok) {
+      if (lane == 0) {
+        raise_timeout(s_abort, P.status);
+        umma_commit(smem_u32(drain_bar));        // wait for MMAs in flight before teardown
+        int never = 0;
+        mbar_wait(smem_u32(drain_bar), 0, &never);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;                 // TMEM lanes this warp may access
+    const int r = quarter * 32 + lane;            // tile row owned by this thread
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      const TileCoord tc = decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles);
+      bool ok = mbar_wait(smem_u32(&tfull_bar[acc]), acc_ph, s_abort);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) raise_timeout(s_abort, P.status);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t tbase = lane_base + static_cast<uint32_t>(acc * kBN);
+      const bool row_ok = r < tc.rows;
+      const long long grow = static_cast<long long>(tc.row0) + r;
+      if (MODE == kEpiSwiGLU) {
+        const int col0 = tc.n_blk * 128;
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(P.out);
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          if (col0 + c >= P.N) break;              // warp-uniform
+          uint32_t g[32], u[32];
+          tmem_ld_32cols(tbase + c, g);
+          tmem_ld_32cols(tbase + 128 + c, u);
+          tmem_ld_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int col = col0 + c + v * 8;
+              if (col < P.N) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  const float g0 = __uint_as_float(g[v * 8 + 2 * q]);
+                  const float g1 = __uint_as_float(g[v * 8 + 2 * q + 1]);
+                  const float u0 = __uint_as_float(u[v * 8 + 2 * q]);
+                  const float u1 = __uint_as_float(u[v * 8 + 2 * q + 1]);
+                  const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
+                  const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+                  pk[q] = pack_bf16x2(h0, h1);
+                }
+                *reinterpret_cast<uint4*>(out + grow * P.ldo + col) =
+                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              }
+            }
+          }
+        }
+      } else {
+        const int col0 = tc.n_blk * 256;
+#pragma unroll 1
+        for (int c = 0; c < 256; c += 32) {
+          if (col0 + c >= P.N) break;              // warp-uniform
+          uint32_t a[32];
+          tmem_ld_32cols(tbase + c, a);
+          tmem_ld_wait();
+          if (!row_ok) continue;
+          if (MODE == kEpiBF16) {
+            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(P.out);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int col = col0 + c + v * 8;
+              if (col < P.N) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  pk[q] = pack_bf16x2(__uint_as_float(a[v * 8 + 2 * q]),
+                                      __uint_as_float(a[v * 8 + 2 * q + 1]));
+                *reinterpret_cast<uint4*>(out + grow * P.ldo + col) =
+                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              }
+            }
+          } else {
+            float* out = reinterpret_cast<float*>(P.out);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const int col = col0 + c + v * 4;
+              float* dst = out + grow * P.ldo + col;
+              if (col + 4 <= P.N) {
+                *reinterpret_cast<float4*>(dst) =
+                    make_float4(__uint_as_float(a[v * 4]), __uint_as_float(a[v * 4 + 1]),
+                                __uint_as_float(a[v * 4 + 2]), __uint_as_float(a[v * 4 + 3]));
+              } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  if (col + q < P.N) dst[q] = __uint_as_float(a[v * 4 + q]);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before_sync();
+      mbar_arrive(smem_u32(&tempty_bar[acc]));
+      if (++acc == kNumAcc) { acc = 0; acc_ph ^= 1u; }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+}  // namespace moe

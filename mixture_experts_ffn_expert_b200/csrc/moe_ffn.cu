@@ -1,0 +1,552 @@
+// moe_ffn.cu - host planner and C ABI of libmoe_ffn.so (declared in
+// include/moe_ffn.h): validates arguments, lays out the caller's workspace,
+// encodes the TMA tensor maps and enqueues the layer's kernels on the caller's
+// stream. It never synchronises the host in moe_forward and never allocates
+// device memory.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "moe_ffn.h"
+#include "gemm_sm100.cuh"
+#include "route.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+thread_local int g_last_status = MOE_OK;
+
+int fail(int status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  g_last_status = status;
+  return status;
+}
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+constexpr int kMaxKernels = 16;
+
+struct Layout {
+  size_t status, scores, idx, gate, chunk_counts, counts, offsets, mtiles, perm_src, inv_pos;
+  size_t xperm, hidden, yrouted, hshared, yshared, total;
+  int lds;        // row stride of the fp32 router scores
+  int tpc;        // tokens per routing chunk
+  int n_chunks;
+};
+
+}  // namespace
+
+struct moe_plan {
+  int d, f, n_routed, top_k, n_shared, renorm;
+  int device, num_sms;
+  const float* bias = nullptr;
+  char* ws = nullptr;
+  size_t ws_bytes = 0;
+  int64_t last_T = -1;
+  bool timing = false;
+  int n_launch = 0;
+  const char* names[kMaxKernels] = {};
+  cudaEvent_t ev[kMaxKernels + 1] = {};
+  bool events_made = false;
+};
+
+namespace {
+
+Layout make_layout(const moe_plan* p, int64_t T) {
+  Layout L{};
+  const int64_t A = T * p->top_k;
+  const int nsf = p->n_shared * p->f;
+  // chunking of the routing kernels: about two chunks per SM, 8..128 tokens each
+  int64_t tpc = (T + 2 * p->num_sms - 1) / (2 * p->num_sms);
+  tpc = tpc < 8 ? 8 : (tpc > 128 ? 128 : tpc);
+  L.tpc = static_cast<int>(tpc);
+  L.n_chunks = static_cast<int>((T + tpc - 1) / tpc);
+  L.lds = static_cast<int>(align_up(p->n_routed, 8));
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
+  L.status = take(256);
+  L.scores = take(size_t(T) * L.lds * 4);
+  L.idx = take(size_t(A) * 4);
+  L.gate = take(size_t(A) * 4);
+  L.chunk_counts = take(size_t(p->n_routed) * (L.n_chunks > 0 ? L.n_chunks : 1) * 4);
+  L.counts = take(size_t(p->n_routed) * 4);
+  L.offsets = take(size_t(p->n_routed + 1) * 4);
+  L.mtiles = take(size_t(p->n_routed + 1) * 4);
+  L.perm_src = take(size_t(A) * 4);
+  L.inv_pos = take(size_t(A) * 4);
+  L.xperm = take(size_t(A) * p->d * 2);
+  L.hidden = take(size_t(A) * p->f * 2);
+  L.yrouted = take(size_t(A) * p->d * 2);
+  L.hshared = take(size_t(T) * nsf * 2);
+  L.yshared = take(p->n_shared > 0 ? size_t(T) * p->d * 4 : 0);
+  L.total = o;
+  return L;
+}
+
+// ------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// bf16 matrix (rows, cols) row-major, optionally stacked `batch` times; box of
+// 64 columns (128 B, one swizzle row) x 128 rows, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* m, const void* base, uint64_t batch, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cols, rows, batch};
+  cuuint64_t strides[2] = {cols * 2, rows * cols * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const cuuint32_t rank = batch > 0 ? 3 : 2;
+  if (batch == 0) dims[2] = 1;
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------- launches
+struct Launcher {
+  moe_plan* p;
+  cudaStream_t st;
+  int status = MOE_OK;
+
+  void mark(const char* name) {
+    if (p->n_launch < kMaxKernels) {
+      p->names[p->n_launch] = name;
+      if (p->timing) cudaEventRecord(p->ev[p->n_launch], st);
+    }
+    ++p->n_launch;
+  }
+  bool check(const char* what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      status = fail(MOE_CUDA_ERROR, "%s launch failed: %s", what, cudaGetErrorString(e));
+      return false;
+    }
+    return true;
+  }
+  void finish() {
+    if (p->timing && p->n_launch <= kMaxKernels) cudaEventRecord(p->ev[p->n_launch], st);
+  }
+};
+
+template <int MODE>
+bool launch_gemm(Launcher& L, const char* name, const CUtensorMap& a, const CUtensorMap& b0,
+                 const CUtensorMap& b1, const moe::GemmParams& prm, int max_tiles) {
+  const int num_groups = prm.group_offsets ? prm.num_groups : 1;
+  const size_t smem = moe::gemm_smem_bytes(num_groups);
+  int grid = max_tiles < L.p->num_sms ? max_tiles : L.p->num_sms;
+  if (grid < 1) grid = 1;
+  L.mark(name);
+  moe::moe_gemm_kernel<MODE><<<grid, moe::kGemmThreads, smem, L.st>>>(a, b0, b1, prm);
+  return L.check(name);
+}
+
+int set_kernel_attributes() {
+  const size_t smem = moe::gemm_smem_bytes(moe::kMaxRouted);
+  cudaError_t e1 = cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiSwiGLU>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  cudaError_t e2 = cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiBF16>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  cudaError_t e3 = cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiF32>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess)
+    return fail(MOE_CUDA_ERROR, "cudaFuncSetAttribute failed: %s",
+                cudaGetErrorString(e1 != cudaSuccess ? e1 : (e2 != cudaSuccess ? e2 : e3)));
+  return MOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+moe_plan_t moe_plan_create(int d, int f, int n_routed, int top_k, int n_shared, int renorm) {
+  g_last_status = MOE_OK;
+  if (d < 1 || f < 1 || n_routed < 1 || top_k < 1 || n_shared < 0 || top_k > n_routed) {
+    fail(MOE_INVALID_CONFIG,
+         "invalid expert configuration d=%d f=%d n_routed=%d top_k=%d n_shared=%d", d, f,
+         n_routed, top_k, n_shared);
+    return nullptr;
+  }
+  if (d % 8 || f % 8 || n_routed > moe::kMaxRouted || top_k > moe::kMaxTopK ||
+      static_cast<long long>(n_shared) * f > (1LL << 24) || d > (1 << 24) || f > (1 << 24)) {
+    fail(MOE_UNSUPPORTED,
+         "unsupported shape: need d, f multiples of 8, n_routed <= %d, top_k <= %d, "
+         "n_shared*f <= 2^24",
+         moe::kMaxRouted, moe::kMaxTopK);
+    return nullptr;
+  }
+  int dev = 0, sms = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    fail(MOE_CUDA_ERROR, "no usable CUDA device");
+    return nullptr;
+  }
+  if (major != 10 || minor != 0) {
+    fail(MOE_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a only", dev,
+         major, minor);
+    return nullptr;
+  }
+  if (set_kernel_attributes() != MOE_OK) return nullptr;
+  if (!encode_fn()) {
+    fail(MOE_CUDA_ERROR, "cuTensorMapEncodeTiled is not available from the driver");
+    return nullptr;
+  }
+  moe_plan* p = new moe_plan();
+  p->d = d;
+  p->f = f;
+  p->n_routed = n_routed;
+  p->top_k = top_k;
+  p->n_shared = n_shared;
+  p->renorm = renorm ? 1 : 0;
+  p->device = dev;
+  p->num_sms = sms;
+  return p;
+}
+
+int moe_last_status(void) { return g_last_status; }
+
+int moe_plan_set_logit_bias(moe_plan_t p, const float* bias) {
+  if (!p) return fail(MOE_INVALID_ARG, "null plan");
+  if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u))
+    return fail(MOE_INVALID_ARG, "bias must be 4-byte aligned");
+  p->bias = bias;
+  return MOE_OK;
+}
+
+size_t moe_workspace_bytes(moe_plan_t p, int64_t T) {
+  if (!p || T < 0) return 0;
+  return make_layout(p, T).total;
+}
+
+int moe_plan_set_workspace(moe_plan_t p, void* ws, size_t bytes) {
+  if (!p) return fail(MOE_INVALID_ARG, "null plan");
+  if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(MOE_INVALID_ARG, "workspace must be 256-byte aligned");
+  p->ws = static_cast<char*>(ws);
+  p->ws_bytes = ws ? bytes : 0;
+  p->last_T = -1;
+  if (ws) {
+    cudaError_t e = cudaMemset(ws, 0, 256);   // device status word
+    if (e != cudaSuccess) return fail(MOE_CUDA_ERROR, "cudaMemset: %s", cudaGetErrorString(e));
+  }
+  return MOE_OK;
+}
+
+int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* W_g,
+                const moe_bf16_t* W1, const moe_bf16_t* W3, const moe_bf16_t* W2,
+                const moe_bf16_t* W1s, const moe_bf16_t* W3s, const moe_bf16_t* W2s,
+                moe_bf16_t* out, void* stream) {
+  if (!p) return fail(MOE_INVALID_ARG, "null plan");
+  if (T < 0) return fail(MOE_INVALID_ARG, "T must be >= 0");
+  if (T == 0) {
+    p->n_launch = 0;
+    p->last_T = 0;
+    return MOE_OK;
+  }
+  if (T * p->top_k > (1LL << 30))
+    return fail(MOE_UNSUPPORTED, "T*top_k = %lld exceeds 2^30 rows", (long long)(T * p->top_k));
+  if (!x || !W_g || !W1 || !W3 || !W2 || !out)
+    return fail(MOE_INVALID_ARG, "x, W_g, W1, W3, W2 and out must be non-null");
+  if ((p->n_shared > 0) != (W1s != nullptr) || (p->n_shared > 0) != (W3s != nullptr) ||
+      (p->n_shared > 0) != (W2s != nullptr))
+    return fail(MOE_INVALID_ARG, "W1s, W3s, W2s must be non-null exactly when n_shared > 0");
+  const void* ptrs[] = {x, W_g, W1, W3, W2, out, W1s, W3s, W2s};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return fail(MOE_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (!p->ws) return fail(MOE_INVALID_ARG, "no workspace set (moe_plan_set_workspace)");
+  const Layout Lw = make_layout(p, T);
+  if (Lw.total > p->ws_bytes)
+    return fail(MOE_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, T=%lld needs %zu",
+                p->ws_bytes, (long long)T, Lw.total);
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != p->device)
+    return fail(MOE_INVALID_ARG, "plan was created on device %d, current device is %d",
+                p->device, dev);
+  if (p->timing && !p->events_made) {
+    for (int i = 0; i <= kMaxKernels; ++i) cudaEventCreate(&p->ev[i]);
+    p->events_made = true;
+  }
+
+  const int d = p->d, f = p->f, nr = p->n_routed, k = p->top_k;
+  const int nsf = p->n_shared * f;
+  const int64_t A = T * k;
+  char* ws = p->ws;
+  int* status = reinterpret_cast<int*>(ws + Lw.status);
+  float* scores = reinterpret_cast<float*>(ws + Lw.scores);
+  int* idx = reinterpret_cast<int*>(ws + Lw.idx);
+  float* gate = reinterpret_cast<float*>(ws + Lw.gate);
+  int* chunk_counts = reinterpret_cast<int*>(ws + Lw.chunk_counts);
+  int* counts = reinterpret_cast<int*>(ws + Lw.counts);
+  int* offsets = reinterpret_cast<int*>(ws + Lw.offsets);
+  int* mtiles = reinterpret_cast<int*>(ws + Lw.mtiles);
+  int* perm_src = reinterpret_cast<int*>(ws + Lw.perm_src);
+  int* inv_pos = reinterpret_cast<int*>(ws + Lw.inv_pos);
+  void* xperm = ws + Lw.xperm;
+  void* hidden = ws + Lw.hidden;
+  void* yrouted = ws + Lw.yrouted;
+  void* hshared = ws + Lw.hshared;
+  float* yshared = p->n_shared > 0 ? reinterpret_cast<float*>(ws + Lw.yshared) : nullptr;
+
+  CUtensorMap mX, mWg, mXp, mW1, mW3, mH, mW2, mW1s, mW3s, mHs, mW2s;
+  bool ok = make_map(&mX, x, 0, T, d) && make_map(&mWg, W_g, 1, nr, d) &&
+            make_map(&mXp, xperm, 0, A, d) && make_map(&mW1, W1, nr, f, d) &&
+            make_map(&mW3, W3, nr, f, d) && make_map(&mH, hidden, 0, A, f) &&
+            make_map(&mW2, W2, nr, d, f);
+  if (ok && p->n_shared > 0)
+    ok = make_map(&mW1s, W1s, 1, nsf, d) && make_map(&mW3s, W3s, 1, nsf, d) &&
+         make_map(&mHs, hshared, 0, T, nsf) && make_map(&mW2s, W2s, 1, d, nsf);
+  if (!ok) return fail(MOE_CUDA_ERROR, "cuTensorMapEncodeTiled rejected a tensor map");
+
+  cudaGetLastError();  // clear any stale error so launch checks are precise
+  p->n_launch = 0;
+  p->last_T = T;
+  Launcher L{p, static_cast<cudaStream_t>(stream)};
+
+  // 1. router scores s = x W_g^T (fp32), dense over T rows
+  {
+    moe::GemmParams g{};
+    g.dense_rows = static_cast<int>(T);
+    g.K = d;
+    g.N = nr;
+    g.n_tiles = (nr + 255) / 256;
+    g.out = scores;
+    g.ldo = Lw.lds;
+    g.status = status;
+    const int tiles = static_cast<int>((T + 127) / 128) * g.n_tiles;
+    if (!launch_gemm<moe::kEpiF32>(L, "router_gemm", mX, mWg, mWg, g, tiles)) return L.status;
+  }
+  // 2. softmax + top-k + gates + per-chunk histogram
+  {
+    const size_t smem = size_t(nr) * 4;
+    const int npl = (nr + 31) / 32;
+    L.mark("route_topk");
+#define MOE_TOPK_CASE(N)                                                                     \
+  moe::route_topk_kernel<N><<<Lw.n_chunks, moe::kRouteThreads, smem, L.st>>>(               \
+      scores, Lw.lds, p->bias, static_cast<int>(T), nr, k, p->renorm, Lw.tpc, Lw.n_chunks, \
+      idx, gate, chunk_counts)
+    if (npl <= 1) MOE_TOPK_CASE(1);
+    else if (npl <= 2) MOE_TOPK_CASE(2);
+    else if (npl <= 4) MOE_TOPK_CASE(4);
+    else if (npl <= 8) MOE_TOPK_CASE(8);
+    else if (npl <= 16) MOE_TOPK_CASE(16);
+    else MOE_TOPK_CASE(32);
+#undef MOE_TOPK_CASE
+    if (!L.check("route_topk")) return L.status;
+  }
+  // 3. per-expert prefix over chunks, offsets, m-tile prefix
+  L.mark("route_scan");
+  moe::route_scan_kernel<<<1, 1024, 0, L.st>>>(chunk_counts, Lw.n_chunks, nr, counts, offsets,
+                                               mtiles, moe::kBM);
+  if (!L.check("route_scan")) return L.status;
+  // 4. stable permutation + 16-byte row copies into the grouped batch
+  {
+    const size_t smem = size_t(nr) * 4 + size_t(Lw.tpc) * k * 4;
+    L.mark("route_scatter");
+    moe::route_scatter_kernel<<<Lw.n_chunks, moe::kRouteThreads, smem, L.st>>>(
+        idx, chunk_counts, offsets, static_cast<int>(T), k, nr, Lw.tpc, Lw.n_chunks,
+        reinterpret_cast<const uint4*>(x), d / 8, reinterpret_cast<uint4*>(xperm), perm_src,
+        inv_pos);
+    if (!L.check("route_scatter")) return L.status;
+  }
+  const int max_mtiles = static_cast<int>((A + 127) / 128 + (A < nr ? A : nr));
+  // 5. grouped gate/up GEMM with the SiLU(gate) * up epilogue
+  {
+    moe::GemmParams g{};
+    g.group_offsets = offsets;
+    g.group_mtiles = mtiles;
+    g.num_groups = nr;
+    g.K = d;
+    g.N = f;
+    g.n_tiles = (f + 127) / 128;
+    g.out = hidden;
+    g.ldo = f;
+    g.status = status;
+    if (!launch_gemm<moe::kEpiSwiGLU>(L, "grouped_gate_up", mXp, mW1, mW3, g,
+                                      max_mtiles * g.n_tiles))
+      return L.status;
+  }
+  // 6. grouped down GEMM
+  {
+    moe::GemmParams g{};
+    g.group_offsets = offsets;
+    g.group_mtiles = mtiles;
+    g.num_groups = nr;
+    g.K = f;
+    g.N = d;
+    g.n_tiles = (d + 255) / 256;
+    g.out = yrouted;
+    g.ldo = d;
+    g.status = status;
+    if (!launch_gemm<moe::kEpiBF16>(L, "grouped_down", mH, mW2, mW2, g, max_mtiles * g.n_tiles))
+      return L.status;
+  }
+  // 7. shared SwiGLU over all T rows (coefficient 1, outside the routing)
+  if (p->n_shared > 0) {
+    const int mt = static_cast<int>((T + 127) / 128);
+    moe::GemmParams g{};
+    g.dense_rows = static_cast<int>(T);
+    g.K = d;
+    g.N = nsf;
+    g.n_tiles = (nsf + 127) / 128;
+    g.out = hshared;
+    g.ldo = nsf;
+    g.status = status;
+    if (!launch_gemm<moe::kEpiSwiGLU>(L, "shared_gate_up", mX, mW1s, mW3s, g, mt * g.n_tiles))
+      return L.status;
+    moe::GemmParams h{};
+    h.dense_rows = static_cast<int>(T);
+    h.K = nsf;
+    h.N = d;
+    h.n_tiles = (d + 255) / 256;
+    h.out = yshared;
+    h.ldo = d;
+    h.status = status;
+    if (!launch_gemm<moe::kEpiF32>(L, "shared_down", mHs, mW2s, mW2s, h, mt * h.n_tiles))
+      return L.status;
+  }
+  // 8. weighted combine + shared add, one bf16 rounding
+  L.mark("combine");
+  moe::combine_kernel<<<static_cast<unsigned>(T), moe::kCombineThreads, 0, L.st>>>(
+      reinterpret_cast<const uint4*>(yrouted), yshared, inv_pos, gate, k, d / 8,
+      reinterpret_cast<uint4*>(out));
+  if (!L.check("combine")) return L.status;
+  L.finish();
+  return MOE_OK;
+}
+
+int moe_get_routing(moe_plan_t p, int64_t T, int32_t* idx, float* w, int32_t* counts,
+                    int32_t* offsets, void* stream) {
+  if (!p) return fail(MOE_INVALID_ARG, "null plan");
+  if (T != p->last_T || T < 0) return fail(MOE_INVALID_ARG, "T does not match the last forward");
+  if (T == 0) return MOE_OK;
+  const Layout Lw = make_layout(p, T);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t A = size_t(T) * p->top_k;
+  cudaError_t e = cudaSuccess;
+  if (idx && e == cudaSuccess)
+    e = cudaMemcpyAsync(idx, p->ws + Lw.idx, A * 4, cudaMemcpyDeviceToDevice, st);
+  if (w && e == cudaSuccess)
+    e = cudaMemcpyAsync(w, p->ws + Lw.gate, A * 4, cudaMemcpyDeviceToDevice, st);
+  if (counts && e == cudaSuccess)
+    e = cudaMemcpyAsync(counts, p->ws + Lw.counts, size_t(p->n_routed) * 4,
+                        cudaMemcpyDeviceToDevice, st);
+  if (offsets && e == cudaSuccess)
+    e = cudaMemcpyAsync(offsets, p->ws + Lw.offsets, size_t(p->n_routed + 1) * 4,
+                        cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return fail(MOE_CUDA_ERROR, "cudaMemcpyAsync: %s", cudaGetErrorString(e));
+  return MOE_OK;
+}
+
+int moe_get_permutation(moe_plan_t p, int64_t T, int32_t* perm_src, int32_t* inv_pos,
+                        void* stream) {
+  if (!p) return fail(MOE_INVALID_ARG, "null plan");
+  if (T != p->last_T || T < 0) return fail(MOE_INVALID_ARG, "T does not match the last forward");
+  if (T == 0) return MOE_OK;
+  const Layout Lw = make_layout(p, T);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t A = size_t(T) * p->top_k;
+  cudaError_t e = cudaSuccess;
+  if (perm_src)
+    e = cudaMemcpyAsync(perm_src, p->ws + Lw.perm_src, A * 4, cudaMemcpyDeviceToDevice, st);
+  if (inv_pos && e == cudaSuccess)
+    e = cudaMemcpyAsync(inv_pos, p->ws + Lw.inv_pos, A * 4, cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return fail(MOE_CUDA_ERROR, "cudaMemcpyAsync: %s", cudaGetErrorString(e));
+  return MOE_OK;
+}
+
+int moe_plan_device_status(moe_plan_t p) {
+  if (!p) return fail(MOE_INVALID_ARG, "null plan");
+  if (!p->ws) return MOE_OK;
+  int v = 0;
+  cudaError_t e = cudaMemcpy(&v, p->ws, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(p->ws, 0, sizeof(int));
+  if (e != cudaSuccess) return fail(MOE_CUDA_ERROR, "device status read: %s", cudaGetErrorString(e));
+  if (v != MOE_OK) return fail(v, "a kernel gave up a bounded wait (device status %d)", v);
+  return MOE_OK;
+}
+
+int moe_plan_enable_timing(moe_plan_t p, int enable) {
+  if (!p) return fail(MOE_INVALID_ARG, "null plan");
+  p->timing = enable != 0;
+  return MOE_OK;
+}
+
+int moe_plan_kernel_times(moe_plan_t p, float* ms, int cap) {
+  if (!p) return -fail(MOE_INVALID_ARG, "null plan");
+  if (!p->timing || !p->events_made) return -fail(MOE_INVALID_ARG, "timing is not enabled");
+  const int n = p->n_launch < kMaxKernels ? p->n_launch : kMaxKernels;
+  if (n == 0) return 0;
+  cudaError_t e = cudaEventSynchronize(p->ev[n]);
+  if (e != cudaSuccess) return -fail(MOE_CUDA_ERROR, "event sync: %s", cudaGetErrorString(e));
+  for (int i = 0; i < n && i < cap; ++i) {
+    float t = 0.0f;
+    e = cudaEventElapsedTime(&t, p->ev[i], p->ev[i + 1]);
+    if (e != cudaSuccess) return -fail(MOE_CUDA_ERROR, "event time: %s", cudaGetErrorString(e));
+    ms[i] = t;
+  }
+  return n;
+}
+
+const char* moe_plan_kernel_name(moe_plan_t p, int i) {
+  if (!p || i < 0 || i >= p->n_launch || i >= kMaxKernels) return nullptr;
+  return p->names[i];
+}
+
+int moe_plan_last_launch_count(moe_plan_t p) { return p ? p->n_launch : 0; }
+
+void moe_plan_destroy(moe_plan_t p) {
+  if (!p) return;
+  if (p->events_made)
+    for (int i = 0; i <= kMaxKernels; ++i) cudaEventDestroy(p->ev[i]);
+  delete p;
+}
+
+const char* moe_strerror(int s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_INVALID_CONFIG: return "invalid expert configuration";
+    case MOE_INVALID_ARG: return "invalid argument";
+    case MOE_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MOE_CUDA_ERROR: return "CUDA error";
+    case MOE_UNSUPPORTED: return "unsupported shape";
+    case MOE_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+    default: return "unknown status";
+  }
+}
+
+const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

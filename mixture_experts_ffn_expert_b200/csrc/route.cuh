@@ -1,0 +1,266 @@
+// route.cuh - routing and combine kernels of the MoE layer (CUDA cores,
+// HBM/latency-bound work around the tensor-core GEMMs).
+//
+//  route_topk     softmax over the N_r router scores of a token, top-k with
+//                 ties to the lower expert index, raw or renormalised gates
+//                 ("What is an "expert," really?", glossary: router / gate,
+//                 top-k, softmax; panel 2), and a per-chunk expert histogram.
+//  route_scan     per-expert prefix over chunks, exclusive scan over experts
+//                 (offsets) and the prefix of 128-row m-tiles the grouped GEMM
+//                 scheduler walks.
+//  route_scatter  stable (token, slot) order inside each expert group; writes
+//                 the permutation and copies each token row to its k grouped
+//                 rows with 16-byte vectors.
+//  combine        out[t] = shared[t] + sum_j g[t,j] * Y[inv_pos[t,j]] in fp32,
+//                 one bf16 rounding ("Shared Expert (DeepSeek-V3)", eq. (12)
+//                 without the residual; shared term coefficient 1).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kRouteThreads = 256;             // 8 warps
+constexpr int kMaxTopK = 32;
+constexpr int kMaxRouted = 1024;
+
+// One warp per token; block = one chunk of `tpc` consecutive tokens.
+// NPL = router scores held per lane (N_r <= 32 * NPL).
+template <int NPL>
+__global__ void __launch_bounds__(kRouteThreads)
+    route_topk_kernel(const float* __restrict__ scores, int lds, const float* __restrict__ bias,
+                      int T, int n_routed, int top_k, int renorm, int tpc, int n_chunks,
+                      int* __restrict__ idx, float* __restrict__ gate,
+                      int* __restrict__ chunk_counts) {
+  extern __shared__ int s_hist[];               // [n_routed]
+  for (int e = threadIdx.x; e < n_routed; e += blockDim.x) s_hist[e] = 0;
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x;
+  const int t_begin = chunk * tpc;
+  const int t_end = min(T, t_begin + tpc);
+  for (int t = t_begin + warp; t < t_end; t += kRouteThreads / 32) {
+    const float* row = scores + static_cast<long long>(t) * lds;
+    float v[NPL];
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const int e = lane + 32 * i;
+      v[i] = -INFINITY;
+      if (e < n_routed) v[i] = row[e] + (bias ? bias[e] : 0.0f);
+      m = fmaxf(m, v[i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float sum = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+      if (lane + 32 * i < n_routed) sum += expf(v[i] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+
+    uint32_t taken = 0;
+    float sel_sum = 0.0f, my_p = 0.0f;
+    int my_e = -1;
+    for (int j = 0; j < top_k; ++j) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;     // ascending within the lane: '>' keeps the lower index
+        if (e < n_routed && !((taken >> i) & 1u) && (v[i] > bv || be == 0x7fffffff)) {
+          bv = v[i];
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+      }
+      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      const float p = expf(bv - m) / sum;
+      sel_sum += p;
+      if (lane == j) { my_p = p; my_e = be; }
+    }
+    if (lane < top_k) {
+      const long long o = static_cast<long long>(t) * top_k + lane;
+      idx[o] = my_e;
+      gate[o] = renorm ? my_p / sel_sum : my_p;
+      atomicAdd(&s_hist[my_e], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n_routed; e += blockDim.x)
+    chunk_counts[static_cast<long long>(e) * n_chunks + chunk] = s_hist[e];
+}
+
+// Single block of 1024 threads. chunk_counts [N_r][n_chunks] is turned in place
+// into the exclusive prefix over chunks of each expert.
+__global__ void __launch_bounds__(1024)
+    route_scan_kernel(int* __restrict__ chunk_counts, int n_chunks, int n_routed,
+                      int* __restrict__ counts, int* __restrict__ offsets,
+                      int* __restrict__ mtiles, int tile_rows) {
+  __shared__ int s_cnt[kMaxRouted];
+  __shared__ int s_wsum[32], s_wmt[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = warp; e < n_routed; e += 32) {
+    int* row = chunk_counts + static_cast<long long>(e) * n_chunks;
+    int running = 0;
+    for (int c0 = 0; c0 < n_chunks; c0 += 32) {
+      const int c = c0 + lane;
+      const int v = c < n_chunks ? row[c] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+      }
+      if (c < n_chunks) row[c] = running + incl - v;
+      running += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_cnt[e] = running;
+  }
+  __syncthreads();
+  const int e = threadIdx.x;
+  const int c = e < n_routed ? s_cnt[e] : 0;
+  const int mt = (c + tile_rows - 1) / tile_rows;
+  int ic = c, im = mt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int nc = __shfl_up_sync(0xffffffffu, ic, o);
+    const int nm = __shfl_up_sync(0xffffffffu, im, o);
+    if (lane >= o) { ic += nc; im += nm; }
+  }
+  if (lane == 31) { s_wsum[warp] = ic; s_wmt[warp] = im; }
+  __syncthreads();
+  if (warp == 0) {
+    int a = s_wsum[lane], b = s_wmt[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int na = __shfl_up_sync(0xffffffffu, a, o);
+      const int nb = __shfl_up_sync(0xffffffffu, b, o);
+      if (lane >= o) { a += na; b += nb; }
+    }
+    s_wsum[lane] = a - s_wsum[lane];     // exclusive prefix of warp totals
+    s_wmt[lane] = b - s_wmt[lane];
+  }
+  __syncthreads();
+  const int ex_c = s_wsum[warp] + ic - c;
+  const int ex_m = s_wmt[warp] + im - mt;
+  if (e < n_routed) {
+    counts[e] = c;
+    offsets[e] = ex_c;
+    mtiles[e] = ex_m;
+  }
+  if (e == n_routed - 1) {
+    offsets[n_routed] = ex_c + c;
+    mtiles[n_routed] = ex_m + mt;
+  }
+}
+
+// Block = one chunk. Warp 0 ranks the chunk's (token, slot) entries in order
+// with match-any, so rows inside an expert group follow ascending (t, j); then
+// every warp copies token rows (d_vec 16-byte vectors each) to their k rows.
+__global__ void __launch_bounds__(kRouteThreads)
+    route_scatter_kernel(const int* __restrict__ idx, const int* __restrict__ chunk_base,
+                         const int* __restrict__ offsets, int T, int top_k, int n_routed,
+                         int tpc, int n_chunks, const uint4* __restrict__ x, int d_vec,
+                         uint4* __restrict__ xperm, int* __restrict__ perm_src,
+                         int* __restrict__ inv_pos) {
+  extern __shared__ int smem_i[];
+  int* s_run = smem_i;                  // [n_routed]
+  int* s_pos = smem_i + n_routed;       // [tpc * top_k]
+  for (int e = threadIdx.x; e < n_routed; e += blockDim.x) s_run[e] = 0;
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x;
+  const int t0 = chunk * tpc;
+  const int ntok = min(tpc, T - t0);
+  const int n_ent = ntok * top_k;
+  const long long ebase = static_cast<long long>(t0) * top_k;
+  if (warp == 0) {
+    for (int b = 0; b < n_ent; b += 32) {
+      const int i = b + lane;
+      const bool valid = i < n_ent;
+      const int e = valid ? idx[ebase + i] : -1;
+      const uint32_t same = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(same & ((1u << lane) - 1u));
+      if (valid)
+        s_pos[i] = offsets[e] + chunk_base[static_cast<long long>(e) * n_chunks + chunk] +
+                   s_run[e] + rank;
+      __syncwarp();
+      if (valid && lane == 31 - __clz(same)) s_run[e] += __popc(same);
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_ent; i += blockDim.x) {
+    const int pos = s_pos[i];
+    inv_pos[ebase + i] = pos;
+    perm_src[pos] = t0 + i / top_k;
+  }
+  for (int tl = warp; tl < ntok; tl += kRouteThreads / 32) {
+    const uint4* src = x + static_cast<long long>(t0 + tl) * d_vec;
+    const int* pos = s_pos + tl * top_k;
+    for (int v = lane; v < d_vec; v += 32) {
+      const uint4 val = src[v];
+      for (int j = 0; j < top_k; ++j) xperm[static_cast<long long>(pos[j]) * d_vec + v] = val;
+    }
+  }
+}
+
+__device__ __forceinline__ void bf16x8_fma(float (&acc)[8], uint4 v, float w) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    acc[2 * q] = fmaf(w, __uint_as_float(u[q] << 16), acc[2 * q]);
+    acc[2 * q + 1] = fmaf(w, __uint_as_float(u[q] & 0xFFFF0000u), acc[2 * q + 1]);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+constexpr int kCombineThreads = 128;
+
+// Block = one token. shared (fp32, (T, d)) may be null when N_s = 0.
+__global__ void __launch_bounds__(kCombineThreads)
+    combine_kernel(const uint4* __restrict__ Y, const float* __restrict__ shared,
+                   const int* __restrict__ inv_pos, const float* __restrict__ gate, int top_k,
+                   int d_vec, uint4* __restrict__ out) {
+  __shared__ int s_pos[kMaxTopK];
+  __shared__ float s_w[kMaxTopK];
+  const long long t = blockIdx.x;
+  if (threadIdx.x < top_k) {
+    s_pos[threadIdx.x] = inv_pos[t * top_k + threadIdx.x];
+    s_w[threadIdx.x] = gate[t * top_k + threadIdx.x];
+  }
+  __syncthreads();
+  for (int v = threadIdx.x; v < d_vec; v += blockDim.x) {
+    float acc[8];
+    if (shared) {
+      const float4* s = reinterpret_cast<const float4*>(shared + (t * d_vec + v) * 8);
+      const float4 a = s[0], b = s[1];
+      acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
+      acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+    }
+    for (int j = 0; j < top_k; ++j)
+      bf16x8_fma(acc, Y[static_cast<long long>(s_pos[j]) * d_vec + v], s_w[j]);
+    out[t * d_vec + v] = make_uint4(pack2_bf16(acc[0], acc[1]), pack2_bf16(acc[2], acc[3]),
+                                    pack2_bf16(acc[4], acc[5]), pack2_bf16(acc[6], acc[7]));
+  }
+}
+
+}  // namespace moe

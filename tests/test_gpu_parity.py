@@ -1,0 +1,124 @@
+"""GPU parity: the CUDA layer through the C ABI against the fp64 oracle.
+
+Small layers are compared on every output element; the five page-shaped
+workloads at full size are compared on every token's routing and permutation
+and on a seeded sample of output rows (tokens are independent given the
+routing, so a sampled row is checked exactly).
+"""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_ffn_expert_b200.inputs import LayerShape, WORKLOADS, make_layer_inputs
+
+from parity import full_parity
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    # name, T, d, f, N_r, k, N_s, renorm, bias
+    ("one_token", 1, 128, 64, 31, 7, 1, True, "none"),
+    ("three_tokens", 3, 128, 64, 8, 2, 0, True, "none"),
+    ("ragged_17", 17, 256, 128, 16, 4, 1, False, "normal_var0.5"),
+    ("k_equals_n", 40, 128, 64, 12, 12, 0, False, "none"),
+    ("top1_single_expert", 50, 128, 96, 1, 1, 0, True, "none"),
+    ("top1_plus_shared", 70, 128, 64, 16, 1, 1, True, "none"),
+    ("two_shared_raw", 129, 192, 64, 10, 3, 2, False, "none"),
+    ("ragged_tiles", 600, 384, 320, 6, 2, 1, True, "none"),        # several m/n tiles + tails
+    ("k_tail_not_64", 77, 136, 72, 9, 3, 1, True, "none"),         # K and N not multiples of 64
+    ("wide_router", 96, 256, 64, 512, 10, 1, True, "zipf1.1"),      # 16 scores per lane, 2 n-tiles
+    ("max_router", 64, 128, 32, 1024, 32, 0, True, "none"),         # N_r and k at their limits
+    ("skewed_groups", 1000, 256, 128, 64, 6, 1, True, "zipf1.1"),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_small_layers_all_outputs(case):
+    name, T, d, f, n, k, ns, renorm, bias = case
+    shape = LayerShape(name, T, d, f, n, k, ns, renorm, bias)
+    inp = make_layer_inputs(shape, seed=1, device="cuda")
+    res = full_parity(inp, shape)
+    assert res["near_ties"] <= max(2, T * k // 20)
+
+
+def test_tiny_workload_all_outputs():
+    shape = WORKLOADS["tiny_t256_d128_f64_e31k7_s1"]
+    inp = make_layer_inputs(shape, seed=0, device="cuda")
+    full_parity(inp, shape)
+
+
+@pytest.mark.parametrize("name,n_tokens", [
+    ("coarse_t4096_d4096_f14336_e8k2_s0", 48),
+    ("dsmoe_small_t8192_d2048_f1408_e64k6_s2", 96),
+    ("dsv3_prefill_t4096_d7168_f2048_e256k8_s1", 24),
+    ("decode_t128_d2048_f512_e512k10_s1", 128),
+])
+def test_full_size_workloads(name, n_tokens):
+    shape = WORKLOADS[name]
+    inp = make_layer_inputs(shape, seed=0, device="cuda")
+    rng = np.random.default_rng(1234)
+    tokens = np.sort(rng.choice(shape.T, size=min(n_tokens, shape.T), replace=False))
+    res = full_parity(inp, shape, tokens=tokens)
+    print(f"{name}: near ties {res['near_ties']}, rel-L2 {res['rel_l2']:.2e}, "
+          f"max-abs {res['max_abs']:.2e} of max|ref| {res['max_ref']:.2e}")
+    del inp
+    torch.cuda.empty_cache()
+
+
+def test_zero_tokens_is_a_noop():
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    shape = WORKLOADS["tiny_t256_d128_f64_e31k7_s1"]
+    inp = make_layer_inputs(shape, seed=0, device="cuda", T=0)
+    layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared, True,
+                     inp, device="cuda")
+    out = layer(inp["x"])
+    torch.cuda.synchronize()
+    assert out.shape == (0, shape.d)
+    assert layer.plan.last_launch_count() == 0
+
+
+def test_repeated_forwards_are_deterministic():
+    shape = LayerShape("det", 300, 256, 128, 16, 4, 1, True, "none")
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    inp = make_layer_inputs(shape, seed=3, device="cuda")
+    layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared, True,
+                     inp, device="cuda")
+    a = layer(inp["x"]).clone()
+    b = layer(inp["x"]).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_error_paths_on_device():
+    from mixture_experts_ffn_expert_b200.binding import MoEError, Plan
+    shape = WORKLOADS["tiny_t256_d128_f64_e31k7_s1"]
+    inp = make_layer_inputs(shape, seed=0, device="cuda")
+    plan = Plan(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared, True)
+    T = shape.T
+    need = plan.workspace_bytes(T)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(inp["x"])
+    p = {k: (v.data_ptr() if v is not None else None) for k, v in inp.items()}
+    args = (p["x"], p["W_g"], p["W1"], p["W3"], p["W2"], p["W1s"], p["W3s"], p["W2s"],
+            out.data_ptr())
+    with pytest.raises(MoEError) as e:          # no workspace yet
+        plan.forward(T, *args)
+    assert e.value.status == 2
+    plan.set_workspace(ws.data_ptr(), need - 256)
+    with pytest.raises(MoEError) as e:
+        plan.forward(T, *args)
+    assert e.value.status == 3
+    plan.set_workspace(ws.data_ptr(), need)
+    with pytest.raises(MoEError) as e:          # shared weights missing while N_s = 1
+        plan.forward(T, *args[:5], None, None, None, args[8])
+    assert e.value.status == 2
+    with pytest.raises(MoEError) as e:          # misaligned pointer
+        plan.forward(T, args[0] + 2, *args[1:])
+    assert e.value.status == 2
+    with pytest.raises(MoEError) as e:
+        plan.forward(-1, *args)
+    assert e.value.status == 2
+    plan.forward(T, *args)
+    torch.cuda.synchronize()
+    assert plan.device_status() == 0
+    plan.close()
