@@ -1,0 +1,447 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE feed-forward layer forward pass on B200.
+
+One step = one full forward of the layer (router scores, softmax + top-k,
+histogram/scan/permutation, grouped gate/up + SiLU GEMM, grouped down GEMM,
+shared SwiGLU, weighted combine) over one batch of T synthetic tokens, with
+every input already resident in HBM. Prints ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the fp64 CPU oracle, rank 0 only
+
+Multi-GPU (torchrun): every rank runs an independent replica of the workload
+on its own GPU (the layer has no exchange step on one node); the timed region
+is bracketed by a barrier and a device synchronise, its device time is the
+max over ranks, and `value` counts the tokens of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "coarse_t4096_d4096_f14336_e8k2_s0"
+METRIC = "MoE-layer tokens/s at 1 B200; TFLOP/s vs bf16 peak (HBM GB/s when weight-bound)"
+L2_FLUSH_BYTES = 256 << 20          # twice the 126 MB L2
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--tokens", type=int, default=None, help="override T (profiling runs)")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the oracle timing (profiling runs)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU seconds of the oracle sample")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------- peaks, profiles
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            m = json.load(fh)
+        return {k: float(m[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("gemm_sm100.cuh", "ptx_sm100.cuh"):
+        with open(os.path.join(ROOT, "mixture_experts_ffn_expert_b200", "csrc", name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, or None when there is
+    none or the kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.txt")
+    if not os.path.exists(path):
+        return None
+    text = open(path, encoding="utf-8").read()
+    m_t = re.search(r"^traffic_bytes_per_launch:\s*([0-9.eE+]+)", text, re.M)
+    m_h = re.search(r"^kernel_source_sha256_16:\s*([0-9a-f]+)", text, re.M)
+    if not m_t or not m_h or m_h.group(1) != kernel_source_hash():
+        return None
+    return float(m_t.group(1))
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.idx, self.period = device_index, period_s
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            props = torch.cuda.get_device_properties(device_index)
+            try:     # CUDA and NVML number devices differently under CUDA_VISIBLE_DEVICES
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId_v2(bus)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except AttributeError:
+            bits = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        for b, name in self.REASONS.items():
+            if bits & b and name != "gpu_idle":
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def start(self):
+        if self.ok:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread:
+            self._stop.set()
+            self._thread.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples), "source": "nvml" if self.ok else "unavailable"}
+
+
+# ----------------------------------------------------------------- work accounting
+def kernel_work(name, shape, T, touched):
+    """(flops, bytes) the kernel cannot avoid: its inputs, outputs and weights."""
+    d, f, n, k = shape.d, shape.f, shape.n_routed, shape.top_k
+    A, nsf = T * k, shape.n_shared * shape.f
+    table = {
+        "router_gemm": (2 * T * d * n, 2 * n * d + 2 * T * d + 4 * T * n),
+        "route_topk": (0, 4 * T * n + 8 * A),
+        "route_scan": (0, 0),
+        "route_scatter": (0, 2 * T * d + 2 * A * d + 12 * A),
+        "grouped_gate_up": (4 * A * d * f, touched * 4 * d * f + 2 * A * d + 2 * A * f),
+        "grouped_down": (2 * A * d * f, touched * 2 * d * f + 2 * A * f + 2 * A * d),
+        "shared_gate_up": (4 * T * d * nsf, 4 * nsf * d + 2 * T * d + 2 * T * nsf),
+        "shared_down": (2 * T * d * nsf, 2 * nsf * d + 2 * T * nsf + 4 * T * d),
+        "combine": (0, 2 * A * d + (4 * T * d if nsf else 0) + 2 * T * d + 8 * A),
+    }
+    return table.get(name, (0, 0))
+
+
+# ----------------------------------------------------------------- oracle (CPU)
+def oracle_sample_run(inp, shape, tokens, expert_cache):
+    """Run the fp64 oracle on the rows `tokens` of x; returns seconds."""
+    import numpy as np
+    import torch
+    from oracle import moe_layer
+
+    x = inp["x"][torch.as_tensor(tokens)].to(torch.float64).numpy()
+    wg = inp["W_g"].to(torch.float64).numpy()
+    bias = None if inp["bias"] is None else inp["bias"].to(torch.float64).numpy()
+
+    def expert(e):
+        w1, w3, w2 = expert_cache(e)
+        return (w1.to(torch.float64).numpy(), w3.to(torch.float64).numpy(),
+                w2.to(torch.float64).numpy())
+
+    shared = None
+    if shape.n_shared > 0:
+        shared = tuple(inp[k].to(torch.float64).numpy() for k in ("W1s", "W3s", "W2s"))
+    t0 = time.perf_counter()
+    r = moe_layer(x, wg, bias, expert, shared, shape.top_k, shape.renorm)
+    dt = time.perf_counter() - t0
+    assert np.all(np.isfinite(r["out"]))
+    return dt
+
+
+def host_copy_of_inputs(inp_dev):
+    """bf16 host copies (D2H once, outside any timing)."""
+    return {k: (None if v is None else v.cpu()) for k, v in inp_dev.items()}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def timed_oracle(inp_host, shape, target_s, max_tokens=None):
+    """Grow a seeded token sample until one oracle run costs about target_s."""
+    import numpy as np
+    rng = np.random.default_rng(0)
+    T = shape.T if max_tokens is None else max_tokens
+    order = rng.permutation(T)
+    cache = lambda e: (inp_host["W1"][e], inp_host["W3"][e], inp_host["W2"][e])  # noqa: E731
+    n = min(8, T)
+    while True:
+        dt = oracle_sample_run(inp_host, shape, np.sort(order[:n]), cache)
+        if dt >= 0.6 * target_s or n >= T:
+            return n, dt
+        n = min(T, max(n + 1, int(n * min(8.0, max(2.0, target_s / max(dt, 1e-3))))))
+
+
+# ----------------------------------------------------------------- arms
+def run_reference(args, info):
+    """The fp64 oracle as it stands, timed on this machine's host cores (rank 0 only)."""
+    import torch
+    from mixture_experts_ffn_expert_b200.inputs import WORKLOADS, make_layer_inputs
+
+    if info.rank != 0:
+        return None
+    shape = WORKLOADS[args.workload]
+    if args.tokens:
+        shape = shape.with_tokens(args.tokens)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = host_copy_of_inputs(make_layer_inputs(shape, seed=0, device=dev))
+    # size one step to about (a few minutes) / (steps + warmup)
+    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    n_tok, _ = timed_oracle(inp, shape, per_step)
+    import numpy as np
+    rng = np.random.default_rng(1)
+    cache = lambda e: (inp["W1"][e], inp["W3"][e], inp["W2"][e])  # noqa: E731
+    for _ in range(args.warmup):
+        oracle_sample_run(inp, shape, np.sort(rng.choice(shape.T, n_tok, replace=False)), cache)
+    times = []
+    for _ in range(args.steps):
+        times.append(oracle_sample_run(inp, shape,
+                                       np.sort(rng.choice(shape.T, n_tok, replace=False)), cache))
+    total = sum(times)
+    value = n_tok * args.steps / total
+    cores = cpu_threads()
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(shape, args),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n_tok} seeded tokens of T={shape.T} per step (routing and "
+                                   f"experts for those tokens only)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def workload_config(shape, args):
+    return {"workload": shape.name, "T": shape.T, "d": shape.d, "f": shape.f,
+            "n_routed": shape.n_routed, "top_k": shape.top_k, "n_shared": shape.n_shared,
+            "renorm": shape.renorm, "logit_bias": shape.bias, "seed": 0,
+            "parallelism": f"replicas x{args.gpus}",
+            "l2": "flushed between timed steps (256 MiB write outside the step events); "
+                  "weights also exceed L2"}
+
+
+def run_ours(args, info):
+    import torch
+    from mixture_experts_ffn_expert_b200.inputs import WORKLOADS, make_layer_inputs
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    from mixture_experts_ffn_expert_b200 import replicas
+
+    dev = torch.device("cuda", info.local_rank)
+    torch.cuda.set_device(dev)
+    shape = WORKLOADS[args.workload]
+    if args.tokens:
+        shape = shape.with_tokens(args.tokens)
+    T = shape.T
+    inp = make_layer_inputs(shape, seed=0, device=dev)
+    layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
+                     shape.renorm, inp, bias=inp["bias"], device=dev)
+    x = inp["x"]
+    out = torch.empty_like(x)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(max(args.warmup, 3)):
+        layer(x, out)
+        flush.fill_(1)
+    torch.cuda.synchronize(dev)
+    routing = layer.routing()
+    counts = routing["counts"].cpu()
+    touched = int((counts > 0).sum())
+    launches_per_step = layer.plan.last_launch_count()
+
+    # ---- timed region: device time of K steps, max over ranks
+    layer.plan.enable_timing(True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    ktimes = {}
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    replicas.barrier(info)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    names = None
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        layer(x, out)
+        ev[i][1].record(stream)
+        flush.fill_(1)
+        if names is None:
+            names = layer.plan.kernel_names()
+        if i > 0:     # read the previous step while this one is queued
+            for name, t in zip(names, layer.plan.kernel_times(back=1)):
+                ktimes.setdefault(name, []).append(t)
+    for name, t in zip(names, layer.plan.kernel_times(back=0)):
+        ktimes.setdefault(name, []).append(t)
+    torch.cuda.synchronize(dev)
+    clock_info = clocks.stop()
+    replicas.barrier(info)
+    layer.plan.enable_timing(False)
+    assert layer.device_status() == 0, "a kernel reported a bounded-wait timeout"
+    local_ms = sum(a.elapsed_time(b) for a, b in ev)
+    total_ms = replicas.max_over_ranks(local_ms, info, device=dev)
+    ms_per_step = total_ms / args.steps
+    value = info.world_size * T * args.steps / (total_ms / 1e3)
+
+    # ---- per-kernel times and the dominant kernel's roofline
+    peaks, peak_src = load_peaks()
+    kavg = {k: sum(v) / len(v) for k, v in ktimes.items()}
+    dominant = max(kavg, key=kavg.get)
+    flops, nbytes = kernel_work(dominant, shape, T, touched)
+    t_dom = kavg[dominant] / 1e3
+    t_tensor = flops / (peaks["bf16_tflops_sustained"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    if flops and t_tensor >= t_hbm:
+        achieved, peak, unit, bound = flops / t_dom / 1e12, peaks["bf16_tflops_sustained"], \
+            "TFLOP/s", "tensor"
+    else:
+        achieved, peak, unit, bound = nbytes / t_dom / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
+    roofline = {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+                "frac": round(achieved / peak, 4), "kernel": dominant,
+                "peak_source": f"{peak_src} ({'bf16 sustained' if bound == 'tensor' else 'HBM copy'})",
+                "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": nbytes,
+                "avg_launch_ms": round(kavg[dominant], 4),
+                "traffic": profiled_traffic(dominant, shape.name)}
+    if bound == "tensor":
+        roofline["frac_of_burst_peak"] = round(achieved / peaks["bf16_tflops"], 4)
+    layer_flops = (2 * T * shape.d * shape.n_routed + 6 * T * shape.top_k * shape.d * shape.f
+                   + 6 * T * shape.d * shape.n_shared * shape.f)
+
+    # ---- end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        x_host = x.cpu().pin_memory()
+        out_host = torch.empty_like(x_host).pin_memory()
+        x_dev = torch.empty_like(x)
+        for _ in range(3):
+            x_dev.copy_(x_host, non_blocking=True)
+            layer(x_dev, out)
+            out_host.copy_(out, non_blocking=True)
+        torch.cuda.synchronize(dev)
+        n_e2e = max(3, min(args.steps, 50))
+        eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n_e2e)]
+        replicas.barrier(info)
+        torch.cuda.synchronize(dev)
+        for i in range(n_e2e):
+            eev[i][0].record(stream)
+            x_dev.copy_(x_host, non_blocking=True)
+            layer(x_dev, out)
+            out_host.copy_(out, non_blocking=True)
+            eev[i][1].record(stream)
+            flush.fill_(1)
+        torch.cuda.synchronize(dev)
+        e_ms = replicas.max_over_ranks(sum(a.elapsed_time(b) for a, b in eev), info, device=dev)
+        e2e = {"value": info.world_size * T * n_e2e / (e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+               "d2h_bytes_per_step": out_host.numel() * out_host.element_size(),
+               "steps": n_e2e, "path": "pinned host x -> device, moe_forward, device -> pinned host out"}
+
+    # ---- CPU baseline: the oracle on a bounded sample, rank 0 at N=1 only
+    cpu = None
+    if not args.no_cpu_baseline and info.rank == 0 and info.world_size == 1:
+        inp_host = host_copy_of_inputs(inp)
+        n_tok, dt = timed_oracle(inp_host, shape, args.cpu_seconds)
+        cpu = {"value": n_tok / dt, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"{n_tok} seeded tokens of T={T} (routing and experts for those "
+                         f"tokens), one run of {dt:.1f} s"}
+
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": info.world_size,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; random-init weights scaled 1/sqrt(fan_in))",
+        "config": workload_config(shape, args),
+        "tflops": layer_flops / (ms_per_step / 1e3) / 1e12 * info.world_size,
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clock_info,
+        "kernels_ms": {k: round(v, 4) for k, v in kavg.items()},
+        "routing": {"touched_experts": touched, "max_rows": int(counts.max()),
+                    "median_rows": float(counts.float().median()),
+                    "min_rows": int(counts.min())},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    from mixture_experts_ffn_expert_b200 import replicas
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return 0
+        info = replicas.RankInfo(0, 1, 0, False)
+        res = run_reference(args, info)
+    else:
+        info = replicas.init_from_env("nccl")
+        try:
+            res = run_ours(args, info)
+        finally:
+            replicas.shutdown(info)
+    if res is not None and info.rank == 0:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -124,13 +124,15 @@ int moe_get_permutation(moe_plan_t plan, int64_t T, int32_t* perm_src,
 int moe_plan_device_status(moe_plan_t plan);
 
 /* Timing: when enabled, moe_forward records a CUDA event on its stream before
- * every kernel launch and after the last one. moe_plan_kernel_times waits for
- * the last forward's final event and writes up to `cap` per-kernel durations
- * in milliseconds; it returns how many kernels the last forward launched (or a
- * negative moe_status). moe_plan_kernel_name gives the name of kernel i of the
- * last forward (static string; NULL when out of range). */
+ * every kernel launch and after the last one, into one of 4 event sets used in
+ * turn, so the host can read forward i-1 while forward i is still queued.
+ * moe_plan_kernel_times waits for the final event of the timed forward `back`
+ * steps before the latest one (0 = latest, at most 3) and writes up to `cap`
+ * per-kernel durations in milliseconds; it returns how many kernels that
+ * forward launched, or a negative moe_status. moe_plan_kernel_name gives the
+ * name of kernel i of the last forward (static string; NULL when out of range). */
 int moe_plan_enable_timing(moe_plan_t plan, int enable);
-int moe_plan_kernel_times(moe_plan_t plan, float* ms, int cap);
+int moe_plan_kernel_times(moe_plan_t plan, int back, float* ms, int cap);
 const char* moe_plan_kernel_name(moe_plan_t plan, int i);
 
 /* Number of kernels the last forward of this plan launched. */

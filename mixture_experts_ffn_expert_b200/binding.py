@@ -60,7 +60,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_get_permutation": (_i, [_vp, _i64, _vp, _vp, _vp]),
         "moe_plan_device_status": (_i, [_vp]),
         "moe_plan_enable_timing": (_i, [_vp, _i]),
-        "moe_plan_kernel_times": (_i, [_vp, ctypes.POINTER(ctypes.c_float), _i]),
+        "moe_plan_kernel_times": (_i, [_vp, _i, ctypes.POINTER(ctypes.c_float), _i]),
         "moe_plan_kernel_name": (ctypes.c_char_p, [_vp, _i]),
         "moe_plan_last_launch_count": (_i, [_vp]),
         "moe_plan_destroy": (None, [_vp]),
@@ -127,9 +127,10 @@ class Plan:
     def enable_timing(self, on: bool = True) -> None:
         _check(self.lib, self.lib.moe_plan_enable_timing(self.handle, int(on)))
 
-    def kernel_times(self) -> List[float]:
+    def kernel_times(self, back: int = 0) -> List[float]:
+        """Per-kernel milliseconds of the timed forward `back` steps before the latest."""
         buf = (ctypes.c_float * 16)()
-        n = self.lib.moe_plan_kernel_times(self.handle, buf, 16)
+        n = self.lib.moe_plan_kernel_times(self.handle, back, buf, 16)
         if n < 0:
             _check(self.lib, -n)
         return [float(buf[i]) for i in range(min(n, 16))]

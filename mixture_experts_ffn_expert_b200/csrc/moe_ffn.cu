@@ -36,6 +36,7 @@ int fail(int status, const char* fmt, ...) {
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 constexpr int kMaxKernels = 16;
+constexpr int kTimingRing = 4;   // event sets: forward i records into set i % kTimingRing
 
 struct Layout {
   size_t status, scores, idx, gate, chunk_counts, counts, offsets, mtiles, perm_src, inv_pos;
@@ -57,7 +58,10 @@ struct moe_plan {
   bool timing = false;
   int n_launch = 0;
   const char* names[kMaxKernels] = {};
-  cudaEvent_t ev[kMaxKernels + 1] = {};
+  cudaEvent_t ev[kTimingRing][kMaxKernels + 1] = {};
+  int ring_launches[kTimingRing] = {};
+  long long timed_forwards = 0;     // forwards that recorded events
+  int cur_set = 0;
   bool events_made = false;
 };
 
@@ -140,7 +144,7 @@ struct Launcher {
   void mark(const char* name) {
     if (p->n_launch < kMaxKernels) {
       p->names[p->n_launch] = name;
-      if (p->timing) cudaEventRecord(p->ev[p->n_launch], st);
+      if (p->timing) cudaEventRecord(p->ev[p->cur_set][p->n_launch], st);
     }
     ++p->n_launch;
   }
@@ -153,7 +157,11 @@ struct Launcher {
     return true;
   }
   void finish() {
-    if (p->timing && p->n_launch <= kMaxKernels) cudaEventRecord(p->ev[p->n_launch], st);
+    if (p->timing && p->n_launch <= kMaxKernels) {
+      cudaEventRecord(p->ev[p->cur_set][p->n_launch], st);
+      p->ring_launches[p->cur_set] = p->n_launch;
+      ++p->timed_forwards;
+    }
   }
 };
 
@@ -296,9 +304,11 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     return fail(MOE_INVALID_ARG, "plan was created on device %d, current device is %d",
                 p->device, dev);
   if (p->timing && !p->events_made) {
-    for (int i = 0; i <= kMaxKernels; ++i) cudaEventCreate(&p->ev[i]);
+    for (int r = 0; r < kTimingRing; ++r)
+      for (int i = 0; i <= kMaxKernels; ++i) cudaEventCreate(&p->ev[r][i]);
     p->events_made = true;
   }
+  if (p->timing) p->cur_set = static_cast<int>(p->timed_forwards % kTimingRing);
 
   const int d = p->d, f = p->f, nr = p->n_routed, k = p->top_k;
   const int nsf = p->n_shared * f;
@@ -504,16 +514,19 @@ int moe_plan_enable_timing(moe_plan_t p, int enable) {
   return MOE_OK;
 }
 
-int moe_plan_kernel_times(moe_plan_t p, float* ms, int cap) {
+int moe_plan_kernel_times(moe_plan_t p, int back, float* ms, int cap) {
   if (!p) return -fail(MOE_INVALID_ARG, "null plan");
-  if (!p->timing || !p->events_made) return -fail(MOE_INVALID_ARG, "timing is not enabled");
-  const int n = p->n_launch < kMaxKernels ? p->n_launch : kMaxKernels;
+  if (!p->events_made) return -fail(MOE_INVALID_ARG, "timing is not enabled");
+  if (back < 0 || back >= kTimingRing || back >= p->timed_forwards)
+    return -fail(MOE_INVALID_ARG, "no timed forward %d steps back", back);
+  const int set = static_cast<int>((p->timed_forwards - 1 - back) % kTimingRing);
+  const int n = p->ring_launches[set];
   if (n == 0) return 0;
-  cudaError_t e = cudaEventSynchronize(p->ev[n]);
+  cudaError_t e = cudaEventSynchronize(p->ev[set][n]);
   if (e != cudaSuccess) return -fail(MOE_CUDA_ERROR, "event sync: %s", cudaGetErrorString(e));
   for (int i = 0; i < n && i < cap; ++i) {
     float t = 0.0f;
-    e = cudaEventElapsedTime(&t, p->ev[i], p->ev[i + 1]);
+    e = cudaEventElapsedTime(&t, p->ev[set][i], p->ev[set][i + 1]);
     if (e != cudaSuccess) return -fail(MOE_CUDA_ERROR, "event time: %s", cudaGetErrorString(e));
     ms[i] = t;
   }
@@ -530,7 +543,8 @@ int moe_plan_last_launch_count(moe_plan_t p) { return p ? p->n_launch : 0; }
 void moe_plan_destroy(moe_plan_t p) {
   if (!p) return;
   if (p->events_made)
-    for (int i = 0; i <= kMaxKernels; ++i) cudaEventDestroy(p->ev[i]);
+    for (int r = 0; r < kTimingRing; ++r)
+      for (int i = 0; i <= kMaxKernels; ++i) cudaEventDestroy(p->ev[r][i]);
   delete p;
 }
 
