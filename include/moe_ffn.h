@@ -135,6 +135,29 @@ int moe_plan_enable_timing(moe_plan_t plan, int enable);
 int moe_plan_kernel_times(moe_plan_t plan, int back, float* ms, int cap);
 const char* moe_plan_kernel_name(moe_plan_t plan, int i);
 
+/* Forward for callers that cannot allocate device memory - for instance a
+ * plugin whose host application owns the whole device-memory budget, or a
+ * latency-critical loop where cudaMalloc would synchronise the device. The
+ * pages have no counterpart of this call; it is a deployment convenience.
+ * Same arguments and result as moe_forward, but the scratch the layer needs
+ * lives in one static device array of 32 MiB inside the library (held on
+ * every GPU that loads the library until the process exits) instead of the
+ * plan's workspace; the caller passes only inputs and outputs, and nothing is
+ * allocated by the call. T whose scratch would exceed 32 MiB is rejected with
+ * MOE_WORKSPACE_TOO_SMALL before anything is enqueued (the 512-expert decode
+ * shape d=2048, f=512, N_r=512, k=10, N_s=1 needs about 13 MiB at T=128).
+ * The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture. All calls
+ * share the one array and it keeps the last call's contents: two calls that
+ * overlap on the GPU (different streams, plans or threads) race, so keep them
+ * on one stream. Timing events are not recorded, and moe_get_routing /
+ * moe_get_permutation / moe_plan_device_status do not see these forwards. */
+int moe_forward_noalloc(moe_plan_t plan, int64_t T, const moe_bf16_t* x,
+                        const moe_bf16_t* W_g, const moe_bf16_t* W1,
+                        const moe_bf16_t* W3, const moe_bf16_t* W2,
+                        const moe_bf16_t* W1s, const moe_bf16_t* W3s,
+                        const moe_bf16_t* W2s, moe_bf16_t* out, void* stream);
+
 /* Number of kernels the last forward of this plan launched. */
 int moe_plan_last_launch_count(moe_plan_t plan);
 

@@ -20,7 +20,7 @@ EXPORTED_SYMBOLS = [
     "moe_plan_set_workspace", "moe_forward", "moe_get_routing", "moe_get_permutation",
     "moe_plan_device_status", "moe_plan_enable_timing", "moe_plan_kernel_times",
     "moe_plan_kernel_name", "moe_plan_last_launch_count", "moe_plan_destroy", "moe_strerror",
-    "moe_last_error",
+    "moe_last_error", "moe_forward_noalloc",
 ]
 
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_INVALID_CONFIG", 2: "MOE_INVALID_ARG",
@@ -56,6 +56,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_workspace_bytes": (_sz, [_vp, _i64]),
         "moe_plan_set_workspace": (_i, [_vp, _vp, _sz]),
         "moe_forward": (_i, [_vp, _i64] + [_vp] * 10),
+        "moe_forward_noalloc": (_i, [_vp, _i64] + [_vp] * 10),
         "moe_get_routing": (_i, [_vp, _i64, _vp, _vp, _vp, _vp, _vp]),
         "moe_get_permutation": (_i, [_vp, _i64, _vp, _vp, _vp]),
         "moe_plan_device_status": (_i, [_vp]),

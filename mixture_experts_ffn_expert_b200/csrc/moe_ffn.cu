@@ -540,6 +540,89 @@ const char* moe_plan_kernel_name(moe_plan_t p, int i) {
 
 int moe_plan_last_launch_count(moe_plan_t p) { return p ? p->n_launch : 0; }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Forward without caller-provided scratch.
+//
+// Some callers cannot allocate device memory at all: a plugin inside a host
+// application that owns the whole device-memory budget through its own pool,
+// or a latency-critical loop where cudaMalloc would synchronise the device.
+// For them the layer's scratch lives in one file-scope device array instead
+// of a caller workspace. Every GPU that loads this library holds the array
+// (kNoAllocScratchBytes) until the process exits.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;   // 32 MiB
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the array on the current device. In host code the
+// array's name only stands in for the symbol, so the address is looked up once
+// per device (with that device current) and cached.
+int noalloc_scratch(int dev, void** out) {
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return fail(MOE_UNSUPPORTED, "device %d is beyond the %d devices supported", dev,
+                kNoAllocMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || !ptr)
+      return fail(MOE_CUDA_ERROR, "cudaGetSymbolAddress of the static scratch failed: %s",
+                  cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_forward_noalloc(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* W_g,
+                        const moe_bf16_t* W1, const moe_bf16_t* W3, const moe_bf16_t* W2,
+                        const moe_bf16_t* W1s, const moe_bf16_t* W3s, const moe_bf16_t* W2s,
+                        moe_bf16_t* out, void* stream) {
+  if (!p) return fail(MOE_INVALID_ARG, "null plan");
+  if (T < 0) return fail(MOE_INVALID_ARG, "T must be >= 0");
+  const size_t need = make_layout(p, T).total;
+  if (need > kNoAllocScratchBytes)
+    return fail(MOE_WORKSPACE_TOO_SMALL,
+                "T=%lld needs %zu bytes of scratch; the static scratch of moe_forward_noalloc "
+                "holds %zu bytes (use moe_forward with a caller workspace)",
+                (long long)T, need, kNoAllocScratchBytes);
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != p->device)
+    return fail(MOE_INVALID_ARG, "plan was created on device %d, current device is %d",
+                p->device, dev);
+  void* scratch = nullptr;
+  int rc = noalloc_scratch(dev, &scratch);
+  if (rc != MOE_OK) return rc;
+  // The status word is the only scratch that must start at zero.
+  cudaError_t e = cudaMemsetAsync(scratch, 0, 256, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(MOE_CUDA_ERROR, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+  // Run the regular forward on the static scratch, with timing off so that no
+  // events are created, then give the plan its own workspace back.
+  char* saved_ws = p->ws;
+  const size_t saved_bytes = p->ws_bytes;
+  const bool saved_timing = p->timing;
+  p->ws = static_cast<char*>(scratch);
+  p->ws_bytes = kNoAllocScratchBytes;
+  p->timing = false;
+  rc = moe_forward(p, T, x, W_g, W1, W3, W2, W1s, W3s, W2s, out, stream);
+  p->ws = saved_ws;
+  p->ws_bytes = saved_bytes;
+  p->timing = saved_timing;
+  p->last_T = -1;   // the routing getters read the plan's own workspace only
+  return rc;
+}
+
 void moe_plan_destroy(moe_plan_t p) {
   if (!p) return;
   if (p->events_made)
