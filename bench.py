@@ -47,6 +47,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle timing (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time plain stream launches instead of CUDA-graph replays")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU seconds of the oracle sample")
     return ap.parse_args(argv)
@@ -309,20 +311,53 @@ def run_ours(args, info):
     touched = int((counts > 0).sum())
     launches_per_step = layer.plan.last_launch_count()
 
+    # ---- the step: one forward, replayed from a CUDA graph (default) or launched
+    graph = None
+    if not args.no_graph:
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            layer(x, out)
+        stream.wait_stream(cap)
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            layer(x, out)
+        torch.cuda.synchronize(dev)
+        for _ in range(3):
+            graph.replay()
+            flush.fill_(1)
+        torch.cuda.synchronize(dev)
+
+    def step():
+        if graph is not None:
+            graph.replay()
+        else:
+            layer(x, out)
+
     # ---- timed region: device time of K steps, max over ranks
-    layer.plan.enable_timing(True)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
-    ktimes = {}
     clocks = ClockSampler(dev.index if dev.index is not None else 0)
     replicas.barrier(info)
     torch.cuda.synchronize(dev)
     clocks.start()
-    names = None
     for i in range(args.steps):
         ev[i][0].record(stream)
-        layer(x, out)
+        step()
         ev[i][1].record(stream)
+        flush.fill_(1)
+    torch.cuda.synchronize(dev)
+    replicas.barrier(info)
+    local_ms = sum(a.elapsed_time(b) for a, b in ev)
+
+    # ---- per-kernel times: the same number of plain launches with events
+    #      recorded around every kernel on the stream it runs on
+    layer.plan.enable_timing(True)
+    ktimes = {}
+    names = None
+    for i in range(args.steps):
+        layer(x, out)
         flush.fill_(1)
         if names is None:
             names = layer.plan.kernel_names()
@@ -333,10 +368,8 @@ def run_ours(args, info):
         ktimes.setdefault(name, []).append(t)
     torch.cuda.synchronize(dev)
     clock_info = clocks.stop()
-    replicas.barrier(info)
     layer.plan.enable_timing(False)
     assert layer.device_status() == 0, "a kernel reported a bounded-wait timeout"
-    local_ms = sum(a.elapsed_time(b) for a, b in ev)
     total_ms = replicas.max_over_ranks(local_ms, info, device=dev)
     ms_per_step = total_ms / args.steps
     value = info.world_size * T * args.steps / (total_ms / 1e3)
@@ -413,6 +446,9 @@ def run_ours(args, info):
         "tflops": layer_flops / (ms_per_step / 1e3) / 1e12 * info.world_size,
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
+        "step_launch": "cuda graph replay" if graph is not None else "stream launches",
+        "kernel_times_from": f"{args.steps} plain forwards after the timed region, CUDA events "
+                             "around each kernel on its own stream",
         "clocks": clock_info,
         "kernels_ms": {k: round(v, 4) for k, v in kavg.items()},
         "routing": {"touched_experts": touched, "max_rows": int(counts.max()),

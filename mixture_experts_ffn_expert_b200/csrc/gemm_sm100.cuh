@@ -62,6 +62,9 @@ struct GemmParams {
   void* out;                 // bf16 or fp32, row-major
   long long ldo;             // elements between output rows
   int* status;               // device status word (moe_status codes)
+  int k_splits;              // split-K factor (fp32 epilogue only; 1 elsewhere): split s
+  int kb_per_split;          //   covers k-blocks [s*kb_per_split, ...) and writes its
+  long long split_stride;    //   partial sums at out + s*split_stride
 };
 
 // Dynamic shared memory the kernel needs for a given number of groups.
@@ -71,11 +74,15 @@ __host__ __device__ constexpr size_t gemm_smem_bytes(int num_groups) {
 }
 
 struct TileCoord {
-  int group, n_blk, row0, rows;
+  int group, n_blk, row0, rows, split;
 };
 
 __device__ __forceinline__ TileCoord decode_tile(int tile, const int* s_off, const int* s_mp,
                                                  int num_groups, int n_tiles) {
+  // split-K outermost: tiles of split s follow those of split s-1
+  const int per_split = s_mp[num_groups] * n_tiles;
+  const int split = tile / per_split;
+  tile -= split * per_split;
   // largest g with s_mp[g] * n_tiles <= tile (empty groups share a prefix value,
   // the largest index among them is the next non-empty group)
   int lo = 0, hi = num_groups;
@@ -92,6 +99,7 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, const int* s_off, con
   c.n_blk = n_blk;
   c.row0 = s_off[lo] + m_blk * kBM;
   c.rows = min(kBM, s_off[lo + 1] - c.row0);
+  c.split = split;
   return c;
 }
 
@@ -161,7 +169,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem_base = *s_tmem;
 
-  const int total_tiles = s_mp[num_groups] * P.n_tiles;
+  const int total_tiles = s_mp[num_groups] * P.n_tiles * P.k_splits;
   const int num_kb = (P.K + kBK - 1) / kBK;
 
   if (warp == 0) {
@@ -173,7 +181,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
       const TileCoord tc = decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles);
       const int z = P.group_offsets ? tc.group : 0;
-      for (int kb = 0; kb < num_kb; ++kb) {
+      const int kb_begin = tc.split * P.kb_per_split;
+      const int kb_end = min(num_kb, kb_begin + P.kb_per_split);
+      for (int kb = kb_begin; kb < kb_end; ++kb) {
         ok = mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, s_abort);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) {
@@ -218,12 +228,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_ph = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      const int split = tile / (s_mp[num_groups] * P.n_tiles);
+      const int kb_begin = split * P.kb_per_split;
+      const int kb_end = min(num_kb, kb_begin + P.kb_per_split);
       ok = mbar_wait(smem_u32(&tempty_bar[acc]), acc_ph ^ 1u, s_abort);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after_sync();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
-      for (int kb = 0; kb < num_kb; ++kb) {
+      for (int kb = kb_begin; kb < kb_end; ++kb) {
         ok = mbar_wait(smem_u32(&full_bar[s]), ph, s_abort);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
@@ -235,7 +248,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int k = 0; k < kBK / kUK; ++k) {
             umma_bf16(d_tmem, sdesc_kmajor_sw128(a_base + k * kUK * 2),
                       sdesc_kmajor_sw128(b_base + k * kUK * 2), idesc,
-                      (kb > 0 || k > 0) ? 1u : 0u);
+                      (kb > kb_begin || k > 0) ? 1u : 0u);
           }
           umma_commit(smem_u32(&empty_bar[s]));   // frees the stage when these MMAs finish
         }
@@ -332,7 +345,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               }
             }
           } else {
-            float* out = reinterpret_cast<float*>(P.out);
+            float* out = reinterpret_cast<float*>(P.out) + tc.split * P.split_stride;
 #pragma unroll
             for (int v = 0; v < 8; ++v) {
               const int col = col0 + c + v * 4;

@@ -41,9 +41,11 @@ constexpr int kTimingRing = 4;   // event sets: forward i records into set i % k
 struct Layout {
   size_t status, scores, idx, gate, chunk_counts, counts, offsets, mtiles, perm_src, inv_pos;
   size_t xperm, hidden, yrouted, hshared, yshared, total;
-  int lds;        // row stride of the fp32 router scores
-  int tpc;        // tokens per routing chunk
+  int lds;            // row stride of the fp32 router scores
+  int tpc;            // tokens per routing chunk
   int n_chunks;
+  int router_splits;  // split-K factor of the router GEMM (partials summed by route_topk)
+  int router_kb_per;  // k-blocks per split
 };
 
 }  // namespace
@@ -58,11 +60,15 @@ struct moe_plan {
   bool timing = false;
   int n_launch = 0;
   const char* names[kMaxKernels] = {};
-  cudaEvent_t ev[kTimingRing][kMaxKernels + 1] = {};
+  // per kernel a start and an end event, recorded on the stream it runs on
+  cudaEvent_t ev[kTimingRing][2 * kMaxKernels] = {};
   int ring_launches[kTimingRing] = {};
   long long timed_forwards = 0;     // forwards that recorded events
   int cur_set = 0;
   bool events_made = false;
+  // the shared expert runs on a forked stream, concurrently with the routing
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
 };
 
 namespace {
@@ -77,10 +83,20 @@ Layout make_layout(const moe_plan* p, int64_t T) {
   L.tpc = static_cast<int>(tpc);
   L.n_chunks = static_cast<int>((T + tpc - 1) / tpc);
   L.lds = static_cast<int>(align_up(p->n_routed, 8));
+  // split-K of the router GEMM so that it occupies most SMs even for few tokens
+  {
+    const int64_t tiles = ((T + moe::kBM - 1) / moe::kBM) * ((p->n_routed + moe::kBN - 1) / moe::kBN);
+    const int num_kb = (p->d + moe::kBK - 1) / moe::kBK;
+    int64_t sp = tiles > 0 ? p->num_sms / tiles : 1;
+    sp = sp < 1 ? 1 : (sp > 8 ? 8 : sp);
+    if (sp > num_kb) sp = num_kb;
+    L.router_kb_per = static_cast<int>((num_kb + sp - 1) / sp);
+    L.router_splits = (num_kb + L.router_kb_per - 1) / L.router_kb_per;
+  }
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
   L.status = take(256);
-  L.scores = take(size_t(T) * L.lds * 4);
+  L.scores = take(size_t(L.router_splits) * T * L.lds * 4);
   L.idx = take(size_t(A) * 4);
   L.gate = take(size_t(A) * 4);
   L.chunk_counts = take(size_t(p->n_routed) * (L.n_chunks > 0 ? L.n_chunks : 1) * 4);
@@ -138,17 +154,19 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t batch, uint64_t rows, u
 // ------------------------------------------------------------- launches
 struct Launcher {
   moe_plan* p;
-  cudaStream_t st;
+  cudaStream_t st;     // the caller's stream
   int status = MOE_OK;
 
-  void mark(const char* name) {
+  void begin(const char* name, cudaStream_t s) {
     if (p->n_launch < kMaxKernels) {
       p->names[p->n_launch] = name;
-      if (p->timing) cudaEventRecord(p->ev[p->cur_set][p->n_launch], st);
+      if (p->timing) cudaEventRecord(p->ev[p->cur_set][2 * p->n_launch], s);
     }
-    ++p->n_launch;
   }
-  bool check(const char* what) {
+  bool end(const char* what, cudaStream_t s) {
+    if (p->timing && p->n_launch < kMaxKernels)
+      cudaEventRecord(p->ev[p->cur_set][2 * p->n_launch + 1], s);
+    ++p->n_launch;
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
       status = fail(MOE_CUDA_ERROR, "%s launch failed: %s", what, cudaGetErrorString(e));
@@ -158,7 +176,6 @@ struct Launcher {
   }
   void finish() {
     if (p->timing && p->n_launch <= kMaxKernels) {
-      cudaEventRecord(p->ev[p->cur_set][p->n_launch], st);
       p->ring_launches[p->cur_set] = p->n_launch;
       ++p->timed_forwards;
     }
@@ -166,15 +183,16 @@ struct Launcher {
 };
 
 template <int MODE>
-bool launch_gemm(Launcher& L, const char* name, const CUtensorMap& a, const CUtensorMap& b0,
-                 const CUtensorMap& b1, const moe::GemmParams& prm, int max_tiles) {
+bool launch_gemm(Launcher& L, cudaStream_t s, const char* name, const CUtensorMap& a,
+                 const CUtensorMap& b0, const CUtensorMap& b1, const moe::GemmParams& prm,
+                 int max_tiles) {
   const int num_groups = prm.group_offsets ? prm.num_groups : 1;
   const size_t smem = moe::gemm_smem_bytes(num_groups);
   int grid = max_tiles < L.p->num_sms ? max_tiles : L.p->num_sms;
   if (grid < 1) grid = 1;
-  L.mark(name);
-  moe::moe_gemm_kernel<MODE><<<grid, moe::kGemmThreads, smem, L.st>>>(a, b0, b1, prm);
-  return L.check(name);
+  L.begin(name, s);
+  moe::moe_gemm_kernel<MODE><<<grid, moe::kGemmThreads, smem, s>>>(a, b0, b1, prm);
+  return L.end(name, s);
 }
 
 int set_kernel_attributes() {
@@ -241,6 +259,14 @@ moe_plan_t moe_plan_create(int d, int f, int n_routed, int top_k, int n_shared, 
   p->renorm = renorm ? 1 : 0;
   p->device = dev;
   p->num_sms = sms;
+  if (cudaStreamCreateWithFlags(&p->side, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&p->fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&p->join, cudaEventDisableTiming) != cudaSuccess) {
+    cudaGetLastError();
+    fail(MOE_CUDA_ERROR, "could not create the plan's side stream and events");
+    moe_plan_destroy(p);
+    return nullptr;
+  }
   return p;
 }
 
@@ -305,7 +331,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
                 p->device, dev);
   if (p->timing && !p->events_made) {
     for (int r = 0; r < kTimingRing; ++r)
-      for (int i = 0; i <= kMaxKernels; ++i) cudaEventCreate(&p->ev[r][i]);
+      for (int i = 0; i < 2 * kMaxKernels; ++i) cudaEventCreate(&p->ev[r][i]);
     p->events_made = true;
   }
   if (p->timing) p->cur_set = static_cast<int>(p->timed_forwards % kTimingRing);
@@ -345,7 +371,55 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   p->last_T = T;
   Launcher L{p, static_cast<cudaStream_t>(stream)};
 
-  // 1. router scores s = x W_g^T (fp32), dense over T rows
+  cudaStream_t main_st = L.st;
+  // The shared SwiGLU (coefficient 1, outside the routing) is independent of
+  // the routing. When it is small (at most half the SMs' worth of tiles, the
+  // decode regime) it runs on the plan's side stream, forked here and joined
+  // before the combine, so it hides behind the latency-bound routing kernels;
+  // a larger one would take SMs from the routing chain, so it runs inline on
+  // the main stream after the routed GEMMs instead.
+  const int shared_mt = static_cast<int>((T + 127) / 128);
+  const bool shared_forked =
+      p->n_shared > 0 && shared_mt * ((nsf + 127) / 128) <= p->num_sms / 2;
+  cudaStream_t shared_st = shared_forked ? p->side : main_st;
+  auto launch_shared = [&]() -> int {
+    moe::GemmParams g{};
+    g.dense_rows = static_cast<int>(T);
+    g.K = d;
+    g.N = nsf;
+    g.n_tiles = (nsf + 127) / 128;
+    g.out = hshared;
+    g.ldo = nsf;
+    g.status = status;
+    g.k_splits = 1;
+    g.kb_per_split = (d + moe::kBK - 1) / moe::kBK;
+    if (!launch_gemm<moe::kEpiSwiGLU>(L, shared_st, "shared_gate_up", mX, mW1s, mW3s, g,
+                                      shared_mt * g.n_tiles))
+      return L.status;
+    moe::GemmParams h{};
+    h.dense_rows = static_cast<int>(T);
+    h.K = nsf;
+    h.N = d;
+    h.n_tiles = (d + 255) / 256;
+    h.out = yshared;
+    h.ldo = d;
+    h.status = status;
+    h.k_splits = 1;
+    h.kb_per_split = (nsf + moe::kBK - 1) / moe::kBK;
+    if (!launch_gemm<moe::kEpiF32>(L, shared_st, "shared_down", mHs, mW2s, mW2s, h,
+                                   shared_mt * h.n_tiles))
+      return L.status;
+    return MOE_OK;
+  };
+  if (shared_forked) {
+    if (cudaEventRecord(p->fork, main_st) != cudaSuccess ||
+        cudaStreamWaitEvent(p->side, p->fork, 0) != cudaSuccess)
+      return fail(MOE_CUDA_ERROR, "fork of the shared-expert stream failed");
+    if (launch_shared() != MOE_OK) return L.status;
+    if (cudaEventRecord(p->join, p->side) != cudaSuccess)
+      return fail(MOE_CUDA_ERROR, "join record of the shared-expert stream failed");
+  }
+  // 1. router scores s = x W_g^T (fp32 partial sums of a split-K), dense over T rows
   {
     moe::GemmParams g{};
     g.dense_rows = static_cast<int>(T);
@@ -355,18 +429,22 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.out = scores;
     g.ldo = Lw.lds;
     g.status = status;
-    const int tiles = static_cast<int>((T + 127) / 128) * g.n_tiles;
-    if (!launch_gemm<moe::kEpiF32>(L, "router_gemm", mX, mWg, mWg, g, tiles)) return L.status;
+    g.k_splits = Lw.router_splits;
+    g.kb_per_split = Lw.router_kb_per;
+    g.split_stride = static_cast<long long>(T) * Lw.lds;
+    const int tiles = static_cast<int>((T + 127) / 128) * g.n_tiles * g.k_splits;
+    if (!launch_gemm<moe::kEpiF32>(L, main_st, "router_gemm", mX, mWg, mWg, g, tiles))
+      return L.status;
   }
   // 2. softmax + top-k + gates + per-chunk histogram
   {
     const size_t smem = size_t(nr) * 4;
     const int npl = (nr + 31) / 32;
-    L.mark("route_topk");
-#define MOE_TOPK_CASE(N)                                                                     \
-  moe::route_topk_kernel<N><<<Lw.n_chunks, moe::kRouteThreads, smem, L.st>>>(               \
-      scores, Lw.lds, p->bias, static_cast<int>(T), nr, k, p->renorm, Lw.tpc, Lw.n_chunks, \
-      idx, gate, chunk_counts)
+    L.begin("route_topk", main_st);
+#define MOE_TOPK_CASE(N)                                                                    \
+  moe::route_topk_kernel<N><<<Lw.n_chunks, moe::kRouteThreads, smem, main_st>>>(           \
+      scores, Lw.lds, Lw.router_splits, static_cast<long long>(T) * Lw.lds, p->bias,        \
+      static_cast<int>(T), nr, k, p->renorm, Lw.tpc, Lw.n_chunks, idx, gate, chunk_counts)
     if (npl <= 1) MOE_TOPK_CASE(1);
     else if (npl <= 2) MOE_TOPK_CASE(2);
     else if (npl <= 4) MOE_TOPK_CASE(4);
@@ -374,22 +452,25 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     else if (npl <= 16) MOE_TOPK_CASE(16);
     else MOE_TOPK_CASE(32);
 #undef MOE_TOPK_CASE
-    if (!L.check("route_topk")) return L.status;
+    if (!L.end("route_topk", main_st)) return L.status;
   }
-  // 3. per-expert prefix over chunks, offsets, m-tile prefix
-  L.mark("route_scan");
-  moe::route_scan_kernel<<<1, 1024, 0, L.st>>>(chunk_counts, Lw.n_chunks, nr, counts, offsets,
-                                               mtiles, moe::kBM);
-  if (!L.check("route_scan")) return L.status;
-  // 4. stable permutation + 16-byte row copies into the grouped batch
+  // 3. per-expert prefix over chunks and expert totals (one warp per expert)
   {
-    const size_t smem = size_t(nr) * 4 + size_t(Lw.tpc) * k * 4;
-    L.mark("route_scatter");
-    moe::route_scatter_kernel<<<Lw.n_chunks, moe::kRouteThreads, smem, L.st>>>(
-        idx, chunk_counts, offsets, static_cast<int>(T), k, nr, Lw.tpc, Lw.n_chunks,
+    const int warps = moe::kRouteThreads / 32;
+    L.begin("route_scan", main_st);
+    moe::route_scan_kernel<<<(nr + warps - 1) / warps, moe::kRouteThreads, 0, main_st>>>(
+        chunk_counts, Lw.n_chunks, nr, counts);
+    if (!L.end("route_scan", main_st)) return L.status;
+  }
+  // 4. offsets + m-tile prefix, stable permutation, 16-byte row copies
+  {
+    const size_t smem = size_t(moe::kMaxRouted + nr) * 4 + size_t(Lw.tpc) * k * 4;
+    L.begin("route_scatter", main_st);
+    moe::route_scatter_kernel<<<Lw.n_chunks, moe::kRouteThreads, smem, main_st>>>(
+        idx, chunk_counts, counts, static_cast<int>(T), k, nr, Lw.tpc, Lw.n_chunks, moe::kBM,
         reinterpret_cast<const uint4*>(x), d / 8, reinterpret_cast<uint4*>(xperm), perm_src,
-        inv_pos);
-    if (!L.check("route_scatter")) return L.status;
+        inv_pos, offsets, mtiles);
+    if (!L.end("route_scatter", main_st)) return L.status;
   }
   const int max_mtiles = static_cast<int>((A + 127) / 128 + (A < nr ? A : nr));
   // 5. grouped gate/up GEMM with the SiLU(gate) * up epilogue
@@ -404,7 +485,9 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.out = hidden;
     g.ldo = f;
     g.status = status;
-    if (!launch_gemm<moe::kEpiSwiGLU>(L, "grouped_gate_up", mXp, mW1, mW3, g,
+    g.k_splits = 1;
+    g.kb_per_split = (d + moe::kBK - 1) / moe::kBK;
+    if (!launch_gemm<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1, mW3, g,
                                       max_mtiles * g.n_tiles))
       return L.status;
   }
@@ -420,39 +503,27 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.out = yrouted;
     g.ldo = d;
     g.status = status;
-    if (!launch_gemm<moe::kEpiBF16>(L, "grouped_down", mH, mW2, mW2, g, max_mtiles * g.n_tiles))
+    g.k_splits = 1;
+    g.kb_per_split = (f + moe::kBK - 1) / moe::kBK;
+    if (!launch_gemm<moe::kEpiBF16>(L, main_st, "grouped_down", mH, mW2, mW2, g,
+                                    max_mtiles * g.n_tiles))
       return L.status;
   }
-  // 7. shared SwiGLU over all T rows (coefficient 1, outside the routing)
-  if (p->n_shared > 0) {
-    const int mt = static_cast<int>((T + 127) / 128);
-    moe::GemmParams g{};
-    g.dense_rows = static_cast<int>(T);
-    g.K = d;
-    g.N = nsf;
-    g.n_tiles = (nsf + 127) / 128;
-    g.out = hshared;
-    g.ldo = nsf;
-    g.status = status;
-    if (!launch_gemm<moe::kEpiSwiGLU>(L, "shared_gate_up", mX, mW1s, mW3s, g, mt * g.n_tiles))
-      return L.status;
-    moe::GemmParams h{};
-    h.dense_rows = static_cast<int>(T);
-    h.K = nsf;
-    h.N = d;
-    h.n_tiles = (d + 255) / 256;
-    h.out = yshared;
-    h.ldo = d;
-    h.status = status;
-    if (!launch_gemm<moe::kEpiF32>(L, "shared_down", mHs, mW2s, mW2s, h, mt * h.n_tiles))
-      return L.status;
+  // 7. the shared expert (inline, or joined from the side stream), then the
+  //    weighted combine + shared add with one bf16 rounding
+  if (p->n_shared > 0 && !shared_forked && launch_shared() != MOE_OK) return L.status;
+  if (shared_forked && cudaStreamWaitEvent(main_st, p->join, 0) != cudaSuccess)
+    return fail(MOE_CUDA_ERROR, "join of the shared-expert stream failed");
+  {
+    const int d_vec = d / 8;
+    const dim3 grid(static_cast<unsigned>(T),
+                    static_cast<unsigned>((d_vec + moe::kCombineThreads - 1) / moe::kCombineThreads));
+    L.begin("combine", main_st);
+    moe::combine_kernel<<<grid, moe::kCombineThreads, 0, main_st>>>(
+        reinterpret_cast<const uint4*>(yrouted), yshared, inv_pos, gate, k, d_vec,
+        reinterpret_cast<uint4*>(out));
+    if (!L.end("combine", main_st)) return L.status;
   }
-  // 8. weighted combine + shared add, one bf16 rounding
-  L.mark("combine");
-  moe::combine_kernel<<<static_cast<unsigned>(T), moe::kCombineThreads, 0, L.st>>>(
-      reinterpret_cast<const uint4*>(yrouted), yshared, inv_pos, gate, k, d / 8,
-      reinterpret_cast<uint4*>(out));
-  if (!L.check("combine")) return L.status;
   L.finish();
   return MOE_OK;
 }
@@ -522,11 +593,13 @@ int moe_plan_kernel_times(moe_plan_t p, int back, float* ms, int cap) {
   const int set = static_cast<int>((p->timed_forwards - 1 - back) % kTimingRing);
   const int n = p->ring_launches[set];
   if (n == 0) return 0;
-  cudaError_t e = cudaEventSynchronize(p->ev[set][n]);
+  // the last kernel (the combine) runs after every other one (it joins the
+  // side stream when the shared expert was forked), so its end event is last
+  cudaError_t e = cudaEventSynchronize(p->ev[set][2 * n - 1]);
   if (e != cudaSuccess) return -fail(MOE_CUDA_ERROR, "event sync: %s", cudaGetErrorString(e));
   for (int i = 0; i < n && i < cap; ++i) {
     float t = 0.0f;
-    e = cudaEventElapsedTime(&t, p->ev[set][i], p->ev[set][i + 1]);
+    e = cudaEventElapsedTime(&t, p->ev[set][2 * i], p->ev[set][2 * i + 1]);
     if (e != cudaSuccess) return -fail(MOE_CUDA_ERROR, "event time: %s", cudaGetErrorString(e));
     ms[i] = t;
   }
@@ -627,7 +700,10 @@ void moe_plan_destroy(moe_plan_t p) {
   if (!p) return;
   if (p->events_made)
     for (int r = 0; r < kTimingRing; ++r)
-      for (int i = 0; i <= kMaxKernels; ++i) cudaEventDestroy(p->ev[r][i]);
+      for (int i = 0; i < 2 * kMaxKernels; ++i) cudaEventDestroy(p->ev[r][i]);
+  if (p->side) cudaStreamDestroy(p->side);
+  if (p->fork) cudaEventDestroy(p->fork);
+  if (p->join) cudaEventDestroy(p->join);
   delete p;
 }
 

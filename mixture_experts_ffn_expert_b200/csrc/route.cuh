@@ -1,16 +1,19 @@
 // route.cuh - routing and combine kernels of the MoE layer (CUDA cores,
 // HBM/latency-bound work around the tensor-core GEMMs).
 //
-//  route_topk     softmax over the N_r router scores of a token, top-k with
-//                 ties to the lower expert index, raw or renormalised gates
+//  route_topk     sums the router-score partials of a split-K GEMM, adds the
+//                 logit bias, softmax over the N_r scores of a token, top-k
+//                 with ties to the lower expert index, raw or renormalised gates
 //                 ("What is an "expert," really?", glossary: router / gate,
 //                 top-k, softmax; panel 2), and a per-chunk expert histogram.
-//  route_scan     per-expert prefix over chunks, exclusive scan over experts
-//                 (offsets) and the prefix of 128-row m-tiles the grouped GEMM
-//                 scheduler walks.
-//  route_scatter  stable (token, slot) order inside each expert group; writes
-//                 the permutation and copies each token row to its k grouped
-//                 rows with 16-byte vectors.
+//  route_scan     one warp per expert: exclusive prefix over chunks of that
+//                 expert's counts, and the expert's total.
+//  route_scatter  every block derives the expert offsets (exclusive scan of the
+//                 totals) itself; block 0 also publishes offsets and the prefix
+//                 of 128-row m-tiles the grouped GEMM scheduler walks. Then the
+//                 stable (token, slot) order inside each expert group, the
+//                 permutation, and 16-byte-vector copies of each token row to
+//                 its k grouped rows.
 //  combine        out[t] = shared[t] + sum_j g[t,j] * Y[inv_pos[t,j]] in fp32,
 //                 one bf16 rounding ("Shared Expert (DeepSeek-V3)", eq. (12)
 //                 without the residual; shared term coefficient 1).
@@ -27,11 +30,14 @@ constexpr int kMaxTopK = 32;
 constexpr int kMaxRouted = 1024;
 
 // One warp per token; block = one chunk of `tpc` consecutive tokens.
-// NPL = router scores held per lane (N_r <= 32 * NPL).
+// NPL = router scores held per lane (N_r <= 32 * NPL). The scores arrive as
+// `splits` fp32 partial sums (split-K of the router GEMM), `split_stride`
+// elements apart, and are added in split order.
 template <int NPL>
 __global__ void __launch_bounds__(kRouteThreads)
-    route_topk_kernel(const float* __restrict__ scores, int lds, const float* __restrict__ bias,
-                      int T, int n_routed, int top_k, int renorm, int tpc, int n_chunks,
+    route_topk_kernel(const float* __restrict__ scores, int lds, int splits,
+                      long long split_stride, const float* __restrict__ bias, int T,
+                      int n_routed, int top_k, int renorm, int tpc, int n_chunks,
                       int* __restrict__ idx, float* __restrict__ gate,
                       int* __restrict__ chunk_counts) {
   extern __shared__ int s_hist[];               // [n_routed]
@@ -45,12 +51,25 @@ __global__ void __launch_bounds__(kRouteThreads)
   for (int t = t_begin + warp; t < t_end; t += kRouteThreads / 32) {
     const float* row = scores + static_cast<long long>(t) * lds;
     float v[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const int e = lane + 32 * i;
+      v[i] = e < n_routed ? row[e] : 0.0f;
+    }
+    // split-outer so that each split's NPL loads are in flight together
+    for (int sp = 1; sp < splits; ++sp) {
+      const float* r = row + sp * split_stride;
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < n_routed) v[i] += r[e];
+      }
+    }
     float m = -INFINITY;
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
       const int e = lane + 32 * i;
-      v[i] = -INFINITY;
-      if (e < n_routed) v[i] = row[e] + (bias ? bias[e] : 0.0f);
+      v[i] = e < n_routed ? v[i] + (bias ? bias[e] : 0.0f) : -INFINITY;
       m = fmaxf(m, v[i]);
     }
 #pragma unroll
@@ -99,68 +118,77 @@ __global__ void __launch_bounds__(kRouteThreads)
     chunk_counts[static_cast<long long>(e) * n_chunks + chunk] = s_hist[e];
 }
 
-// Single block of 1024 threads. chunk_counts [N_r][n_chunks] is turned in place
-// into the exclusive prefix over chunks of each expert.
-__global__ void __launch_bounds__(1024)
-    route_scan_kernel(int* __restrict__ chunk_counts, int n_chunks, int n_routed,
-                      int* __restrict__ counts, int* __restrict__ offsets,
-                      int* __restrict__ mtiles, int tile_rows) {
-  __shared__ int s_cnt[kMaxRouted];
-  __shared__ int s_wsum[32], s_wmt[32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int e = warp; e < n_routed; e += 32) {
-    int* row = chunk_counts + static_cast<long long>(e) * n_chunks;
-    int running = 0;
-    for (int c0 = 0; c0 < n_chunks; c0 += 32) {
-      const int c = c0 + lane;
-      const int v = c < n_chunks ? row[c] : 0;
-      int incl = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
-      }
-      if (c < n_chunks) row[c] = running + incl - v;
-      running += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) s_cnt[e] = running;
-  }
-  __syncthreads();
-  const int e = threadIdx.x;
-  const int c = e < n_routed ? s_cnt[e] : 0;
-  const int mt = (c + tile_rows - 1) / tile_rows;
-  int ic = c, im = mt;
+__device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int nc = __shfl_up_sync(0xffffffffu, ic, o);
-    const int nm = __shfl_up_sync(0xffffffffu, im, o);
-    if (lane >= o) { ic += nc; im += nm; }
+    const int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
   }
-  if (lane == 31) { s_wsum[warp] = ic; s_wmt[warp] = im; }
-  __syncthreads();
-  if (warp == 0) {
-    int a = s_wsum[lane], b = s_wmt[lane];
+  return v;
+}
+
+// One warp per expert (8 experts per block). chunk_counts [N_r][n_chunks]
+// becomes, in place, the exclusive prefix over chunks of each expert; the
+// warp's loads for up to 32*kScanPrefetch chunks are issued before any scan.
+constexpr int kScanPrefetch = 16;
+
+__global__ void __launch_bounds__(kRouteThreads)
+    route_scan_kernel(int* __restrict__ chunk_counts, int n_chunks, int n_routed,
+                      int* __restrict__ counts) {
+  const int lane = threadIdx.x & 31;
+  const int e = blockIdx.x * (kRouteThreads / 32) + (threadIdx.x >> 5);
+  if (e >= n_routed) return;
+  int* row = chunk_counts + static_cast<long long>(e) * n_chunks;
+  int running = 0;
+  for (int c0 = 0; c0 < n_chunks; c0 += 32 * kScanPrefetch) {
+    int v[kScanPrefetch];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int na = __shfl_up_sync(0xffffffffu, a, o);
-      const int nb = __shfl_up_sync(0xffffffffu, b, o);
-      if (lane >= o) { a += na; b += nb; }
+    for (int b = 0; b < kScanPrefetch; ++b) {
+      const int c = c0 + b * 32 + lane;
+      v[b] = c < n_chunks ? row[c] : 0;
     }
-    s_wsum[lane] = a - s_wsum[lane];     // exclusive prefix of warp totals
-    s_wmt[lane] = b - s_wmt[lane];
+#pragma unroll
+    for (int b = 0; b < kScanPrefetch; ++b) {
+      const int c = c0 + b * 32 + lane;
+      const int incl = warp_inclusive_scan(v[b], lane);
+      if (c < n_chunks) row[c] = running + incl - v[b];
+      running += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+  if (lane == 0) counts[e] = running;
+}
+
+// Exclusive scan of n (<= kMaxRouted) ints in shared memory by a 256-thread
+// block, in place; returns the total to every thread. `tmp` holds 8 ints.
+__device__ __forceinline__ int block_exclusive_scan(int* s, int n, int* tmp) {
+  constexpr int kPer = kMaxRouted / kRouteThreads;   // 4 consecutive items per thread
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int base = threadIdx.x * kPer;
+  int loc[kPer];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    loc[i] = base + i < n ? s[base + i] : 0;
+    sum += loc[i];
+  }
+  const int incl = warp_inclusive_scan(sum, lane);
+  if (lane == 31) tmp[warp] = incl;
+  __syncthreads();
+  int wbase = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < kRouteThreads / 32; ++w) {
+    const int t = tmp[w];
+    if (w < warp) wbase += t;
+    total += t;
+  }
+  int run = wbase + incl - sum;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    if (base + i < n) s[base + i] = run;
+    run += loc[i];
   }
   __syncthreads();
-  const int ex_c = s_wsum[warp] + ic - c;
-  const int ex_m = s_wmt[warp] + im - mt;
-  if (e < n_routed) {
-    counts[e] = c;
-    offsets[e] = ex_c;
-    mtiles[e] = ex_m;
-  }
-  if (e == n_routed - 1) {
-    offsets[n_routed] = ex_c + c;
-    mtiles[n_routed] = ex_m + mt;
-  }
+  return total;
 }
 
 // Block = one chunk. Warp 0 ranks the chunk's (token, slot) entries in order
@@ -168,15 +196,38 @@ __global__ void __launch_bounds__(1024)
 // every warp copies token rows (d_vec 16-byte vectors each) to their k rows.
 __global__ void __launch_bounds__(kRouteThreads)
     route_scatter_kernel(const int* __restrict__ idx, const int* __restrict__ chunk_base,
-                         const int* __restrict__ offsets, int T, int top_k, int n_routed,
-                         int tpc, int n_chunks, const uint4* __restrict__ x, int d_vec,
-                         uint4* __restrict__ xperm, int* __restrict__ perm_src,
-                         int* __restrict__ inv_pos) {
+                         const int* __restrict__ counts, int T, int top_k, int n_routed,
+                         int tpc, int n_chunks, int tile_rows, const uint4* __restrict__ x,
+                         int d_vec, uint4* __restrict__ xperm, int* __restrict__ perm_src,
+                         int* __restrict__ inv_pos, int* __restrict__ offsets_out,
+                         int* __restrict__ mtiles_out) {
   extern __shared__ int smem_i[];
-  int* s_run = smem_i;                  // [n_routed]
-  int* s_pos = smem_i + n_routed;       // [tpc * top_k]
-  for (int e = threadIdx.x; e < n_routed; e += blockDim.x) s_run[e] = 0;
+  int* s_off = smem_i;                        // [kMaxRouted] expert offsets
+  int* s_run = smem_i + kMaxRouted;           // [n_routed]
+  int* s_pos = s_run + n_routed;              // [tpc * top_k]
+  __shared__ int s_tmp[kRouteThreads / 32];
+  for (int e = threadIdx.x; e < n_routed; e += blockDim.x) {
+    s_off[e] = counts[e];
+    s_run[e] = 0;
+  }
   __syncthreads();
+  const int total = block_exclusive_scan(s_off, n_routed, s_tmp);
+  if (blockIdx.x == 0) {
+    // publish offsets and the m-tile prefix for the grouped GEMMs
+    for (int e = threadIdx.x; e < n_routed; e += blockDim.x) offsets_out[e] = s_off[e];
+    if (threadIdx.x == 0) offsets_out[n_routed] = total;
+    __syncthreads();
+    for (int e = threadIdx.x; e < n_routed; e += blockDim.x)
+      s_run[e] = (counts[e] + tile_rows - 1) / tile_rows;
+    __syncthreads();
+    const int total_mt = block_exclusive_scan(s_run, n_routed, s_tmp);
+    for (int e = threadIdx.x; e < n_routed; e += blockDim.x) {
+      mtiles_out[e] = s_run[e];
+      s_run[e] = 0;
+    }
+    if (threadIdx.x == 0) mtiles_out[n_routed] = total_mt;
+    __syncthreads();
+  }
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x;
@@ -192,7 +243,7 @@ __global__ void __launch_bounds__(kRouteThreads)
       const uint32_t same = __match_any_sync(0xffffffffu, e);
       const int rank = __popc(same & ((1u << lane) - 1u));
       if (valid)
-        s_pos[i] = offsets[e] + chunk_base[static_cast<long long>(e) * n_chunks + chunk] +
+        s_pos[i] = s_off[e] + chunk_base[static_cast<long long>(e) * n_chunks + chunk] +
                    s_run[e] + rank;
       __syncwarp();
       if (valid && lane == 31 - __clz(same)) s_run[e] += __popc(same);
@@ -231,8 +282,10 @@ __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
 }
 
 constexpr int kCombineThreads = 128;
+constexpr int kCombineBatch = 8;               // routed rows loaded before any FMA
 
-// Block = one token. shared (fp32, (T, d)) may be null when N_s = 0.
+// Grid (T, ceil(d_vec / 128)): block = one token and 128 16-byte column vectors.
+// shared (fp32, (T, d)) may be null when N_s = 0. The slots are added in order.
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const uint4* __restrict__ Y, const float* __restrict__ shared,
                    const int* __restrict__ inv_pos, const float* __restrict__ gate, int top_k,
@@ -245,22 +298,29 @@ __global__ void __launch_bounds__(kCombineThreads)
     s_w[threadIdx.x] = gate[t * top_k + threadIdx.x];
   }
   __syncthreads();
-  for (int v = threadIdx.x; v < d_vec; v += blockDim.x) {
-    float acc[8];
-    if (shared) {
-      const float4* s = reinterpret_cast<const float4*>(shared + (t * d_vec + v) * 8);
-      const float4 a = s[0], b = s[1];
-      acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
-      acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
-    } else {
+  const int v = blockIdx.y * kCombineThreads + threadIdx.x;
+  if (v >= d_vec) return;
+  float acc[8];
+  if (shared) {
+    const float4* s = reinterpret_cast<const float4*>(shared + (t * d_vec + v) * 8);
+    const float4 a = s[0], b = s[1];
+    acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
+    acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
+  } else {
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
-    }
-    for (int j = 0; j < top_k; ++j)
-      bf16x8_fma(acc, Y[static_cast<long long>(s_pos[j]) * d_vec + v], s_w[j]);
-    out[t * d_vec + v] = make_uint4(pack2_bf16(acc[0], acc[1]), pack2_bf16(acc[2], acc[3]),
-                                    pack2_bf16(acc[4], acc[5]), pack2_bf16(acc[6], acc[7]));
+    for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
   }
+  for (int j0 = 0; j0 < top_k; j0 += kCombineBatch) {
+    uint4 y[kCombineBatch];
+#pragma unroll
+    for (int u = 0; u < kCombineBatch; ++u)
+      if (j0 + u < top_k) y[u] = Y[static_cast<long long>(s_pos[j0 + u]) * d_vec + v];
+#pragma unroll
+    for (int u = 0; u < kCombineBatch; ++u)
+      if (j0 + u < top_k) bf16x8_fma(acc, y[u], s_w[j0 + u]);
+  }
+  out[t * d_vec + v] = make_uint4(pack2_bf16(acc[0], acc[1]), pack2_bf16(acc[2], acc[3]),
+                                  pack2_bf16(acc[4], acc[5]), pack2_bf16(acc[6], acc[7]));
 }
 
 }  // namespace moe

@@ -122,3 +122,32 @@ def test_error_paths_on_device():
     torch.cuda.synchronize()
     assert plan.device_status() == 0
     plan.close()
+
+
+@pytest.mark.parametrize("name", ["decode_t128_d2048_f512_e512k10_s1", "tiny_t256_d128_f64_e31k7_s1"])
+def test_cuda_graph_replay_matches_stream_launch(name):
+    # the whole forward (including the shared expert's forked stream, when used)
+    # is captured once and replayed; replays must reproduce the plain result
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    shape = WORKLOADS[name]
+    inp = make_layer_inputs(shape, seed=2, device="cuda")
+    layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
+                     shape.renorm, inp, bias=inp["bias"], device="cuda")
+    x = inp["x"]
+    want = layer(x).clone()
+    out = torch.empty_like(x)
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        layer(x, out)
+    torch.cuda.current_stream().wait_stream(cap)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        layer(x, out)
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, want)
+    assert layer.device_status() == 0
