@@ -133,17 +133,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  if (P.group_offsets) {
-    for (int i = threadIdx.x; i <= num_groups; i += blockDim.x) {
-      s_off[i] = P.group_offsets[i];
-      s_mp[i] = P.group_mtiles[i];
-    }
-  } else if (threadIdx.x == 0) {
-    s_off[0] = 0;
-    s_off[1] = P.dense_rows;
-    s_mp[0] = 0;
-    s_mp[1] = (P.dense_rows + kBM - 1) / kBM;
-  }
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
@@ -163,6 +153,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     tmem_alloc(smem_u32(s_tmem), kTmemCols);
     tmem_relinquish();
+  }
+  // everything above overlaps the previous kernel; the group tables and the A
+  // operand are written by it
+  pdl_wait();
+  if (P.group_offsets) {
+    for (int i = threadIdx.x; i <= num_groups; i += blockDim.x) {
+      s_off[i] = P.group_offsets[i];
+      s_mp[i] = P.group_mtiles[i];
+    }
+  } else if (threadIdx.x == 0) {
+    s_off[0] = 0;
+    s_off[1] = P.dense_rows;
+    s_mp[0] = 0;
+    s_mp[1] = (P.dense_rows + kBM - 1) / kBM;
   }
   tc_fence_before_sync();
   __syncthreads();

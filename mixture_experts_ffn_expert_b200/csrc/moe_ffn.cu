@@ -12,6 +12,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "moe_ffn.h"
 #include "gemm_sm100.cuh"
@@ -87,8 +88,11 @@ Layout make_layout(const moe_plan* p, int64_t T) {
   {
     const int64_t tiles = ((T + moe::kBM - 1) / moe::kBM) * ((p->n_routed + moe::kBN - 1) / moe::kBN);
     const int num_kb = (p->d + moe::kBK - 1) / moe::kBK;
+    // at most 8 splits, and at most 128 partial scores held per lane in route_topk
+    const int npl = (p->n_routed + 31) / 32;
+    const int64_t cap = npl <= 16 ? 8 : 128 / npl;
     int64_t sp = tiles > 0 ? p->num_sms / tiles : 1;
-    sp = sp < 1 ? 1 : (sp > 8 ? 8 : sp);
+    sp = sp < 1 ? 1 : (sp > cap ? cap : sp);
     if (sp > num_kb) sp = num_kb;
     L.router_kb_per = static_cast<int>((num_kb + sp - 1) / sp);
     L.router_splits = (num_kb + L.router_kb_per - 1) / L.router_kb_per;
@@ -182,6 +186,25 @@ struct Launcher {
   }
 };
 
+// Every kernel is launched with programmatic stream serialisation, so that it
+// can start its prologue while the previous kernel of the stream finishes; each
+// kernel waits (griddepcontrol.wait) before reading what its predecessor wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int MODE>
 bool launch_gemm(Launcher& L, cudaStream_t s, const char* name, const CUtensorMap& a,
                  const CUtensorMap& b0, const CUtensorMap& b1, const moe::GemmParams& prm,
@@ -191,7 +214,8 @@ bool launch_gemm(Launcher& L, cudaStream_t s, const char* name, const CUtensorMa
   int grid = max_tiles < L.p->num_sms ? max_tiles : L.p->num_sms;
   if (grid < 1) grid = 1;
   L.begin(name, s);
-  moe::moe_gemm_kernel<MODE><<<grid, moe::kGemmThreads, smem, s>>>(a, b0, b1, prm);
+  launch_pdl(moe::moe_gemm_kernel<MODE>, dim3(grid), dim3(moe::kGemmThreads), smem, s, a, b0,
+             b1, prm);
   return L.end(name, s);
 }
 
@@ -440,36 +464,47 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   {
     const size_t smem = size_t(nr) * 4;
     const int npl = (nr + 31) / 32;
+    const int sp = Lw.router_splits;
     L.begin("route_topk", main_st);
-#define MOE_TOPK_CASE(N)                                                                    \
-  moe::route_topk_kernel<N><<<Lw.n_chunks, moe::kRouteThreads, smem, main_st>>>(           \
-      scores, Lw.lds, Lw.router_splits, static_cast<long long>(T) * Lw.lds, p->bias,        \
-      static_cast<int>(T), nr, k, p->renorm, Lw.tpc, Lw.n_chunks, idx, gate, chunk_counts)
-    if (npl <= 1) MOE_TOPK_CASE(1);
-    else if (npl <= 2) MOE_TOPK_CASE(2);
-    else if (npl <= 4) MOE_TOPK_CASE(4);
-    else if (npl <= 8) MOE_TOPK_CASE(8);
-    else if (npl <= 16) MOE_TOPK_CASE(16);
-    else MOE_TOPK_CASE(32);
-#undef MOE_TOPK_CASE
+#define MOE_TOPK(N, S)                                                                      \
+  launch_pdl(moe::route_topk_kernel<N, S>, dim3(Lw.n_chunks), dim3(moe::kRouteThreads),     \
+             smem, main_st, (const float*)scores, Lw.lds, sp,                               \
+             static_cast<long long>(T) * Lw.lds, p->bias, static_cast<int>(T), nr, k,       \
+             p->renorm, Lw.tpc, Lw.n_chunks, idx, gate, chunk_counts)
+#define MOE_TOPK_S(N)                                                                       \
+  if (sp <= 1) MOE_TOPK(N, 1);                                                              \
+  else if (sp <= 2) MOE_TOPK(N, 2);                                                         \
+  else if (sp <= 4) MOE_TOPK(N, 4);                                                         \
+  else MOE_TOPK(N, 8)
+    if (npl <= 1) { MOE_TOPK_S(1); }
+    else if (npl <= 2) { MOE_TOPK_S(2); }
+    else if (npl <= 4) { MOE_TOPK_S(4); }
+    else if (npl <= 8) { MOE_TOPK_S(8); }
+    else if (npl <= 16) { MOE_TOPK_S(16); }
+    else if (sp <= 1) MOE_TOPK(32, 1);
+    else if (sp <= 2) MOE_TOPK(32, 2);
+    else MOE_TOPK(32, 4);
+#undef MOE_TOPK_S
+#undef MOE_TOPK
     if (!L.end("route_topk", main_st)) return L.status;
   }
   // 3. per-expert prefix over chunks and expert totals (one warp per expert)
   {
     const int warps = moe::kRouteThreads / 32;
     L.begin("route_scan", main_st);
-    moe::route_scan_kernel<<<(nr + warps - 1) / warps, moe::kRouteThreads, 0, main_st>>>(
-        chunk_counts, Lw.n_chunks, nr, counts);
+    launch_pdl(moe::route_scan_kernel, dim3((nr + warps - 1) / warps), dim3(moe::kRouteThreads),
+               0, main_st, chunk_counts, Lw.n_chunks, nr, counts);
     if (!L.end("route_scan", main_st)) return L.status;
   }
   // 4. offsets + m-tile prefix, stable permutation, 16-byte row copies
   {
-    const size_t smem = size_t(moe::kMaxRouted + nr) * 4 + size_t(Lw.tpc) * k * 4;
+    const size_t smem = size_t(moe::kMaxRouted + nr) * 4 + size_t(2) * Lw.tpc * k * 4;
     L.begin("route_scatter", main_st);
-    moe::route_scatter_kernel<<<Lw.n_chunks, moe::kRouteThreads, smem, main_st>>>(
-        idx, chunk_counts, counts, static_cast<int>(T), k, nr, Lw.tpc, Lw.n_chunks, moe::kBM,
-        reinterpret_cast<const uint4*>(x), d / 8, reinterpret_cast<uint4*>(xperm), perm_src,
-        inv_pos, offsets, mtiles);
+    launch_pdl(moe::route_scatter_kernel, dim3(Lw.n_chunks), dim3(moe::kRouteThreads), smem,
+               main_st, (const int*)idx, (const int*)chunk_counts, (const int*)counts,
+               static_cast<int>(T), k, nr, Lw.tpc, Lw.n_chunks, moe::kBM,
+               reinterpret_cast<const uint4*>(x), d / 8, reinterpret_cast<uint4*>(xperm),
+               perm_src, inv_pos, offsets, mtiles);
     if (!L.end("route_scatter", main_st)) return L.status;
   }
   const int max_mtiles = static_cast<int>((A + 127) / 128 + (A < nr ? A : nr));
@@ -519,9 +554,9 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     const dim3 grid(static_cast<unsigned>(T),
                     static_cast<unsigned>((d_vec + moe::kCombineThreads - 1) / moe::kCombineThreads));
     L.begin("combine", main_st);
-    moe::combine_kernel<<<grid, moe::kCombineThreads, 0, main_st>>>(
-        reinterpret_cast<const uint4*>(yrouted), yshared, inv_pos, gate, k, d_vec,
-        reinterpret_cast<uint4*>(out));
+    launch_pdl(moe::combine_kernel, grid, dim3(moe::kCombineThreads), 0, main_st,
+               reinterpret_cast<const uint4*>(yrouted), (const float*)yshared,
+               (const int*)inv_pos, (const float*)gate, k, d_vec, reinterpret_cast<uint4*>(out));
     if (!L.end("combine", main_st)) return L.status;
   }
   L.finish();

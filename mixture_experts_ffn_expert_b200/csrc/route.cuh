@@ -23,6 +23,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "ptx_sm100.cuh"
+
 namespace moe {
 
 constexpr int kRouteThreads = 256;             // 8 warps
@@ -31,9 +33,10 @@ constexpr int kMaxRouted = 1024;
 
 // One warp per token; block = one chunk of `tpc` consecutive tokens.
 // NPL = router scores held per lane (N_r <= 32 * NPL). The scores arrive as
-// `splits` fp32 partial sums (split-K of the router GEMM), `split_stride`
-// elements apart, and are added in split order.
-template <int NPL>
+// `splits` (<= MAXS) fp32 partial sums (split-K of the router GEMM),
+// `split_stride` elements apart, and are added in split order; all partial
+// loads of a lane are issued before the first add.
+template <int NPL, int MAXS>
 __global__ void __launch_bounds__(kRouteThreads)
     route_topk_kernel(const float* __restrict__ scores, int lds, int splits,
                       long long split_stride, const float* __restrict__ bias, int T,
@@ -41,7 +44,9 @@ __global__ void __launch_bounds__(kRouteThreads)
                       int* __restrict__ idx, float* __restrict__ gate,
                       int* __restrict__ chunk_counts) {
   extern __shared__ int s_hist[];               // [n_routed]
+  pdl_launch_dependents();
   for (int e = threadIdx.x; e < n_routed; e += blockDim.x) s_hist[e] = 0;
+  pdl_wait();                                   // scores come from the router GEMM
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -50,20 +55,21 @@ __global__ void __launch_bounds__(kRouteThreads)
   const int t_end = min(T, t_begin + tpc);
   for (int t = t_begin + warp; t < t_end; t += kRouteThreads / 32) {
     const float* row = scores + static_cast<long long>(t) * lds;
-    float v[NPL];
+    float part[MAXS][NPL];
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      const int e = lane + 32 * i;
-      v[i] = e < n_routed ? row[e] : 0.0f;
-    }
-    // split-outer so that each split's NPL loads are in flight together
-    for (int sp = 1; sp < splits; ++sp) {
-      const float* r = row + sp * split_stride;
+    for (int sp = 0; sp < MAXS; ++sp)
 #pragma unroll
       for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;
-        if (e < n_routed) v[i] += r[e];
+        part[sp][i] = (sp < splits && e < n_routed) ? row[sp * split_stride + e] : 0.0f;
       }
+    float v[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      float a = part[0][i];
+#pragma unroll
+      for (int sp = 1; sp < MAXS; ++sp) a += part[sp][i];
+      v[i] = a;
     }
     float m = -INFINITY;
 #pragma unroll
@@ -135,6 +141,8 @@ constexpr int kScanPrefetch = 16;
 __global__ void __launch_bounds__(kRouteThreads)
     route_scan_kernel(int* __restrict__ chunk_counts, int n_chunks, int n_routed,
                       int* __restrict__ counts) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int e = blockIdx.x * (kRouteThreads / 32) + (threadIdx.x >> 5);
   if (e >= n_routed) return;
@@ -191,9 +199,13 @@ __device__ __forceinline__ int block_exclusive_scan(int* s, int n, int* tmp) {
   return total;
 }
 
-// Block = one chunk. Warp 0 ranks the chunk's (token, slot) entries in order
-// with match-any, so rows inside an expert group follow ascending (t, j); then
-// every warp copies token rows (d_vec 16-byte vectors each) to their k rows.
+// Block = one chunk. The chunk's expert ids and their per-chunk bases are
+// staged in shared memory by all threads; warp 0 then ranks the (token, slot)
+// entries in order with match-any, so rows inside an expert group follow
+// ascending (t, j); every warp then copies token rows (d_vec 16-byte vectors
+// each) to their k rows, four vectors in flight per lane.
+constexpr int kCopyUnroll = 4;
+
 __global__ void __launch_bounds__(kRouteThreads)
     route_scatter_kernel(const int* __restrict__ idx, const int* __restrict__ chunk_base,
                          const int* __restrict__ counts, int T, int top_k, int n_routed,
@@ -204,8 +216,21 @@ __global__ void __launch_bounds__(kRouteThreads)
   extern __shared__ int smem_i[];
   int* s_off = smem_i;                        // [kMaxRouted] expert offsets
   int* s_run = smem_i + kMaxRouted;           // [n_routed]
-  int* s_pos = s_run + n_routed;              // [tpc * top_k]
+  int* s_e = s_run + n_routed;                // [tpc * top_k] expert of each entry
+  int* s_pos = s_e + tpc * top_k;             // [tpc * top_k] chunk base, then row
   __shared__ int s_tmp[kRouteThreads / 32];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int chunk = blockIdx.x;
+  const int t0 = chunk * tpc;
+  const int ntok = min(tpc, T - t0);
+  const int n_ent = ntok * top_k;
+  const long long ebase = static_cast<long long>(t0) * top_k;
+  for (int i = threadIdx.x; i < n_ent; i += blockDim.x) {
+    const int e = idx[ebase + i];
+    s_e[i] = e;
+    s_pos[i] = chunk_base[static_cast<long long>(e) * n_chunks + chunk];
+  }
   for (int e = threadIdx.x; e < n_routed; e += blockDim.x) {
     s_off[e] = counts[e];
     s_run[e] = 0;
@@ -230,21 +255,14 @@ __global__ void __launch_bounds__(kRouteThreads)
   }
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chunk = blockIdx.x;
-  const int t0 = chunk * tpc;
-  const int ntok = min(tpc, T - t0);
-  const int n_ent = ntok * top_k;
-  const long long ebase = static_cast<long long>(t0) * top_k;
   if (warp == 0) {
     for (int b = 0; b < n_ent; b += 32) {
       const int i = b + lane;
       const bool valid = i < n_ent;
-      const int e = valid ? idx[ebase + i] : -1;
+      const int e = valid ? s_e[i] : -1;
       const uint32_t same = __match_any_sync(0xffffffffu, e);
       const int rank = __popc(same & ((1u << lane) - 1u));
-      if (valid)
-        s_pos[i] = s_off[e] + chunk_base[static_cast<long long>(e) * n_chunks + chunk] +
-                   s_run[e] + rank;
+      if (valid) s_pos[i] += s_off[e] + s_run[e] + rank;
       __syncwarp();
       if (valid && lane == 31 - __clz(same)) s_run[e] += __popc(same);
       __syncwarp();
@@ -259,9 +277,17 @@ __global__ void __launch_bounds__(kRouteThreads)
   for (int tl = warp; tl < ntok; tl += kRouteThreads / 32) {
     const uint4* src = x + static_cast<long long>(t0 + tl) * d_vec;
     const int* pos = s_pos + tl * top_k;
-    for (int v = lane; v < d_vec; v += 32) {
-      const uint4 val = src[v];
-      for (int j = 0; j < top_k; ++j) xperm[static_cast<long long>(pos[j]) * d_vec + v] = val;
+    for (int v0 = lane; v0 < d_vec; v0 += 32 * kCopyUnroll) {
+      uint4 val[kCopyUnroll];
+#pragma unroll
+      for (int u = 0; u < kCopyUnroll; ++u)
+        if (v0 + 32 * u < d_vec) val[u] = src[v0 + 32 * u];
+      for (int j = 0; j < top_k; ++j) {
+        uint4* dst = xperm + static_cast<long long>(pos[j]) * d_vec;
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u)
+          if (v0 + 32 * u < d_vec) dst[v0 + 32 * u] = val[u];
+      }
     }
   }
 }
@@ -292,6 +318,8 @@ __global__ void __launch_bounds__(kCombineThreads)
                    int d_vec, uint4* __restrict__ out) {
   __shared__ int s_pos[kMaxTopK];
   __shared__ float s_w[kMaxTopK];
+  pdl_launch_dependents();
+  pdl_wait();
   const long long t = blockIdx.x;
   if (threadIdx.x < top_k) {
     s_pos[threadIdx.x] = inv_pos[t * top_k + threadIdx.x];
