@@ -18,7 +18,9 @@
 //  * warp 0: TMA producer (128B-swizzled boxes, no cluster multicast), a
 //    kStages-deep shared-memory ring guarded by full/empty mbarriers;
 //  * warp 1: allocates 512 TMEM columns, one thread issues
-//    tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) and commits;
+//    tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) and commits; a
+//    tile that owns at most 64 rows (a small expert group) uses M=64 instead,
+//    halving the tensor work spent on rows that are masked anyway;
 //  * warps 2..5: epilogue, each owns one 32-lane quarter of TMEM; two
 //    256-column accumulators let the epilogue of tile i overlap the MMAs of
 //    tile i+1;
@@ -225,14 +227,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN);
+    constexpr uint32_t idesc128 = idesc_bf16_f32(kBM, kBN);
+    constexpr uint32_t idesc64 = idesc_bf16_f32(64, kBN);
     int s = 0;
     uint32_t ph = 0;
     int acc = 0;
     uint32_t acc_ph = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-      const int split = tile / (s_mp[num_groups] * P.n_tiles);
+      const TileCoord tc = decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles);
+      const uint32_t idesc = tc.rows <= 64 ? idesc64 : idesc128;
+      const int split = tc.split;
       const int kb_begin = split * P.kb_per_split;
       const int kb_end = min(num_kb, kb_begin + P.kb_per_split);
       ok = mbar_wait(smem_u32(&tempty_bar[acc]), acc_ph ^ 1u, s_abort);
@@ -275,8 +280,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // M=128 accumulator: row r lives in TMEM lane r. M=64 accumulator: rows
+    // 16q..16q+15 live in lanes 32q..32q+15 of lane quarter q.
     const int quarter = warp & 3;                 // TMEM lanes this warp may access
-    const int r = quarter * 32 + lane;            // tile row owned by this thread
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     int acc = 0;
     uint32_t acc_ph = 0;
@@ -290,7 +296,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after_sync();
       const uint32_t tbase = lane_base + static_cast<uint32_t>(acc * kBN);
-      const bool row_ok = r < tc.rows;
+      const bool m64 = tc.rows <= 64;
+      const int r = m64 ? quarter * 16 + lane : quarter * 32 + lane;   // tile row of this thread
+      const bool row_ok = (!m64 || lane < 16) && r < tc.rows;
       const long long grow = static_cast<long long>(tc.row0) + r;
       if (MODE == kEpiSwiGLU) {
         const int col0 = tc.n_blk * 128;
