@@ -110,7 +110,7 @@ class ClockSampler:
             props = torch.cuda.get_device_properties(device_index)
             try:     # CUDA and NVML number devices differently under CUDA_VISIBLE_DEVICES
                 bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
-                self.h = pynvml.nvmlDeviceGetHandleByPciBusId_v2(bus)
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
             except Exception:
                 self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)

@@ -75,6 +75,15 @@ moe_plan_t moe_plan_create(int d, int f, int n_routed, int top_k, int n_shared,
 /* Status of the last moe_plan_create on this thread (MOE_OK if it succeeded). */
 int moe_last_status(void);
 
+/* Tuning options (moe_plan_set_option). Results do not depend on them.
+ * MOE_OPTION_PAIR_MIN_ROWS: a GEMM whose expected rows per expert group
+ *   (T*top_k/N_r for the routed experts, T for the shared expert) reach this
+ *   value runs as CTA pairs (tcgen05 cta_group::2, 256-row tiles, two SMs per
+ *   tile); smaller groups run one CTA per 128-row tile. Default 256; 0 always
+ *   uses pairs, a value above any T*top_k never does. */
+enum { MOE_OPTION_PAIR_MIN_ROWS = 1 };
+int moe_plan_set_option(moe_plan_t plan, int option, int64_t value);
+
 /* Optional per-expert logit bias: device pointer to N_r fp32 values added to
  * the router scores before the softmax (affects both selection and gates).
  * NULL removes it. The pointer must stay valid while forwards use it. */

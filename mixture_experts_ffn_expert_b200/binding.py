@@ -20,8 +20,9 @@ EXPORTED_SYMBOLS = [
     "moe_plan_set_workspace", "moe_forward", "moe_get_routing", "moe_get_permutation",
     "moe_plan_device_status", "moe_plan_enable_timing", "moe_plan_kernel_times",
     "moe_plan_kernel_name", "moe_plan_last_launch_count", "moe_plan_destroy", "moe_strerror",
-    "moe_last_error", "moe_forward_noalloc",
+    "moe_last_error", "moe_forward_noalloc", "moe_plan_set_option",
 ]
+MOE_OPTION_PAIR_MIN_ROWS = 1
 
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_INVALID_CONFIG", 2: "MOE_INVALID_ARG",
                 3: "MOE_WORKSPACE_TOO_SMALL", 4: "MOE_CUDA_ERROR", 5: "MOE_UNSUPPORTED",
@@ -52,6 +53,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     sig = {
         "moe_plan_create": (_vp, [_i, _i, _i, _i, _i, _i]),
         "moe_last_status": (_i, []),
+        "moe_plan_set_option": (_i, [_vp, _i, _i64]),
         "moe_plan_set_logit_bias": (_i, [_vp, _vp]),
         "moe_workspace_bytes": (_sz, [_vp, _i64]),
         "moe_plan_set_workspace": (_i, [_vp, _vp, _sz]),
@@ -94,6 +96,9 @@ class Plan:
         if not h:
             raise MoEError(self.lib.moe_last_status(), (self.lib.moe_last_error() or b"").decode())
         self.handle = h
+
+    def set_option(self, option: int, value: int) -> None:
+        _check(self.lib, self.lib.moe_plan_set_option(self.handle, option, value))
 
     def workspace_bytes(self, T: int) -> int:
         return int(self.lib.moe_workspace_bytes(self.handle, T))

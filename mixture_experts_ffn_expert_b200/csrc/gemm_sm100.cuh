@@ -76,11 +76,11 @@ __host__ __device__ constexpr size_t gemm_smem_bytes(int num_groups) {
 }
 
 struct TileCoord {
-  int group, n_blk, row0, rows, split;
+  int group, n_blk, row0, rows, split, mtiles;   // mtiles: m-blocks of this tile's group
 };
 
 __device__ __forceinline__ TileCoord decode_tile(int tile, const int* s_off, const int* s_mp,
-                                                 int num_groups, int n_tiles) {
+                                                 int num_groups, int n_tiles, int tile_m = kBM) {
   // split-K outermost: tiles of split s follow those of split s-1
   const int per_split = s_mp[num_groups] * n_tiles;
   const int split = tile / per_split;
@@ -99,9 +99,10 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, const int* s_off, con
   TileCoord c;
   c.group = lo;
   c.n_blk = n_blk;
-  c.row0 = s_off[lo] + m_blk * kBM;
-  c.rows = min(kBM, s_off[lo + 1] - c.row0);
+  c.row0 = s_off[lo] + m_blk * tile_m;
+  c.rows = min(tile_m, s_off[lo + 1] - c.row0);
   c.split = split;
+  c.mtiles = mt;
   return c;
 }
 
@@ -184,9 +185,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t ph = 0;
     uint32_t issued_mask = 0, issued_par = 0;  // per stage: issued at least once / last parity
     bool ok = true;
+    // Grouped GEMMs: the grouped rows are read again by every n-block, so they
+    // are kept in L2 (evict last); a weight tile is streamed (evict first) when
+    // its group has a single m-block, so no other tile will read it. Dense
+    // GEMMs and reused weight tiles use plain loads.
+    const bool grouped = P.group_offsets != nullptr;
+    const uint64_t keep = l2_evict_last_policy(), once = l2_evict_first_policy();
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
       const TileCoord tc = decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles);
       const int z = P.group_offsets ? tc.group : 0;
+      const bool stream = grouped && tc.mtiles == 1;
       const int kb_begin = tc.split * P.kb_per_split;
       const int kb_end = min(num_kb, kb_begin + P.kb_per_split);
       for (int kb = kb_begin; kb < kb_end; ++kb) {
@@ -202,13 +210,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t b_dst = a_dst + kATileBytes;
           const int k0 = kb * kBK;
           mbar_arrive_expect_tx(fb, kStageBytes);
-          tma_load_2d(a_dst, &tmA, fb, k0, tc.row0);
-          if (MODE == kEpiSwiGLU) {
-            tma_load_3d(b_dst, &tmB0, fb, k0, tc.n_blk * 128, z);
-            tma_load_3d(b_dst + kBHalfBytes, &tmB1, fb, k0, tc.n_blk * 128, z);
+          if (grouped)
+            tma_load_2d_hint(a_dst, &tmA, fb, k0, tc.row0, keep);
+          else
+            tma_load_2d(a_dst, &tmA, fb, k0, tc.row0);
+          const CUtensorMap* b1 = MODE == kEpiSwiGLU ? &tmB1 : &tmB0;
+          const int n0 = MODE == kEpiSwiGLU ? tc.n_blk * 128 : tc.n_blk * 256;
+          const int n1 = MODE == kEpiSwiGLU ? n0 : n0 + 128;
+          if (stream) {
+            tma_load_3d_hint(b_dst, &tmB0, fb, k0, n0, z, once);
+            tma_load_3d_hint(b_dst + kBHalfBytes, b1, fb, k0, n1, z, once);
           } else {
-            tma_load_3d(b_dst, &tmB0, fb, k0, tc.n_blk * 256, z);
-            tma_load_3d(b_dst + kBHalfBytes, &tmB0, fb, k0, tc.n_blk * 256 + 128, z);
+            tma_load_3d(b_dst, &tmB0, fb, k0, n0, z);
+            tma_load_3d(b_dst + kBHalfBytes, b1, fb, k0, n1, z);
           }
         }
         __syncwarp();
@@ -385,6 +399,313 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+
+// ---------------------------------------------------------------------------
+// CTA-pair variant (cta_group::2): a cluster of two CTAs on two SMs computes
+// one M=256 x N=256 tile. Each CTA loads its own 128 rows of A and its own
+// half of B (the W1 half on the even CTA and the W3 half on the odd one for
+// the SwiGLU epilogue, N rows 0-127 / 128-255 otherwise) into shared memory;
+// the even CTA issues the MMAs, which read both CTAs' shared memory, and each
+// CTA's TMEM receives its own 128 accumulator rows. Per MMA each SM now
+// supplies 8 KB of operands instead of 12 KB, which is what lets the tensor
+// pipe run closer to its peak; it is used when expert groups are large.
+//   * TMA loads of both CTAs count their bytes on the even CTA's full barrier;
+//   * the MMA commits are multicast to the empty / tmem-full barriers of both;
+//   * both CTAs' epilogue threads arrive on the even CTA's tmem-empty barrier.
+constexpr int kPairTileM = 256;
+constexpr int kPairStages = 6;
+constexpr int kPairStageBytes = kATileBytes + kBHalfBytes;   // 32 KB per CTA
+
+__host__ __device__ constexpr size_t gemm_pair_smem_bytes(int num_groups) {
+  return 1024 + size_t(kPairStages) * kPairStageBytes + 256 +
+         size_t(2) * (num_groups + 1) * sizeof(int);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    moe_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                         const __grid_constant__ CUtensorMap tmB0,
+                         const __grid_constant__ CUtensorMap tmB1, const GemmParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(kPairStages) * kPairStageBytes);
+  uint64_t* full_bar = bars;                          // [kPairStages] (even CTA's are used)
+  uint64_t* empty_bar = bars + kPairStages;           // [kPairStages] both CTAs
+  uint64_t* tfull_bar = bars + 2 * kPairStages;       // [kNumAcc] both CTAs
+  uint64_t* tempty_bar = tfull_bar + kNumAcc;         // [kNumAcc] (even CTA's are used)
+  uint64_t* drain_bar = tempty_bar + kNumAcc;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  int* s_off = reinterpret_cast<int*>(smem + size_t(kPairStages) * kPairStageBytes + 256);
+  const int num_groups = P.group_offsets ? P.num_groups : 1;
+  int* s_mp = s_off + (num_groups + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank & 1u) == 0u;
+  const uint32_t leader_rank = rank & ~1u;
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+
+  pdl_launch_dependents();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    for (int b = 0; b < kNumAcc; ++b) {
+      mbar_init(smem_u32(&tfull_bar[b]), 1);
+      mbar_init(smem_u32(&tempty_bar[b]), 2 * kEpiThreads);
+    }
+    mbar_init(smem_u32(drain_bar), 1);
+    *s_abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(s_tmem), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  pdl_wait();
+  if (P.group_offsets) {
+    for (int i = threadIdx.x; i <= num_groups; i += blockDim.x) {
+      s_off[i] = P.group_offsets[i];
+      s_mp[i] = P.group_mtiles[i];
+    }
+  } else if (threadIdx.x == 0) {
+    s_off[0] = 0;
+    s_off[1] = P.dense_rows;
+    s_mp[0] = 0;
+    s_mp[1] = (P.dense_rows + kPairTileM - 1) / kPairTileM;
+  }
+  // barrier initialisation and the TMEM allocation must be visible to the
+  // other CTA of the pair before either signals the other
+  tc_fence_before_sync();
+  cluster_sync();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *s_tmem;
+
+  const int total_tiles = s_mp[num_groups] * P.n_tiles;
+  const int num_kb = (P.K + kBK - 1) / kBK;
+  const int half = leader ? 0 : 1;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    int s = 0;
+    uint32_t ph = 0;
+    uint32_t issued_mask = 0, issued_par = 0;
+    bool ok = true;
+    // Grouped GEMMs: the grouped rows are read again by every n-block, so they
+    // are kept in L2 (evict last); a weight tile is streamed (evict first) when
+    // its group has a single m-block, so no other tile will read it. Dense
+    // GEMMs and reused weight tiles use plain loads.
+    const bool grouped = P.group_offsets != nullptr;
+    const uint64_t keep = l2_evict_last_policy(), once = l2_evict_first_policy();
+    for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
+      const TileCoord tc = decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles, kPairTileM);
+      const int z = P.group_offsets ? tc.group : 0;
+      const bool stream = grouped && tc.mtiles == 1;
+      const int my_row0 = tc.row0 + half * kBM;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        ok = mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, s_abort);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) {
+          if (lane == 0) raise_timeout(s_abort, P.status);
+          break;
+        }
+        if (lane == 0) {
+          const uint32_t fb = mapa_shared(smem_u32(&full_bar[s]), leader_rank);
+          const uint32_t a_dst = smem_u32(smem + size_t(s) * kPairStageBytes);
+          const uint32_t b_dst = a_dst + kATileBytes;
+          const int k0 = kb * kBK;
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full_bar[s]), 2 * kPairStageBytes);
+          if (grouped)
+            tma_load_2d_pair_hint(a_dst, &tmA, fb, k0, my_row0, keep);
+          else
+            tma_load_2d_pair(a_dst, &tmA, fb, k0, my_row0);
+          const CUtensorMap* bmap = (MODE == kEpiSwiGLU && half) ? &tmB1 : &tmB0;
+          const int n0 = MODE == kEpiSwiGLU ? tc.n_blk * 128 : tc.n_blk * 256 + half * 128;
+          if (stream)
+            tma_load_3d_pair_hint(b_dst, bmap, fb, k0, n0, z, once);
+          else
+            tma_load_3d_pair(b_dst, bmap, fb, k0, n0, z);
+        }
+        __syncwarp();
+        issued_mask |= 1u << s;
+        issued_par = (issued_par & ~(1u << s)) | (ph << s);
+        if (++s == kPairStages) { s = 0; ph ^= 1u; }
+      }
+    }
+    if (!ok && leader && lane == 0) {
+      // the even CTA's full barriers count both CTAs' bytes: give the copies in
+      // flight a bounded chance to land before teardown
+      for (int i = 0; i < kPairStages; ++i)
+        if (issued_mask & (1u << i)) {
+          int never = 0;
+          mbar_wait(smem_u32(&full_bar[i]), (issued_par >> i) & 1u, &never);
+        }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (leader) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kPairTileM, kBN);
+      int s = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t acc_ph = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
+        ok = mbar_wait(smem_u32(&tempty_bar[acc]), acc_ph ^ 1u, s_abort);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          ok = mbar_wait(smem_u32(&full_bar[s]), ph, s_abort);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after_sync();
+          if (lane == 0) {
+            const uint32_t a_base = smem_u32(smem + size_t(s) * kPairStageBytes);
+            const uint32_t b_base = a_base + kATileBytes;
+#pragma unroll
+            for (int k = 0; k < kBK / kUK; ++k)
+              umma_bf16_pair(d_tmem, sdesc_kmajor_sw128(a_base + k * kUK * 2),
+                             sdesc_kmajor_sw128(b_base + k * kUK * 2), idesc,
+                             (kb > 0 || k > 0) ? 1u : 0u);
+            umma_commit_pair(smem_u32(&empty_bar[s]));   // frees the stage in both CTAs
+          }
+          __syncwarp();
+          if (++s == kPairStages) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        if (lane == 0) umma_commit_pair(smem_u32(&tfull_bar[acc]));
+        __syncwarp();
+        if (++acc == kNumAcc) { acc = 0; acc_ph ^= 1u; }
+      }
+      if (!ok) {
+        if (lane == 0) {
+          raise_timeout(s_abort, P.status);
+          umma_commit_pair(smem_u32(drain_bar));
+          int never = 0;
+          mbar_wait(smem_u32(drain_bar), 0, &never);
+        }
+        __syncwarp();
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;                // row of this CTA's 128-row half
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    for (int tile = pair; tile < total_tiles; tile += n_pairs) {
+      const TileCoord tc = decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles, kPairTileM);
+      bool ok = mbar_wait(smem_u32(&tfull_bar[acc]), acc_ph, s_abort);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) raise_timeout(s_abort, P.status);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t tbase = lane_base + static_cast<uint32_t>(acc * kBN);
+      const bool row_ok = r < tc.rows - half * kBM;
+      const long long grow = static_cast<long long>(tc.row0) + half * kBM + r;
+      if (MODE == kEpiSwiGLU) {
+        const int col0 = tc.n_blk * 128;
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(P.out);
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          if (col0 + c >= P.N) break;
+          uint32_t g[32], u[32];
+          tmem_ld_32cols(tbase + c, g);
+          tmem_ld_32cols(tbase + 128 + c, u);
+          tmem_ld_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int col = col0 + c + v * 8;
+              if (col < P.N) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  const float g0 = __uint_as_float(g[v * 8 + 2 * q]);
+                  const float g1 = __uint_as_float(g[v * 8 + 2 * q + 1]);
+                  const float u0 = __uint_as_float(u[v * 8 + 2 * q]);
+                  const float u1 = __uint_as_float(u[v * 8 + 2 * q + 1]);
+                  pk[q] = pack_bf16x2(g0 / (1.0f + __expf(-g0)) * u0,
+                                      g1 / (1.0f + __expf(-g1)) * u1);
+                }
+                *reinterpret_cast<uint4*>(out + grow * P.ldo + col) =
+                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              }
+            }
+          }
+        }
+      } else {
+        const int col0 = tc.n_blk * 256;
+#pragma unroll 1
+        for (int c = 0; c < 256; c += 32) {
+          if (col0 + c >= P.N) break;
+          uint32_t a[32];
+          tmem_ld_32cols(tbase + c, a);
+          tmem_ld_wait();
+          if (!row_ok) continue;
+          if (MODE == kEpiBF16) {
+            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(P.out);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int col = col0 + c + v * 8;
+              if (col < P.N) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  pk[q] = pack_bf16x2(__uint_as_float(a[v * 8 + 2 * q]),
+                                      __uint_as_float(a[v * 8 + 2 * q + 1]));
+                *reinterpret_cast<uint4*>(out + grow * P.ldo + col) =
+                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              }
+            }
+          } else {
+            float* out = reinterpret_cast<float*>(P.out);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const int col = col0 + c + v * 4;
+              float* dst = out + grow * P.ldo + col;
+              if (col + 4 <= P.N) {
+                *reinterpret_cast<float4*>(dst) =
+                    make_float4(__uint_as_float(a[v * 4]), __uint_as_float(a[v * 4 + 1]),
+                                __uint_as_float(a[v * 4 + 2]), __uint_as_float(a[v * 4 + 3]));
+              } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  if (col + q < P.N) dst[q] = __uint_as_float(a[v * 4 + q]);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before_sync();
+      if (leader)
+        mbar_arrive(smem_u32(&tempty_bar[acc]));
+      else
+        mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[acc]), leader_rank));
+      if (++acc == kNumAcc) { acc = 0; acc_ph ^= 1u; }
+    }
+  }
+
+  // neither CTA may leave while the other can still signal its barriers
+  tc_fence_before_sync();
+  cluster_sync();
+  tc_fence_after_sync();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
 }
 
 }  // namespace moe

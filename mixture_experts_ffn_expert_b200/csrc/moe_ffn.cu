@@ -40,7 +40,8 @@ constexpr int kMaxKernels = 16;
 constexpr int kTimingRing = 4;   // event sets: forward i records into set i % kTimingRing
 
 struct Layout {
-  size_t status, scores, idx, gate, chunk_counts, counts, offsets, mtiles, perm_src, inv_pos;
+  size_t status, scores, idx, gate, chunk_counts, counts, offsets, mtiles, mtiles2, perm_src,
+      inv_pos;
   size_t xperm, hidden, yrouted, hshared, yshared, total;
   int lds;            // row stride of the fp32 router scores
   int tpc;            // tokens per routing chunk
@@ -53,6 +54,8 @@ struct Layout {
 
 struct moe_plan {
   int d, f, n_routed, top_k, n_shared, renorm;
+  // GEMMs whose expected rows per group reach this use the CTA-pair kernel
+  long long pair_min_rows = 256;
   int device, num_sms;
   const float* bias = nullptr;
   char* ws = nullptr;
@@ -107,6 +110,7 @@ Layout make_layout(const moe_plan* p, int64_t T) {
   L.counts = take(size_t(p->n_routed) * 4);
   L.offsets = take(size_t(p->n_routed + 1) * 4);
   L.mtiles = take(size_t(p->n_routed + 1) * 4);
+  L.mtiles2 = take(size_t(p->n_routed + 1) * 4);
   L.perm_src = take(size_t(A) * 4);
   L.inv_pos = take(size_t(A) * 4);
   L.xperm = take(size_t(A) * p->d * 2);
@@ -205,6 +209,36 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// CTA-pair GEMM: clusters of two CTAs, one M=256 tile per pair; prm.group_mtiles
+// must be the prefix of 256-row m-tiles. max_tiles counts 256-row tiles.
+template <int MODE>
+bool launch_gemm_pair(Launcher& L, cudaStream_t s, const char* name, const CUtensorMap& a,
+                      const CUtensorMap& b0, const CUtensorMap& b1, const moe::GemmParams& prm,
+                      int max_tiles) {
+  const int num_groups = prm.group_offsets ? prm.num_groups : 1;
+  const size_t smem = moe::gemm_pair_smem_bytes(num_groups);
+  int pairs = L.p->num_sms / 2;
+  if (max_tiles < pairs) pairs = max_tiles;
+  if (pairs < 1) pairs = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(moe::kGemmThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  L.begin(name, s);
+  cudaLaunchKernelEx(&cfg, moe::moe_gemm_pair_kernel<MODE>, a, b0, b1, prm);
+  return L.end(name, s);
+}
+
 template <int MODE>
 bool launch_gemm(Launcher& L, cudaStream_t s, const char* name, const CUtensorMap& a,
                  const CUtensorMap& b0, const CUtensorMap& b1, const moe::GemmParams& prm,
@@ -220,6 +254,17 @@ bool launch_gemm(Launcher& L, cudaStream_t s, const char* name, const CUtensorMa
 }
 
 int set_kernel_attributes() {
+  const size_t smem_pair = moe::gemm_pair_smem_bytes(moe::kMaxRouted);
+  const cudaError_t ep[3] = {
+      cudaFuncSetAttribute(moe::moe_gemm_pair_kernel<moe::kEpiSwiGLU>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_pair)),
+      cudaFuncSetAttribute(moe::moe_gemm_pair_kernel<moe::kEpiBF16>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_pair)),
+      cudaFuncSetAttribute(moe::moe_gemm_pair_kernel<moe::kEpiF32>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_pair))};
+  for (cudaError_t e : ep)
+    if (e != cudaSuccess)
+      return fail(MOE_CUDA_ERROR, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
   const size_t smem = moe::gemm_smem_bytes(moe::kMaxRouted);
   cudaError_t e1 = cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiSwiGLU>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
@@ -295,6 +340,18 @@ moe_plan_t moe_plan_create(int d, int f, int n_routed, int top_k, int n_shared, 
 }
 
 int moe_last_status(void) { return g_last_status; }
+
+int moe_plan_set_option(moe_plan_t p, int option, int64_t value) {
+  if (!p) return fail(MOE_INVALID_ARG, "null plan");
+  switch (option) {
+    case MOE_OPTION_PAIR_MIN_ROWS:
+      if (value < 0) return fail(MOE_INVALID_ARG, "pair_min_rows must be >= 0");
+      p->pair_min_rows = value;
+      return MOE_OK;
+    default:
+      return fail(MOE_INVALID_ARG, "unknown option %d", option);
+  }
+}
 
 int moe_plan_set_logit_bias(moe_plan_t p, const float* bias) {
   if (!p) return fail(MOE_INVALID_ARG, "null plan");
@@ -372,6 +429,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   int* counts = reinterpret_cast<int*>(ws + Lw.counts);
   int* offsets = reinterpret_cast<int*>(ws + Lw.offsets);
   int* mtiles = reinterpret_cast<int*>(ws + Lw.mtiles);
+  int* mtiles2 = reinterpret_cast<int*>(ws + Lw.mtiles2);
   int* perm_src = reinterpret_cast<int*>(ws + Lw.perm_src);
   int* inv_pos = reinterpret_cast<int*>(ws + Lw.inv_pos);
   void* xperm = ws + Lw.xperm;
@@ -406,6 +464,8 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   const bool shared_forked =
       p->n_shared > 0 && shared_mt * ((nsf + 127) / 128) <= p->num_sms / 2;
   cudaStream_t shared_st = shared_forked ? p->side : main_st;
+  const bool shared_pair = static_cast<long long>(T) >= p->pair_min_rows;
+  const int shared_mt2 = static_cast<int>((T + 255) / 256);
   auto launch_shared = [&]() -> int {
     moe::GemmParams g{};
     g.dense_rows = static_cast<int>(T);
@@ -417,8 +477,10 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.status = status;
     g.k_splits = 1;
     g.kb_per_split = (d + moe::kBK - 1) / moe::kBK;
-    if (!launch_gemm<moe::kEpiSwiGLU>(L, shared_st, "shared_gate_up", mX, mW1s, mW3s, g,
-                                      shared_mt * g.n_tiles))
+    if (shared_pair ? !launch_gemm_pair<moe::kEpiSwiGLU>(L, shared_st, "shared_gate_up", mX, mW1s,
+                                                         mW3s, g, shared_mt2 * g.n_tiles)
+                    : !launch_gemm<moe::kEpiSwiGLU>(L, shared_st, "shared_gate_up", mX, mW1s, mW3s,
+                                                    g, shared_mt * g.n_tiles))
       return L.status;
     moe::GemmParams h{};
     h.dense_rows = static_cast<int>(T);
@@ -430,8 +492,10 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     h.status = status;
     h.k_splits = 1;
     h.kb_per_split = (nsf + moe::kBK - 1) / moe::kBK;
-    if (!launch_gemm<moe::kEpiF32>(L, shared_st, "shared_down", mHs, mW2s, mW2s, h,
-                                   shared_mt * h.n_tiles))
+    if (shared_pair ? !launch_gemm_pair<moe::kEpiF32>(L, shared_st, "shared_down", mHs, mW2s, mW2s,
+                                                      h, shared_mt2 * h.n_tiles)
+                    : !launch_gemm<moe::kEpiF32>(L, shared_st, "shared_down", mHs, mW2s, mW2s, h,
+                                                 shared_mt * h.n_tiles))
       return L.status;
     return MOE_OK;
   };
@@ -504,15 +568,17 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
                main_st, (const int*)idx, (const int*)chunk_counts, (const int*)counts,
                static_cast<int>(T), k, nr, Lw.tpc, Lw.n_chunks, moe::kBM,
                reinterpret_cast<const uint4*>(x), d / 8, reinterpret_cast<uint4*>(xperm),
-               perm_src, inv_pos, offsets, mtiles);
+               perm_src, inv_pos, offsets, mtiles, mtiles2);
     if (!L.end("route_scatter", main_st)) return L.status;
   }
   const int max_mtiles = static_cast<int>((A + 127) / 128 + (A < nr ? A : nr));
+  const int max_mtiles2 = static_cast<int>((A + 255) / 256 + (A < nr ? A : nr));
+  const bool routed_pair = A >= p->pair_min_rows * static_cast<long long>(nr);
   // 5. grouped gate/up GEMM with the SiLU(gate) * up epilogue
   {
     moe::GemmParams g{};
     g.group_offsets = offsets;
-    g.group_mtiles = mtiles;
+    g.group_mtiles = routed_pair ? mtiles2 : mtiles;
     g.num_groups = nr;
     g.K = d;
     g.N = f;
@@ -522,15 +588,17 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.status = status;
     g.k_splits = 1;
     g.kb_per_split = (d + moe::kBK - 1) / moe::kBK;
-    if (!launch_gemm<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1, mW3, g,
-                                      max_mtiles * g.n_tiles))
+    if (routed_pair ? !launch_gemm_pair<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1,
+                                                         mW3, g, max_mtiles2 * g.n_tiles)
+                    : !launch_gemm<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1, mW3,
+                                                    g, max_mtiles * g.n_tiles))
       return L.status;
   }
   // 6. grouped down GEMM
   {
     moe::GemmParams g{};
     g.group_offsets = offsets;
-    g.group_mtiles = mtiles;
+    g.group_mtiles = routed_pair ? mtiles2 : mtiles;
     g.num_groups = nr;
     g.K = f;
     g.N = d;
@@ -540,8 +608,10 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.status = status;
     g.k_splits = 1;
     g.kb_per_split = (f + moe::kBK - 1) / moe::kBK;
-    if (!launch_gemm<moe::kEpiBF16>(L, main_st, "grouped_down", mH, mW2, mW2, g,
-                                    max_mtiles * g.n_tiles))
+    if (routed_pair ? !launch_gemm_pair<moe::kEpiBF16>(L, main_st, "grouped_down", mH, mW2, mW2, g,
+                                                       max_mtiles2 * g.n_tiles)
+                    : !launch_gemm<moe::kEpiBF16>(L, main_st, "grouped_down", mH, mW2, mW2, g,
+                                                  max_mtiles * g.n_tiles))
       return L.status;
   }
   // 7. the shared expert (inline, or joined from the side stream), then the
@@ -552,7 +622,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   {
     const int d_vec = d / 8;
     const dim3 grid(static_cast<unsigned>(T),
-                    static_cast<unsigned>((d_vec + moe::kCombineThreads - 1) / moe::kCombineThreads));
+                    static_cast<unsigned>((d_vec + moe::kCombineCols - 1) / moe::kCombineCols));
     L.begin("combine", main_st);
     launch_pdl(moe::combine_kernel, grid, dim3(moe::kCombineThreads), 0, main_st,
                reinterpret_cast<const uint4*>(yrouted), (const float*)yshared,

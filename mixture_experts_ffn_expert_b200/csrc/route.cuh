@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(kRouteThreads)
                          int tpc, int n_chunks, int tile_rows, const uint4* __restrict__ x,
                          int d_vec, uint4* __restrict__ xperm, int* __restrict__ perm_src,
                          int* __restrict__ inv_pos, int* __restrict__ offsets_out,
-                         int* __restrict__ mtiles_out) {
+                         int* __restrict__ mtiles_out, int* __restrict__ mtiles2_out) {
   extern __shared__ int smem_i[];
   int* s_off = smem_i;                        // [kMaxRouted] expert offsets
   int* s_run = smem_i + kMaxRouted;           // [n_routed]
@@ -241,16 +241,21 @@ __global__ void __launch_bounds__(kRouteThreads)
     // publish offsets and the m-tile prefix for the grouped GEMMs
     for (int e = threadIdx.x; e < n_routed; e += blockDim.x) offsets_out[e] = s_off[e];
     if (threadIdx.x == 0) offsets_out[n_routed] = total;
-    __syncthreads();
-    for (int e = threadIdx.x; e < n_routed; e += blockDim.x)
-      s_run[e] = (counts[e] + tile_rows - 1) / tile_rows;
-    __syncthreads();
-    const int total_mt = block_exclusive_scan(s_run, n_routed, s_tmp);
-    for (int e = threadIdx.x; e < n_routed; e += blockDim.x) {
-      mtiles_out[e] = s_run[e];
-      s_run[e] = 0;
+    // prefixes of m-tiles of tile_rows and of 2*tile_rows rows (CTA-pair tiles)
+    for (int pass = 0; pass < 2; ++pass) {
+      const int rows = tile_rows << pass;
+      int* dst = pass ? mtiles2_out : mtiles_out;
+      __syncthreads();
+      for (int e = threadIdx.x; e < n_routed; e += blockDim.x)
+        s_run[e] = (counts[e] + rows - 1) / rows;
+      __syncthreads();
+      const int total_mt = block_exclusive_scan(s_run, n_routed, s_tmp);
+      for (int e = threadIdx.x; e < n_routed; e += blockDim.x) {
+        dst[e] = s_run[e];
+        s_run[e] = 0;
+      }
+      if (threadIdx.x == 0) dst[n_routed] = total_mt;
     }
-    if (threadIdx.x == 0) mtiles_out[n_routed] = total_mt;
     __syncthreads();
   }
 
@@ -308,10 +313,14 @@ __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
 }
 
 constexpr int kCombineThreads = 128;
-constexpr int kCombineBatch = 8;               // routed rows loaded before any FMA
+constexpr int kCombineVec = 4;                 // 16-byte column vectors per thread
+constexpr int kCombineBatch = 4;               // routed rows loaded before any FMA
+constexpr int kCombineCols = kCombineThreads * kCombineVec;
 
-// Grid (T, ceil(d_vec / 128)): block = one token and 128 16-byte column vectors.
-// shared (fp32, (T, d)) may be null when N_s = 0. The slots are added in order.
+// Grid (T, ceil(d_vec / 512)): block = one token and 512 16-byte column vectors,
+// four per thread (strided by 128 so each load instruction is coalesced), all
+// k routed rows of a vector loaded before its FMAs. shared (fp32, (T, d)) may
+// be null when N_s = 0. The slots are added in order after the shared term.
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const uint4* __restrict__ Y, const float* __restrict__ shared,
                    const int* __restrict__ inv_pos, const float* __restrict__ gate, int top_k,
@@ -326,29 +335,45 @@ __global__ void __launch_bounds__(kCombineThreads)
     s_w[threadIdx.x] = gate[t * top_k + threadIdx.x];
   }
   __syncthreads();
-  const int v = blockIdx.y * kCombineThreads + threadIdx.x;
-  if (v >= d_vec) return;
-  float acc[8];
-  if (shared) {
-    const float4* s = reinterpret_cast<const float4*>(shared + (t * d_vec + v) * 8);
-    const float4 a = s[0], b = s[1];
-    acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
-    acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
-  } else {
+  const int v0 = blockIdx.y * kCombineCols + threadIdx.x;
+  float acc[kCombineVec][8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+  for (int u = 0; u < kCombineVec; ++u) {
+    const int v = v0 + u * kCombineThreads;
+    if (shared && v < d_vec) {
+      const float4* s = reinterpret_cast<const float4*>(shared + (t * d_vec + v) * 8);
+      const float4 a = s[0], b = s[1];
+      acc[u][0] = a.x; acc[u][1] = a.y; acc[u][2] = a.z; acc[u][3] = a.w;
+      acc[u][4] = b.x; acc[u][5] = b.y; acc[u][6] = b.z; acc[u][7] = b.w;
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[u][q] = 0.0f;
+    }
   }
   for (int j0 = 0; j0 < top_k; j0 += kCombineBatch) {
-    uint4 y[kCombineBatch];
+    uint4 y[kCombineBatch][kCombineVec];
 #pragma unroll
-    for (int u = 0; u < kCombineBatch; ++u)
-      if (j0 + u < top_k) y[u] = Y[static_cast<long long>(s_pos[j0 + u]) * d_vec + v];
+    for (int jj = 0; jj < kCombineBatch; ++jj)
 #pragma unroll
-    for (int u = 0; u < kCombineBatch; ++u)
-      if (j0 + u < top_k) bf16x8_fma(acc, y[u], s_w[j0 + u]);
+      for (int u = 0; u < kCombineVec; ++u) {
+        const int v = v0 + u * kCombineThreads;
+        if (j0 + jj < top_k && v < d_vec)
+          y[jj][u] = Y[static_cast<long long>(s_pos[j0 + jj]) * d_vec + v];
+      }
+#pragma unroll
+    for (int jj = 0; jj < kCombineBatch; ++jj)
+#pragma unroll
+      for (int u = 0; u < kCombineVec; ++u)
+        if (j0 + jj < top_k) bf16x8_fma(acc[u], y[jj][u], s_w[j0 + jj]);
   }
-  out[t * d_vec + v] = make_uint4(pack2_bf16(acc[0], acc[1]), pack2_bf16(acc[2], acc[3]),
-                                  pack2_bf16(acc[4], acc[5]), pack2_bf16(acc[6], acc[7]));
+#pragma unroll
+  for (int u = 0; u < kCombineVec; ++u) {
+    const int v = v0 + u * kCombineThreads;
+    if (v < d_vec)
+      out[t * d_vec + v] =
+          make_uint4(pack2_bf16(acc[u][0], acc[u][1]), pack2_bf16(acc[u][2], acc[u][3]),
+                     pack2_bf16(acc[u][4], acc[u][5]), pack2_bf16(acc[u][6], acc[u][7]));
+  }
 }
 
 }  // namespace moe

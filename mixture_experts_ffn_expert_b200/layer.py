@@ -10,7 +10,7 @@ from typing import Dict, Optional
 
 import torch
 
-from .binding import MoEError, Plan
+from .binding import MOE_OPTION_PAIR_MIN_ROWS, MoEError, Plan
 
 __all__ = ["MoELayer", "MoEError"]
 
@@ -29,7 +29,8 @@ class MoELayer:
 
     def __init__(self, d: int, f: int, n_routed: int, top_k: int, n_shared: int,
                  renorm: bool, weights: Dict[str, Optional[torch.Tensor]],
-                 bias: Optional[torch.Tensor] = None, device=None):
+                 bias: Optional[torch.Tensor] = None, device=None,
+                 pair_min_rows: Optional[int] = None):
         dev = torch.device(device) if device is not None else torch.device("cuda")
         if dev.type == "cuda" and dev.index is None:
             dev = torch.device("cuda", torch.cuda.current_device())
@@ -38,6 +39,8 @@ class MoELayer:
             raise MoEError(2, "MoELayer runs on a CUDA device only")
         with torch.cuda.device(self.device):
             self.plan = Plan(d, f, n_routed, top_k, n_shared, renorm)
+        if pair_min_rows is not None:
+            self.plan.set_option(MOE_OPTION_PAIR_MIN_ROWS, pair_min_rows)
         self.d, self.f, self.n_routed, self.top_k, self.n_shared = d, f, n_routed, top_k, n_shared
         self.renorm = bool(renorm)
         shapes = {"W_g": (n_routed, d), "W1": (n_routed, f, d), "W3": (n_routed, f, d),

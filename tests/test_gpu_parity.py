@@ -41,6 +41,34 @@ def test_small_layers_all_outputs(case):
     assert res["near_ties"] <= max(2, T * k // 20)
 
 
+PAIR_CASES = ["three_tokens", "ragged_17", "two_shared_raw", "ragged_tiles", "k_tail_not_64",
+              "skewed_groups"]
+
+
+@pytest.mark.parametrize("case", [c for c in SMALL if c[0] in PAIR_CASES],
+                         ids=[c[0] for c in SMALL if c[0] in PAIR_CASES])
+def test_small_layers_cta_pair_kernel(case):
+    # every GEMM (routed and shared) forced onto the cta_group::2 kernel
+    name, T, d, f, n, k, ns, renorm, bias = case
+    shape = LayerShape(name, T, d, f, n, k, ns, renorm, bias)
+    inp = make_layer_inputs(shape, seed=4, device="cuda")
+    full_parity(inp, shape, pair_min_rows=0)
+
+
+@pytest.mark.parametrize("pair_min_rows", [0, 1 << 40])
+def test_pair_and_single_kernels_agree_bitwise(pair_min_rows):
+    # both GEMM kernels accumulate each output in the same k order, so results match exactly
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    shape = LayerShape("agree", 700, 256, 192, 4, 2, 1, True, "none")
+    inp = make_layer_inputs(shape, seed=5, device="cuda")
+    ref = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared, True, inp,
+                   device="cuda", pair_min_rows=1 << 40)(inp["x"]).clone()
+    got = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared, True, inp,
+                   device="cuda", pair_min_rows=pair_min_rows)(inp["x"])
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
+
+
 def test_tiny_workload_all_outputs():
     shape = WORKLOADS["tiny_t256_d128_f64_e31k7_s1"]
     inp = make_layer_inputs(shape, seed=0, device="cuda")
