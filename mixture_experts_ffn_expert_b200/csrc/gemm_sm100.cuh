@@ -185,12 +185,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t ph = 0;
     uint32_t issued_mask = 0, issued_par = 0;  // per stage: issued at least once / last parity
     bool ok = true;
-    // Grouped GEMMs: the grouped rows are read again by every n-block, so they
-    // are kept in L2 (evict last); a weight tile is streamed (evict first) when
-    // its group has a single m-block, so no other tile will read it. Dense
-    // GEMMs and reused weight tiles use plain loads.
+    // Grouped GEMMs stream a weight tile (evict first) when its group has a
+    // single m-block, so no other tile will read it and it should not displace
+    // the grouped rows that every n-block reads again; all other loads are plain.
+    // (Pinning the grouped rows with evict_last was measured to push reused
+    // weight tiles out of L2 and nearly double the DRAM traffic.)
     const bool grouped = P.group_offsets != nullptr;
-    const uint64_t keep = l2_evict_last_policy(), once = l2_evict_first_policy();
+    const uint64_t once = l2_evict_first_policy();
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
       const TileCoord tc = decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles);
       const int z = P.group_offsets ? tc.group : 0;
@@ -210,10 +211,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t b_dst = a_dst + kATileBytes;
           const int k0 = kb * kBK;
           mbar_arrive_expect_tx(fb, kStageBytes);
-          if (grouped)
-            tma_load_2d_hint(a_dst, &tmA, fb, k0, tc.row0, keep);
-          else
-            tma_load_2d(a_dst, &tmA, fb, k0, tc.row0);
+          tma_load_2d(a_dst, &tmA, fb, k0, tc.row0);
           const CUtensorMap* b1 = MODE == kEpiSwiGLU ? &tmB1 : &tmB0;
           const int n0 = MODE == kEpiSwiGLU ? tc.n_blk * 128 : tc.n_blk * 256;
           const int n1 = MODE == kEpiSwiGLU ? n0 : n0 + 128;
@@ -501,12 +499,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t ph = 0;
     uint32_t issued_mask = 0, issued_par = 0;
     bool ok = true;
-    // Grouped GEMMs: the grouped rows are read again by every n-block, so they
-    // are kept in L2 (evict last); a weight tile is streamed (evict first) when
-    // its group has a single m-block, so no other tile will read it. Dense
-    // GEMMs and reused weight tiles use plain loads.
+    // Grouped GEMMs stream a weight tile (evict first) when its group has a
+    // single m-block, so no other tile will read it and it should not displace
+    // the grouped rows that every n-block reads again; all other loads are plain.
+    // (Pinning the grouped rows with evict_last was measured to push reused
+    // weight tiles out of L2 and nearly double the DRAM traffic.)
     const bool grouped = P.group_offsets != nullptr;
-    const uint64_t keep = l2_evict_last_policy(), once = l2_evict_first_policy();
+    const uint64_t once = l2_evict_first_policy();
     for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
       const TileCoord tc = decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles, kPairTileM);
       const int z = P.group_offsets ? tc.group : 0;
@@ -525,10 +524,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t b_dst = a_dst + kATileBytes;
           const int k0 = kb * kBK;
           if (leader) mbar_arrive_expect_tx(smem_u32(&full_bar[s]), 2 * kPairStageBytes);
-          if (grouped)
-            tma_load_2d_pair_hint(a_dst, &tmA, fb, k0, my_row0, keep);
-          else
-            tma_load_2d_pair(a_dst, &tmA, fb, k0, my_row0);
+          tma_load_2d_pair(a_dst, &tmA, fb, k0, my_row0);
           const CUtensorMap* bmap = (MODE == kEpiSwiGLU && half) ? &tmB1 : &tmB0;
           const int n0 = MODE == kEpiSwiGLU ? tc.n_blk * 128 : tc.n_blk * 256 + half * 128;
           if (stream)
