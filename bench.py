@@ -160,6 +160,7 @@ def kernel_work(name, shape, T, touched):
     """(flops, bytes) the kernel cannot avoid: its inputs, outputs and weights."""
     d, f, n, k = shape.d, shape.f, shape.n_routed, shape.top_k
     A, nsf = T * k, shape.n_shared * shape.f
+    name = name.split("[")[0]          # GEMM variant tags do not change the work
     table = {
         "router_gemm": (2 * T * d * n, 2 * n * d + 2 * T * d + 4 * T * n),
         "route_topk": (0, 4 * T * n + 8 * A),
@@ -392,7 +393,7 @@ def run_ours(args, info):
                 "peak_source": f"{peak_src} ({'bf16 sustained' if bound == 'tensor' else 'HBM copy'})",
                 "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": nbytes,
                 "avg_launch_ms": round(kavg[dominant], 4),
-                "traffic": profiled_traffic(dominant, shape.name)}
+                "traffic": profiled_traffic(dominant.split("[")[0], shape.name)}
     if bound == "tensor":
         roofline["frac_of_burst_peak"] = round(achieved / peaks["bf16_tflops"], 4)
     layer_flops = (2 * T * shape.d * shape.n_routed + 6 * T * shape.top_k * shape.d * shape.f

@@ -79,9 +79,15 @@ int moe_last_status(void);
  * MOE_OPTION_PAIR_MIN_ROWS: a GEMM whose expected rows per expert group
  *   (T*top_k/N_r for the routed experts, T for the shared expert) reach this
  *   value runs as CTA pairs (tcgen05 cta_group::2, 256-row tiles, two SMs per
- *   tile); smaller groups run one CTA per 128-row tile. Default 256; 0 always
- *   uses pairs, a value above any T*top_k never does. */
-enum { MOE_OPTION_PAIR_MIN_ROWS = 1 };
+ *   tile); smaller groups run one CTA per 128-row tile. By default only the
+ *   routed down projection uses pairs, from 256 rows per expert; setting the
+ *   option applies the value to every GEMM (0 always uses pairs, a value above
+ *   any T*top_k never does).
+ * MOE_OPTION_WIDE_TILES: CTA-pair tiles of 512 accumulator columns instead of
+ *   256 (fewer operand bytes per FLOP, fewer tiles). -1 (default) chooses per
+ *   GEMM (wide for reductions of at least 4096 with at least 3 waves of
+ *   tiles), 0 never, 1 always. */
+enum { MOE_OPTION_PAIR_MIN_ROWS = 1, MOE_OPTION_WIDE_TILES = 2 };
 int moe_plan_set_option(moe_plan_t plan, int option, int64_t value);
 
 /* Optional per-expert logit bias: device pointer to N_r fp32 values added to
@@ -139,7 +145,9 @@ int moe_plan_device_status(moe_plan_t plan);
  * steps before the latest one (0 = latest, at most 3) and writes up to `cap`
  * per-kernel durations in milliseconds; it returns how many kernels that
  * forward launched, or a negative moe_status. moe_plan_kernel_name gives the
- * name of kernel i of the last forward (static string; NULL when out of range). */
+ * name of kernel i of the last forward, with "[pair]" or "[pair512]" appended
+ * for the CTA-pair GEMM variants (owned by the plan, valid until the next
+ * forward; NULL when out of range). */
 int moe_plan_enable_timing(moe_plan_t plan, int enable);
 int moe_plan_kernel_times(moe_plan_t plan, int back, float* ms, int cap);
 const char* moe_plan_kernel_name(moe_plan_t plan, int i);

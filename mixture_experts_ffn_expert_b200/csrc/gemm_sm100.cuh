@@ -402,42 +402,60 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 // ---------------------------------------------------------------------------
 // CTA-pair variant (cta_group::2): a cluster of two CTAs on two SMs computes
-// one M=256 x N=256 tile. Each CTA loads its own 128 rows of A and its own
-// half of B (the W1 half on the even CTA and the W3 half on the odd one for
-// the SwiGLU epilogue, N rows 0-127 / 128-255 otherwise) into shared memory;
-// the even CTA issues the MMAs, which read both CTAs' shared memory, and each
-// CTA's TMEM receives its own 128 accumulator rows. Per MMA each SM now
-// supplies 8 KB of operands instead of 12 KB, which is what lets the tensor
-// pipe run closer to its peak; it is used when expert groups are large.
+// one M=256 tile of NW*256 accumulator columns. Each CTA loads its own 128 rows
+// of A and its own half of B (the W1 half on the even CTA and the W3 half on
+// the odd one for the SwiGLU epilogue, N rows 0-127 / 128-255 of every 256
+// otherwise) into shared memory; the even CTA issues the MMAs, which read both
+// CTAs' shared memory, and each CTA's TMEM receives its own 128 accumulator
+// rows. Per MMA each SM supplies 8 KB of operands instead of 12 KB.
 //   * TMA loads of both CTAs count their bytes on the even CTA's full barrier;
 //   * the MMA commits are multicast to the empty / tmem-full barriers of both;
-//   * both CTAs' epilogue threads arrive on the even CTA's tmem-empty barrier.
+//   * both CTAs' epilogue threads arrive on the even CTA's tmem-empty barriers.
+// TMEM holds two 256-column regions. NW=1: each tile uses one region, two
+// tiles alternate (the epilogue of one overlaps the MMAs of the next). NW=2
+// (wide tiles, 256x512): each tile uses both regions; the operand bytes per
+// FLOP drop by a quarter, and each region is released as soon as the epilogue
+// has drained it, so the next tile's MMAs into region 0 overlap the epilogue
+// of region 1.
 constexpr int kPairTileM = 256;
-constexpr int kPairStages = 6;
-constexpr int kPairStageBytes = kATileBytes + kBHalfBytes;   // 32 KB per CTA
 
+template <int NW>
+struct PairCfg {
+  static constexpr int kBBytes = NW * kBHalfBytes;            // this CTA's B rows per stage
+  static constexpr int kStageBytes = kATileBytes + kBBytes;   // 32 KB (NW=1), 48 KB (NW=2)
+  static constexpr int kStages = NW == 1 ? 6 : 4;
+};
+
+template <int NW>
 __host__ __device__ constexpr size_t gemm_pair_smem_bytes(int num_groups) {
-  return 1024 + size_t(kPairStages) * kPairStageBytes + 256 +
+  return 1024 + size_t(PairCfg<NW>::kStages) * PairCfg<NW>::kStageBytes + 256 +
          size_t(2) * (num_groups + 1) * sizeof(int);
 }
 
-template <int MODE>
+// Output columns one pair tile produces.
+__host__ __device__ constexpr int pair_tile_cols(int mode, int nw) {
+  return (mode == kEpiSwiGLU ? 128 : 256) * nw;
+}
+
+template <int MODE, int NW>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB0,
                          const __grid_constant__ CUtensorMap tmB1, const GemmParams P) {
+  using Cfg = PairCfg<NW>;
+  constexpr int kS = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(kPairStages) * kPairStageBytes);
-  uint64_t* full_bar = bars;                          // [kPairStages] (even CTA's are used)
-  uint64_t* empty_bar = bars + kPairStages;           // [kPairStages] both CTAs
-  uint64_t* tfull_bar = bars + 2 * kPairStages;       // [kNumAcc] both CTAs
-  uint64_t* tempty_bar = tfull_bar + kNumAcc;         // [kNumAcc] (even CTA's are used)
-  uint64_t* drain_bar = tempty_bar + kNumAcc;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(kS) * Cfg::kStageBytes);
+  uint64_t* full_bar = bars;                          // [kS] (even CTA's are used)
+  uint64_t* empty_bar = bars + kS;                    // [kS] both CTAs
+  uint64_t* tfull_bar = bars + 2 * kS;                // [2] both CTAs
+  uint64_t* tempty_bar = tfull_bar + 2;               // [2] per TMEM region (even CTA's)
+  uint64_t* drain_bar = tempty_bar + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
-  int* s_off = reinterpret_cast<int*>(smem + size_t(kPairStages) * kPairStageBytes + 256);
+  int* s_off = reinterpret_cast<int*>(smem + size_t(kS) * Cfg::kStageBytes + 256);
   const int num_groups = P.group_offsets ? P.num_groups : 1;
   int* s_mp = s_off + (num_groups + 1);
 
@@ -451,11 +469,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   pdl_launch_dependents();
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kPairStages; ++s) {
+    for (int s = 0; s < kS; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
-    for (int b = 0; b < kNumAcc; ++b) {
+    for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&tfull_bar[b]), 1);
       mbar_init(smem_u32(&tempty_bar[b]), 2 * kEpiThreads);
     }
@@ -495,22 +513,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
+    // Grouped GEMMs stream a weight tile (evict first) when its group has a
+    // single m-block, so no other tile will read it; all other loads are plain.
+    const bool grouped = P.group_offsets != nullptr;
+    const uint64_t once = l2_evict_first_policy();
     int s = 0;
     uint32_t ph = 0;
     uint32_t issued_mask = 0, issued_par = 0;
     bool ok = true;
-    // Grouped GEMMs stream a weight tile (evict first) when its group has a
-    // single m-block, so no other tile will read it and it should not displace
-    // the grouped rows that every n-block reads again; all other loads are plain.
-    // (Pinning the grouped rows with evict_last was measured to push reused
-    // weight tiles out of L2 and nearly double the DRAM traffic.)
-    const bool grouped = P.group_offsets != nullptr;
-    const uint64_t once = l2_evict_first_policy();
     for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
       const TileCoord tc = decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles, kPairTileM);
       const int z = P.group_offsets ? tc.group : 0;
       const bool stream = grouped && tc.mtiles == 1;
       const int my_row0 = tc.row0 + half * kBM;
+      const CUtensorMap* bmap = (MODE == kEpiSwiGLU && half) ? &tmB1 : &tmB0;
       for (int kb = 0; kb < num_kb; ++kb) {
         ok = mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, s_abort);
         ok = __all_sync(0xffffffffu, ok);
@@ -520,28 +536,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (lane == 0) {
           const uint32_t fb = mapa_shared(smem_u32(&full_bar[s]), leader_rank);
-          const uint32_t a_dst = smem_u32(smem + size_t(s) * kPairStageBytes);
+          const uint32_t a_dst = smem_u32(smem + size_t(s) * Cfg::kStageBytes);
           const uint32_t b_dst = a_dst + kATileBytes;
           const int k0 = kb * kBK;
-          if (leader) mbar_arrive_expect_tx(smem_u32(&full_bar[s]), 2 * kPairStageBytes);
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full_bar[s]), 2 * Cfg::kStageBytes);
           tma_load_2d_pair(a_dst, &tmA, fb, k0, my_row0);
-          const CUtensorMap* bmap = (MODE == kEpiSwiGLU && half) ? &tmB1 : &tmB0;
-          const int n0 = MODE == kEpiSwiGLU ? tc.n_blk * 128 : tc.n_blk * 256 + half * 128;
-          if (stream)
-            tma_load_3d_pair_hint(b_dst, bmap, fb, k0, n0, z, once);
-          else
-            tma_load_3d_pair(b_dst, bmap, fb, k0, n0, z);
+#pragma unroll
+          for (int j = 0; j < NW; ++j) {
+            const int n = MODE == kEpiSwiGLU ? tc.n_blk * 128 * NW + j * 128
+                                             : tc.n_blk * 256 * NW + j * 256 + half * 128;
+            if (stream)
+              tma_load_3d_pair_hint(b_dst + j * kBHalfBytes, bmap, fb, k0, n, z, once);
+            else
+              tma_load_3d_pair(b_dst + j * kBHalfBytes, bmap, fb, k0, n, z);
+          }
         }
         __syncwarp();
         issued_mask |= 1u << s;
         issued_par = (issued_par & ~(1u << s)) | (ph << s);
-        if (++s == kPairStages) { s = 0; ph ^= 1u; }
+        if (++s == kS) { s = 0; ph ^= 1u; }
       }
     }
     if (!ok && leader && lane == 0) {
       // the even CTA's full barriers count both CTAs' bytes: give the copies in
       // flight a bounded chance to land before teardown
-      for (int i = 0; i < kPairStages; ++i)
+      for (int i = 0; i < kS; ++i)
         if (issued_mask & (1u << i)) {
           int never = 0;
           mbar_wait(smem_u32(&full_bar[i]), (issued_par >> i) & 1u, &never);
@@ -553,37 +572,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       constexpr uint32_t idesc = idesc_bf16_f32(kPairTileM, kBN);
       int s = 0;
       uint32_t ph = 0;
-      int acc = 0;
-      uint32_t acc_ph = 0;
+      int slot = 0;                // NW=1: TMEM region of this tile
+      uint32_t slot_ph = 0;        // phase of the region barriers this tile waits on
       bool ok = true;
       for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
-        ok = mbar_wait(smem_u32(&tempty_bar[acc]), acc_ph ^ 1u, s_abort);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after_sync();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = 0; kb < num_kb && ok; ++kb) {
           ok = mbar_wait(smem_u32(&full_bar[s]), ph, s_abort);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc_fence_after_sync();
-          if (lane == 0) {
-            const uint32_t a_base = smem_u32(smem + size_t(s) * kPairStageBytes);
-            const uint32_t b_base = a_base + kATileBytes;
+          const uint32_t a_base = smem_u32(smem + size_t(s) * Cfg::kStageBytes);
+          const uint32_t b_base = a_base + kATileBytes;
 #pragma unroll
-            for (int k = 0; k < kBK / kUK; ++k)
-              umma_bf16_pair(d_tmem, sdesc_kmajor_sw128(a_base + k * kUK * 2),
-                             sdesc_kmajor_sw128(b_base + k * kUK * 2), idesc,
-                             (kb > 0 || k > 0) ? 1u : 0u);
-            umma_commit_pair(smem_u32(&empty_bar[s]));   // frees the stage in both CTAs
+          for (int j = 0; j < NW; ++j) {
+            const int region = NW == 1 ? slot : j;
+            if (kb == 0) {
+              // the region must have been drained by both epilogues
+              ok = mbar_wait(smem_u32(&tempty_bar[region]), slot_ph ^ 1u, s_abort);
+              ok = __all_sync(0xffffffffu, ok);
+              if (!ok) break;
+              tc_fence_after_sync();
+            }
+            if (lane == 0) {
+              const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(region * kBN);
+#pragma unroll
+              for (int k = 0; k < kBK / kUK; ++k)
+                umma_bf16_pair(d_tmem, sdesc_kmajor_sw128(a_base + k * kUK * 2),
+                               sdesc_kmajor_sw128(b_base + j * kBHalfBytes + k * kUK * 2),
+                               idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            }
+            __syncwarp();
           }
+          if (!ok) break;
+          if (lane == 0) umma_commit_pair(smem_u32(&empty_bar[s]));   // frees the stage in both CTAs
           __syncwarp();
-          if (++s == kPairStages) { s = 0; ph ^= 1u; }
+          if (++s == kS) { s = 0; ph ^= 1u; }
         }
         if (!ok) break;
-        if (lane == 0) umma_commit_pair(smem_u32(&tfull_bar[acc]));
+        if (lane == 0) umma_commit_pair(smem_u32(&tfull_bar[NW == 1 ? slot : 0]));
         __syncwarp();
-        if (++acc == kNumAcc) { acc = 0; acc_ph ^= 1u; }
+        if (NW == 1) {
+          if (++slot == 2) { slot = 0; slot_ph ^= 1u; }
+        } else {
+          slot_ph ^= 1u;
+        }
       }
       if (!ok) {
         if (lane == 0) {
@@ -600,100 +632,110 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                // row of this CTA's 128-row half
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-    int acc = 0;
-    uint32_t acc_ph = 0;
+    int slot = 0;
+    uint32_t slot_ph = 0;
     for (int tile = pair; tile < total_tiles; tile += n_pairs) {
       const TileCoord tc = decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles, kPairTileM);
-      bool ok = mbar_wait(smem_u32(&tfull_bar[acc]), acc_ph, s_abort);
+      const int tb = NW == 1 ? slot : 0;
+      bool ok = mbar_wait(smem_u32(&tfull_bar[tb]), slot_ph, s_abort);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
         if (lane == 0) raise_timeout(s_abort, P.status);
         break;
       }
       tc_fence_after_sync();
-      const uint32_t tbase = lane_base + static_cast<uint32_t>(acc * kBN);
       const bool row_ok = r < tc.rows - half * kBM;
       const long long grow = static_cast<long long>(tc.row0) + half * kBM + r;
-      if (MODE == kEpiSwiGLU) {
-        const int col0 = tc.n_blk * 128;
-        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(P.out);
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          if (col0 + c >= P.N) break;
-          uint32_t g[32], u[32];
-          tmem_ld_32cols(tbase + c, g);
-          tmem_ld_32cols(tbase + 128 + c, u);
-          tmem_ld_wait();
-          if (row_ok) {
+      for (int j = 0; j < NW; ++j) {
+        const int region = NW == 1 ? slot : j;
+        const uint32_t tbase = lane_base + static_cast<uint32_t>(region * kBN);
+        if (MODE == kEpiSwiGLU) {
+          const int col0 = tc.n_blk * 128 * NW + j * 128;
+          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(P.out);
+#pragma unroll 1
+          for (int c = 0; c < 128; c += 32) {
+            if (col0 + c >= P.N) break;
+            uint32_t g[32], u[32];
+            tmem_ld_32cols(tbase + c, g);
+            tmem_ld_32cols(tbase + 128 + c, u);
+            tmem_ld_wait();
+            if (row_ok) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const int col = col0 + c + v * 8;
-              if (col < P.N) {
-                uint32_t pk[4];
+              for (int v = 0; v < 4; ++v) {
+                const int col = col0 + c + v * 8;
+                if (col < P.N) {
+                  uint32_t pk[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  const float g0 = __uint_as_float(g[v * 8 + 2 * q]);
-                  const float g1 = __uint_as_float(g[v * 8 + 2 * q + 1]);
-                  const float u0 = __uint_as_float(u[v * 8 + 2 * q]);
-                  const float u1 = __uint_as_float(u[v * 8 + 2 * q + 1]);
-                  pk[q] = pack_bf16x2(g0 / (1.0f + __expf(-g0)) * u0,
-                                      g1 / (1.0f + __expf(-g1)) * u1);
+                  for (int q = 0; q < 4; ++q) {
+                    const float g0 = __uint_as_float(g[v * 8 + 2 * q]);
+                    const float g1 = __uint_as_float(g[v * 8 + 2 * q + 1]);
+                    const float u0 = __uint_as_float(u[v * 8 + 2 * q]);
+                    const float u1 = __uint_as_float(u[v * 8 + 2 * q + 1]);
+                    pk[q] = pack_bf16x2(g0 / (1.0f + __expf(-g0)) * u0,
+                                        g1 / (1.0f + __expf(-g1)) * u1);
+                  }
+                  *reinterpret_cast<uint4*>(out + grow * P.ldo + col) =
+                      make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
-                *reinterpret_cast<uint4*>(out + grow * P.ldo + col) =
-                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
               }
             }
           }
-        }
-      } else {
-        const int col0 = tc.n_blk * 256;
+        } else {
+          const int col0 = tc.n_blk * 256 * NW + j * 256;
 #pragma unroll 1
-        for (int c = 0; c < 256; c += 32) {
-          if (col0 + c >= P.N) break;
-          uint32_t a[32];
-          tmem_ld_32cols(tbase + c, a);
-          tmem_ld_wait();
-          if (!row_ok) continue;
-          if (MODE == kEpiBF16) {
-            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(P.out);
+          for (int c = 0; c < 256; c += 32) {
+            if (col0 + c >= P.N) break;
+            uint32_t a[32];
+            tmem_ld_32cols(tbase + c, a);
+            tmem_ld_wait();
+            if (!row_ok) continue;
+            if (MODE == kEpiBF16) {
+              __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(P.out);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const int col = col0 + c + v * 8;
-              if (col < P.N) {
-                uint32_t pk[4];
+              for (int v = 0; v < 4; ++v) {
+                const int col = col0 + c + v * 8;
+                if (col < P.N) {
+                  uint32_t pk[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                  pk[q] = pack_bf16x2(__uint_as_float(a[v * 8 + 2 * q]),
-                                      __uint_as_float(a[v * 8 + 2 * q + 1]));
-                *reinterpret_cast<uint4*>(out + grow * P.ldo + col) =
-                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                  for (int q = 0; q < 4; ++q)
+                    pk[q] = pack_bf16x2(__uint_as_float(a[v * 8 + 2 * q]),
+                                        __uint_as_float(a[v * 8 + 2 * q + 1]));
+                  *reinterpret_cast<uint4*>(out + grow * P.ldo + col) =
+                      make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
               }
-            }
-          } else {
-            float* out = reinterpret_cast<float*>(P.out);
+            } else {
+              float* out = reinterpret_cast<float*>(P.out);
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              const int col = col0 + c + v * 4;
-              float* dst = out + grow * P.ldo + col;
-              if (col + 4 <= P.N) {
-                *reinterpret_cast<float4*>(dst) =
-                    make_float4(__uint_as_float(a[v * 4]), __uint_as_float(a[v * 4 + 1]),
-                                __uint_as_float(a[v * 4 + 2]), __uint_as_float(a[v * 4 + 3]));
-              } else {
+              for (int v = 0; v < 8; ++v) {
+                const int col = col0 + c + v * 4;
+                float* dst = out + grow * P.ldo + col;
+                if (col + 4 <= P.N) {
+                  *reinterpret_cast<float4*>(dst) =
+                      make_float4(__uint_as_float(a[v * 4]), __uint_as_float(a[v * 4 + 1]),
+                                  __uint_as_float(a[v * 4 + 2]), __uint_as_float(a[v * 4 + 3]));
+                } else {
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                  if (col + q < P.N) dst[q] = __uint_as_float(a[v * 4 + q]);
+                  for (int q = 0; q < 4; ++q)
+                    if (col + q < P.N) dst[q] = __uint_as_float(a[v * 4 + q]);
+                }
               }
             }
           }
         }
+        // this region is drained: release it to the even CTA's MMA issuer
+        tc_fence_before_sync();
+        if (leader)
+          mbar_arrive(smem_u32(&tempty_bar[region]));
+        else
+          mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[region]), leader_rank));
       }
-      tc_fence_before_sync();
-      if (leader)
-        mbar_arrive(smem_u32(&tempty_bar[acc]));
-      else
-        mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[acc]), leader_rank));
-      if (++acc == kNumAcc) { acc = 0; acc_ph ^= 1u; }
+      if (NW == 1) {
+        if (++slot == 2) { slot = 0; slot_ph ^= 1u; }
+      } else {
+        slot_ph ^= 1u;
+      }
     }
   }
 

@@ -54,8 +54,15 @@ struct Layout {
 
 struct moe_plan {
   int d, f, n_routed, top_k, n_shared, renorm;
-  // GEMMs whose expected rows per group reach this use the CTA-pair kernel
-  long long pair_min_rows = 256;
+  // GEMMs whose expected rows per group reach these use the CTA-pair kernel.
+  // Measured on B200: the pair kernel wins for the routed down projection
+  // (plain epilogue) but not for the SwiGLU GEMMs, where the single-CTA kernel
+  // runs at the same throughput per clock and draws less power, so it holds a
+  // higher clock under the power cap. MOE_OPTION_PAIR_MIN_ROWS sets both.
+  long long pair_min_rows_plain = 256;
+  long long pair_min_rows_swiglu = 1LL << 62;
+  // CTA-pair tiles 512 accumulator columns wide: -1 automatic, 0 never, 1 always
+  int wide_tiles = -1;
   int device, num_sms;
   const float* bias = nullptr;
   char* ws = nullptr;
@@ -63,7 +70,7 @@ struct moe_plan {
   int64_t last_T = -1;
   bool timing = false;
   int n_launch = 0;
-  const char* names[kMaxKernels] = {};
+  char names[kMaxKernels][48] = {};   // kernel of each launch, with the GEMM variant
   // per kernel a start and an end event, recorded on the stream it runs on
   cudaEvent_t ev[kTimingRing][2 * kMaxKernels] = {};
   int ring_launches[kTimingRing] = {};
@@ -165,9 +172,9 @@ struct Launcher {
   cudaStream_t st;     // the caller's stream
   int status = MOE_OK;
 
-  void begin(const char* name, cudaStream_t s) {
+  void begin(const char* name, cudaStream_t s, const char* variant = "") {
     if (p->n_launch < kMaxKernels) {
-      p->names[p->n_launch] = name;
+      snprintf(p->names[p->n_launch], sizeof(p->names[0]), "%s%s", name, variant);
       if (p->timing) cudaEventRecord(p->ev[p->cur_set][2 * p->n_launch], s);
     }
   }
@@ -210,13 +217,14 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 // CTA-pair GEMM: clusters of two CTAs, one M=256 tile per pair; prm.group_mtiles
-// must be the prefix of 256-row m-tiles. max_tiles counts 256-row tiles.
-template <int MODE>
+// must be the prefix of 256-row m-tiles and prm.n_tiles count tiles of
+// pair_tile_cols(MODE, NW) columns. max_tiles bounds the number of tiles.
+template <int MODE, int NW>
 bool launch_gemm_pair(Launcher& L, cudaStream_t s, const char* name, const CUtensorMap& a,
                       const CUtensorMap& b0, const CUtensorMap& b1, const moe::GemmParams& prm,
                       int max_tiles) {
   const int num_groups = prm.group_offsets ? prm.num_groups : 1;
-  const size_t smem = moe::gemm_pair_smem_bytes(num_groups);
+  const size_t smem = moe::gemm_pair_smem_bytes<NW>(num_groups);
   int pairs = L.p->num_sms / 2;
   if (max_tiles < pairs) pairs = max_tiles;
   if (pairs < 1) pairs = 1;
@@ -234,9 +242,32 @@ bool launch_gemm_pair(Launcher& L, cudaStream_t s, const char* name, const CUten
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  L.begin(name, s);
-  cudaLaunchKernelEx(&cfg, moe::moe_gemm_pair_kernel<MODE>, a, b0, b1, prm);
+  L.begin(name, s, NW == 2 ? "[pair512]" : "[pair]");
+  cudaLaunchKernelEx(&cfg, moe::moe_gemm_pair_kernel<MODE, NW>, a, b0, b1, prm);
   return L.end(name, s);
+}
+
+// Launch a pair GEMM over N output columns with expected_mtiles 256-row
+// m-tiles, choosing the tile width: wide (512 accumulator columns) tiles move a
+// quarter fewer operand bytes per FLOP, but give fewer tiles and cannot overlap
+// a whole tile's epilogue with the next tile's MMAs, so automatically they are
+// used for long reductions (at least 64 k-blocks) with at least 3 waves of tiles.
+template <int MODE>
+bool launch_pair_auto(Launcher& L, cudaStream_t s, const char* name, const CUtensorMap& a,
+                      const CUtensorMap& b0, const CUtensorMap& b1, moe::GemmParams prm,
+                      int N, int expected_mtiles, int max_mtiles) {
+  const int cols1 = moe::pair_tile_cols(MODE, 1), cols2 = moe::pair_tile_cols(MODE, 2);
+  const int nt2 = (N + cols2 - 1) / cols2;
+  bool wide = L.p->wide_tiles > 0;
+  if (L.p->wide_tiles < 0)
+    wide = prm.K >= 64 * moe::kBK &&
+           static_cast<long long>(expected_mtiles) * nt2 >= 3LL * (L.p->num_sms / 2);
+  if (wide) {
+    prm.n_tiles = nt2;
+    return launch_gemm_pair<MODE, 2>(L, s, name, a, b0, b1, prm, max_mtiles * nt2);
+  }
+  prm.n_tiles = (N + cols1 - 1) / cols1;
+  return launch_gemm_pair<MODE, 1>(L, s, name, a, b0, b1, prm, max_mtiles * prm.n_tiles);
 }
 
 template <int MODE>
@@ -253,15 +284,19 @@ bool launch_gemm(Launcher& L, cudaStream_t s, const char* name, const CUtensorMa
   return L.end(name, s);
 }
 
+typedef cudaFuncAttribute cudaAttr;
+
 int set_kernel_attributes() {
-  const size_t smem_pair = moe::gemm_pair_smem_bytes(moe::kMaxRouted);
-  const cudaError_t ep[3] = {
-      cudaFuncSetAttribute(moe::moe_gemm_pair_kernel<moe::kEpiSwiGLU>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_pair)),
-      cudaFuncSetAttribute(moe::moe_gemm_pair_kernel<moe::kEpiBF16>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_pair)),
-      cudaFuncSetAttribute(moe::moe_gemm_pair_kernel<moe::kEpiF32>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_pair))};
+  const int sp1 = int(moe::gemm_pair_smem_bytes<1>(moe::kMaxRouted));
+  const int sp2 = int(moe::gemm_pair_smem_bytes<2>(moe::kMaxRouted));
+  const cudaAttr attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  const cudaError_t ep[6] = {
+      cudaFuncSetAttribute(moe::moe_gemm_pair_kernel<moe::kEpiSwiGLU, 1>, attr, sp1),
+      cudaFuncSetAttribute(moe::moe_gemm_pair_kernel<moe::kEpiBF16, 1>, attr, sp1),
+      cudaFuncSetAttribute(moe::moe_gemm_pair_kernel<moe::kEpiF32, 1>, attr, sp1),
+      cudaFuncSetAttribute(moe::moe_gemm_pair_kernel<moe::kEpiSwiGLU, 2>, attr, sp2),
+      cudaFuncSetAttribute(moe::moe_gemm_pair_kernel<moe::kEpiBF16, 2>, attr, sp2),
+      cudaFuncSetAttribute(moe::moe_gemm_pair_kernel<moe::kEpiF32, 2>, attr, sp2)};
   for (cudaError_t e : ep)
     if (e != cudaSuccess)
       return fail(MOE_CUDA_ERROR, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
@@ -346,7 +381,11 @@ int moe_plan_set_option(moe_plan_t p, int option, int64_t value) {
   switch (option) {
     case MOE_OPTION_PAIR_MIN_ROWS:
       if (value < 0) return fail(MOE_INVALID_ARG, "pair_min_rows must be >= 0");
-      p->pair_min_rows = value;
+      p->pair_min_rows_plain = p->pair_min_rows_swiglu = value;
+      return MOE_OK;
+    case MOE_OPTION_WIDE_TILES:
+      if (value < -1 || value > 1) return fail(MOE_INVALID_ARG, "wide_tiles must be -1, 0 or 1");
+      p->wide_tiles = static_cast<int>(value);
       return MOE_OK;
     default:
       return fail(MOE_INVALID_ARG, "unknown option %d", option);
@@ -464,7 +503,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   const bool shared_forked =
       p->n_shared > 0 && shared_mt * ((nsf + 127) / 128) <= p->num_sms / 2;
   cudaStream_t shared_st = shared_forked ? p->side : main_st;
-  const bool shared_pair = static_cast<long long>(T) >= p->pair_min_rows;
+  const bool shared_pair = static_cast<long long>(T) >= p->pair_min_rows_swiglu;
   const int shared_mt2 = static_cast<int>((T + 255) / 256);
   auto launch_shared = [&]() -> int {
     moe::GemmParams g{};
@@ -477,8 +516,8 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.status = status;
     g.k_splits = 1;
     g.kb_per_split = (d + moe::kBK - 1) / moe::kBK;
-    if (shared_pair ? !launch_gemm_pair<moe::kEpiSwiGLU>(L, shared_st, "shared_gate_up", mX, mW1s,
-                                                         mW3s, g, shared_mt2 * g.n_tiles)
+    if (shared_pair ? !launch_pair_auto<moe::kEpiSwiGLU>(L, shared_st, "shared_gate_up", mX, mW1s,
+                                                         mW3s, g, nsf, shared_mt2, shared_mt2)
                     : !launch_gemm<moe::kEpiSwiGLU>(L, shared_st, "shared_gate_up", mX, mW1s, mW3s,
                                                     g, shared_mt * g.n_tiles))
       return L.status;
@@ -492,8 +531,8 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     h.status = status;
     h.k_splits = 1;
     h.kb_per_split = (nsf + moe::kBK - 1) / moe::kBK;
-    if (shared_pair ? !launch_gemm_pair<moe::kEpiF32>(L, shared_st, "shared_down", mHs, mW2s, mW2s,
-                                                      h, shared_mt2 * h.n_tiles)
+    if (shared_pair ? !launch_pair_auto<moe::kEpiF32>(L, shared_st, "shared_down", mHs, mW2s, mW2s,
+                                                      h, d, shared_mt2, shared_mt2)
                     : !launch_gemm<moe::kEpiF32>(L, shared_st, "shared_down", mHs, mW2s, mW2s, h,
                                                  shared_mt * h.n_tiles))
       return L.status;
@@ -573,12 +612,17 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   }
   const int max_mtiles = static_cast<int>((A + 127) / 128 + (A < nr ? A : nr));
   const int max_mtiles2 = static_cast<int>((A + 255) / 256 + (A < nr ? A : nr));
-  const bool routed_pair = A >= p->pair_min_rows * static_cast<long long>(nr);
+  // expected rows per expert against the thresholds (a division: the
+  // thresholds may be huge, and a product with N_r could overflow)
+  const long long rows_per_expert = A / nr;
+  const bool routed_pair_swiglu = rows_per_expert >= p->pair_min_rows_swiglu;
+  const bool routed_pair = rows_per_expert >= p->pair_min_rows_plain;
+  const int expected_mtiles2 = static_cast<int>((A + 255) / 256);
   // 5. grouped gate/up GEMM with the SiLU(gate) * up epilogue
   {
     moe::GemmParams g{};
     g.group_offsets = offsets;
-    g.group_mtiles = routed_pair ? mtiles2 : mtiles;
+    g.group_mtiles = routed_pair_swiglu ? mtiles2 : mtiles;
     g.num_groups = nr;
     g.K = d;
     g.N = f;
@@ -588,8 +632,8 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.status = status;
     g.k_splits = 1;
     g.kb_per_split = (d + moe::kBK - 1) / moe::kBK;
-    if (routed_pair ? !launch_gemm_pair<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1,
-                                                         mW3, g, max_mtiles2 * g.n_tiles)
+    if (routed_pair_swiglu ? !launch_pair_auto<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1,
+                                                         mW3, g, f, expected_mtiles2, max_mtiles2)
                     : !launch_gemm<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1, mW3,
                                                     g, max_mtiles * g.n_tiles))
       return L.status;
@@ -608,8 +652,8 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.status = status;
     g.k_splits = 1;
     g.kb_per_split = (f + moe::kBK - 1) / moe::kBK;
-    if (routed_pair ? !launch_gemm_pair<moe::kEpiBF16>(L, main_st, "grouped_down", mH, mW2, mW2, g,
-                                                       max_mtiles2 * g.n_tiles)
+    if (routed_pair ? !launch_pair_auto<moe::kEpiBF16>(L, main_st, "grouped_down", mH, mW2, mW2, g,
+                                                       d, expected_mtiles2, max_mtiles2)
                     : !launch_gemm<moe::kEpiBF16>(L, main_st, "grouped_down", mH, mW2, mW2, g,
                                                   max_mtiles * g.n_tiles))
       return L.status;

@@ -45,28 +45,45 @@ PAIR_CASES = ["three_tokens", "ragged_17", "two_shared_raw", "ragged_tiles", "k_
               "skewed_groups"]
 
 
+@pytest.mark.parametrize("wide", [0, 1], ids=["pair256", "pair512"])
 @pytest.mark.parametrize("case", [c for c in SMALL if c[0] in PAIR_CASES],
                          ids=[c[0] for c in SMALL if c[0] in PAIR_CASES])
-def test_small_layers_cta_pair_kernel(case):
-    # every GEMM (routed and shared) forced onto the cta_group::2 kernel
+def test_small_layers_cta_pair_kernel(case, wide):
+    # every GEMM (routed and shared) forced onto the cta_group::2 kernel, with
+    # 256- or 512-column tiles
     name, T, d, f, n, k, ns, renorm, bias = case
     shape = LayerShape(name, T, d, f, n, k, ns, renorm, bias)
     inp = make_layer_inputs(shape, seed=4, device="cuda")
-    full_parity(inp, shape, pair_min_rows=0)
+    full_parity(inp, shape, pair_min_rows=0, wide_tiles=wide)
 
 
-@pytest.mark.parametrize("pair_min_rows", [0, 1 << 40])
-def test_pair_and_single_kernels_agree_bitwise(pair_min_rows):
-    # both GEMM kernels accumulate each output in the same k order, so results match exactly
+@pytest.mark.parametrize("pair_min_rows,wide", [(0, 0), (0, 1), (1 << 40, -1)])
+def test_pair_and_single_kernels_agree_bitwise(pair_min_rows, wide):
+    # all GEMM kernels accumulate each output in the same k order, so results match exactly
     from mixture_experts_ffn_expert_b200.layer import MoELayer
     shape = LayerShape("agree", 700, 256, 192, 4, 2, 1, True, "none")
     inp = make_layer_inputs(shape, seed=5, device="cuda")
     ref = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared, True, inp,
                    device="cuda", pair_min_rows=1 << 40)(inp["x"]).clone()
     got = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared, True, inp,
-                   device="cuda", pair_min_rows=pair_min_rows)(inp["x"])
+                   device="cuda", pair_min_rows=pair_min_rows, wide_tiles=wide)(inp["x"])
     torch.cuda.synchronize()
     assert torch.equal(got, ref)
+
+
+def test_default_gemm_variants_on_coarse_shape():
+    # defaults: SwiGLU GEMMs on the single-CTA kernel, the routed down projection
+    # with many rows per expert and a long reduction on wide CTA pairs
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    shape = LayerShape("variants", 8192, 2048, 4096, 8, 2, 0, True, "none")
+    inp = make_layer_inputs(shape, seed=6, device="cuda")
+    layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared, True, inp,
+                     device="cuda")
+    layer(inp["x"])
+    torch.cuda.synchronize()
+    names = layer.plan.kernel_names()
+    assert "grouped_gate_up" in names, names
+    assert "grouped_down[pair512]" in names, names
 
 
 def test_tiny_workload_all_outputs():
