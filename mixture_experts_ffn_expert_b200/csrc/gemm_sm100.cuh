@@ -111,8 +111,6 @@ __device__ __forceinline__ void raise_timeout(volatile int* s_abort, int* status
   atomicExch(status, 6 /* MOE_DEVICE_TIMEOUT */);
 }
 
-__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
