@@ -86,8 +86,13 @@ int moe_last_status(void);
  * MOE_OPTION_WIDE_TILES: CTA-pair tiles of 512 accumulator columns instead of
  *   256 (fewer operand bytes per FLOP, fewer tiles). -1 (default) chooses per
  *   GEMM (wide for reductions of at least 4096 with at least 3 waves of
- *   tiles), 0 never, 1 always. */
-enum { MOE_OPTION_PAIR_MIN_ROWS = 1, MOE_OPTION_WIDE_TILES = 2 };
+ *   tiles), 0 never, 1 always.
+ * MOE_OPTION_MERGE_SHARED: when the shared expert runs on the main stream and a
+ *   routed GEMM runs one CTA per tile, compute the matching shared GEMM as extra
+ *   tiles of that same launch, spread evenly among the routed tiles (0, the
+ *   default: never; 1: whenever possible). Off by default because the merged
+ *   launches measured slower on B200 for the DeepSeek-style layer shapes. */
+enum { MOE_OPTION_PAIR_MIN_ROWS = 1, MOE_OPTION_WIDE_TILES = 2, MOE_OPTION_MERGE_SHARED = 3 };
 int moe_plan_set_option(moe_plan_t plan, int option, int64_t value);
 
 /* Optional per-expert logit bias: device pointer to N_r fp32 values added to

@@ -67,6 +67,14 @@ struct GemmParams {
   int k_splits;              // split-K factor (fp32 epilogue only; 1 elsewhere): split s
   int kb_per_split;          //   covers k-blocks [s*kb_per_split, ...) and writes its
   long long split_stride;    //   partial sums at out + s*split_stride
+  // Optional extra dense problem run by the same launch (the shared expert):
+  // x_tiles tiles spread evenly among the grouped tiles, A/B from the kernel's
+  // second set of tensor maps.
+  int x_tiles;               // 0: none
+  int x_rows, x_K, x_N;
+  void* x_out;
+  long long x_ldo;
+  int x_out_f32;             // plain epilogue: store fp32 instead of bf16
 };
 
 // Dynamic shared memory the kernel needs for a given number of groups.
@@ -106,6 +114,35 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, const int* s_off, con
   return c;
 }
 
+// Tile t of a launch that may carry an extra dense problem: the X extra tiles
+// sit at positions floor(i*total/X) of the combined list (so they are spread
+// evenly over time and over SMs), the grouped tiles fill the others in order.
+__device__ __forceinline__ TileCoord decode_tile_mixed(int tile, const int* s_off, const int* s_mp,
+                                                       int num_groups, const GemmParams& P,
+                                                       int grouped_tiles, bool& extra) {
+  if (P.x_tiles > 0) {
+    const long long total = static_cast<long long>(grouped_tiles) + P.x_tiles;
+    // number of extra positions <= tile
+    const long long cnt = ((static_cast<long long>(tile) + 1) * P.x_tiles + total - 1) / total;
+    const long long i = cnt - 1;
+    if (i >= 0 && (i * total) / P.x_tiles == tile) {
+      extra = true;
+      const int mt = (P.x_rows + kBM - 1) / kBM;
+      TileCoord c;
+      c.group = 0;
+      c.n_blk = static_cast<int>(i / mt);
+      c.row0 = static_cast<int>(i % mt) * kBM;
+      c.rows = min(kBM, P.x_rows - c.row0);
+      c.split = 0;
+      c.mtiles = mt;
+      return c;
+    }
+    tile -= static_cast<int>(cnt);
+  }
+  extra = false;
+  return decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles);
+}
+
 __device__ __forceinline__ void raise_timeout(volatile int* s_abort, int* status) {
   *s_abort = 1;
   atomicExch(status, 6 /* MOE_DEVICE_TIMEOUT */);
@@ -115,7 +152,9 @@ __device__ __forceinline__ void raise_timeout(volatile int* s_abort, int* status
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                    const __grid_constant__ CUtensorMap tmB1, const GemmParams P) {
+                    const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmA2,
+                    const __grid_constant__ CUtensorMap tmB0x, const __grid_constant__ CUtensorMap tmB1x,
+                    const GemmParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -150,6 +189,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB0);
     tma_prefetch_desc(&tmB1);
+    if (P.x_tiles > 0) {
+      tma_prefetch_desc(&tmA2);
+      tma_prefetch_desc(&tmB0x);
+      tma_prefetch_desc(&tmB1x);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(s_tmem), kTmemCols);
@@ -174,8 +218,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem_base = *s_tmem;
 
-  const int total_tiles = s_mp[num_groups] * P.n_tiles * P.k_splits;
-  const int num_kb = (P.K + kBK - 1) / kBK;
+  const int grouped_tiles = s_mp[num_groups] * P.n_tiles * P.k_splits;
+  const int total_tiles = grouped_tiles + P.x_tiles;
+  // k-block range of a tile: its split's share (split-K launches carry no extra
+  // problem), else the whole reduction of the tile's problem
+  auto kb_range = [&](const TileCoord& tc, bool ex, int& kb_begin, int& kb_end) {
+    const int nkb = ((ex ? P.x_K : P.K) + kBK - 1) / kBK;
+    kb_begin = P.k_splits > 1 ? tc.split * P.kb_per_split : 0;
+    kb_end = P.k_splits > 1 ? min(nkb, kb_begin + P.kb_per_split) : nkb;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -191,11 +242,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const bool grouped = P.group_offsets != nullptr;
     const uint64_t once = l2_evict_first_policy();
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-      const TileCoord tc = decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles);
-      const int z = P.group_offsets ? tc.group : 0;
-      const bool stream = grouped && tc.mtiles == 1;
-      const int kb_begin = tc.split * P.kb_per_split;
-      const int kb_end = min(num_kb, kb_begin + P.kb_per_split);
+      bool ex;
+      const TileCoord tc = decode_tile_mixed(tile, s_off, s_mp, num_groups, P, grouped_tiles, ex);
+      const int z = (P.group_offsets && !ex) ? tc.group : 0;
+      const bool stream = grouped && !ex && tc.mtiles == 1;
+      const CUtensorMap* mA = ex ? &tmA2 : &tmA;
+      const CUtensorMap* mB0 = ex ? &tmB0x : &tmB0;
+      const CUtensorMap* mB1 = ex ? &tmB1x : &tmB1;
+      int kb_begin, kb_end;
+      kb_range(tc, ex, kb_begin, kb_end);
       for (int kb = kb_begin; kb < kb_end; ++kb) {
         ok = mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, s_abort);
         ok = __all_sync(0xffffffffu, ok);
@@ -209,15 +264,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t b_dst = a_dst + kATileBytes;
           const int k0 = kb * kBK;
           mbar_arrive_expect_tx(fb, kStageBytes);
-          tma_load_2d(a_dst, &tmA, fb, k0, tc.row0);
-          const CUtensorMap* b1 = MODE == kEpiSwiGLU ? &tmB1 : &tmB0;
+          tma_load_2d(a_dst, mA, fb, k0, tc.row0);
+          const CUtensorMap* b1 = MODE == kEpiSwiGLU ? mB1 : mB0;
           const int n0 = MODE == kEpiSwiGLU ? tc.n_blk * 128 : tc.n_blk * 256;
           const int n1 = MODE == kEpiSwiGLU ? n0 : n0 + 128;
           if (stream) {
-            tma_load_3d_hint(b_dst, &tmB0, fb, k0, n0, z, once);
+            tma_load_3d_hint(b_dst, mB0, fb, k0, n0, z, once);
             tma_load_3d_hint(b_dst + kBHalfBytes, b1, fb, k0, n1, z, once);
           } else {
-            tma_load_3d(b_dst, &tmB0, fb, k0, n0, z);
+            tma_load_3d(b_dst, mB0, fb, k0, n0, z);
             tma_load_3d(b_dst + kBHalfBytes, b1, fb, k0, n1, z);
           }
         }
@@ -245,11 +300,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_ph = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-      const TileCoord tc = decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles);
+      bool ex;
+      const TileCoord tc = decode_tile_mixed(tile, s_off, s_mp, num_groups, P, grouped_tiles, ex);
       const uint32_t idesc = tc.rows <= 64 ? idesc64 : idesc128;
-      const int split = tc.split;
-      const int kb_begin = split * P.kb_per_split;
-      const int kb_end = min(num_kb, kb_begin + P.kb_per_split);
+      int kb_begin, kb_end;
+      kb_range(tc, ex, kb_begin, kb_end);
       ok = mbar_wait(smem_u32(&tempty_bar[acc]), acc_ph ^ 1u, s_abort);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -297,7 +352,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t acc_ph = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      const TileCoord tc = decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles);
+      bool ex;
+      const TileCoord tc = decode_tile_mixed(tile, s_off, s_mp, num_groups, P, grouped_tiles, ex);
+      void* const out_base = ex ? P.x_out : P.out;
+      const long long ldo = ex ? P.x_ldo : P.ldo;
+      const int n_valid = ex ? P.x_N : P.N;
+      const bool to_f32 = MODE == kEpiF32 || (ex && P.x_out_f32);
       bool ok = mbar_wait(smem_u32(&tfull_bar[acc]), acc_ph, s_abort);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
@@ -312,10 +372,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const long long grow = static_cast<long long>(tc.row0) + r;
       if (MODE == kEpiSwiGLU) {
         const int col0 = tc.n_blk * 128;
-        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(P.out);
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(out_base);
 #pragma unroll 1
         for (int c = 0; c < 128; c += 32) {
-          if (col0 + c >= P.N) break;              // warp-uniform
+          if (col0 + c >= n_valid) break;              // warp-uniform
           uint32_t g[32], u[32];
           tmem_ld_32cols(tbase + c, g);
           tmem_ld_32cols(tbase + 128 + c, u);
@@ -324,7 +384,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               const int col = col0 + c + v * 8;
-              if (col < P.N) {
+              if (col < n_valid) {
                 uint32_t pk[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -336,7 +396,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                   const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
                   pk[q] = pack_bf16x2(h0, h1);
                 }
-                *reinterpret_cast<uint4*>(out + grow * P.ldo + col) =
+                *reinterpret_cast<uint4*>(out + grow * ldo + col) =
                     make_uint4(pk[0], pk[1], pk[2], pk[3]);
               }
             }
@@ -346,40 +406,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int col0 = tc.n_blk * 256;
 #pragma unroll 1
         for (int c = 0; c < 256; c += 32) {
-          if (col0 + c >= P.N) break;              // warp-uniform
+          if (col0 + c >= n_valid) break;              // warp-uniform
           uint32_t a[32];
           tmem_ld_32cols(tbase + c, a);
           tmem_ld_wait();
           if (!row_ok) continue;
-          if (MODE == kEpiBF16) {
-            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(P.out);
+          if (!to_f32) {
+            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(out_base);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               const int col = col0 + c + v * 8;
-              if (col < P.N) {
+              if (col < n_valid) {
                 uint32_t pk[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
                   pk[q] = pack_bf16x2(__uint_as_float(a[v * 8 + 2 * q]),
                                       __uint_as_float(a[v * 8 + 2 * q + 1]));
-                *reinterpret_cast<uint4*>(out + grow * P.ldo + col) =
+                *reinterpret_cast<uint4*>(out + grow * ldo + col) =
                     make_uint4(pk[0], pk[1], pk[2], pk[3]);
               }
             }
           } else {
-            float* out = reinterpret_cast<float*>(P.out) + tc.split * P.split_stride;
+            float* out = reinterpret_cast<float*>(out_base) + tc.split * P.split_stride;
 #pragma unroll
             for (int v = 0; v < 8; ++v) {
               const int col = col0 + c + v * 4;
-              float* dst = out + grow * P.ldo + col;
-              if (col + 4 <= P.N) {
+              float* dst = out + grow * ldo + col;
+              if (col + 4 <= n_valid) {
                 *reinterpret_cast<float4*>(dst) =
                     make_float4(__uint_as_float(a[v * 4]), __uint_as_float(a[v * 4 + 1]),
                                 __uint_as_float(a[v * 4 + 2]), __uint_as_float(a[v * 4 + 3]));
               } else {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                  if (col + q < P.N) dst[q] = __uint_as_float(a[v * 4 + q]);
+                  if (col + q < n_valid) dst[q] = __uint_as_float(a[v * 4 + q]);
               }
             }
           }

@@ -63,6 +63,11 @@ struct moe_plan {
   long long pair_min_rows_swiglu = 1LL << 62;
   // CTA-pair tiles 512 accumulator columns wide: -1 automatic, 0 never, 1 always
   int wide_tiles = -1;
+  // shared expert as extra tiles of the routed single-CTA GEMM launches (when
+  // it is not forked onto the side stream): 0 never, 1 whenever possible. Off
+  // by default: measured on B200 it ran the merged launches at a lower clock
+  // under the power cap and lost 5% on the DeepSeek-V3 layer shape.
+  int merge_shared = 0;
   int device, num_sms;
   const float* bias = nullptr;
   char* ws = nullptr;
@@ -270,17 +275,22 @@ bool launch_pair_auto(Launcher& L, cudaStream_t s, const char* name, const CUten
   return launch_gemm_pair<MODE, 1>(L, s, name, a, b0, b1, prm, max_mtiles * prm.n_tiles);
 }
 
+// Single-CTA GEMM. x (optional) holds the A, B0, B1 maps of the extra dense
+// problem that prm.x_tiles describes; max_tiles bounds the grouped tiles only.
 template <int MODE>
 bool launch_gemm(Launcher& L, cudaStream_t s, const char* name, const CUtensorMap& a,
                  const CUtensorMap& b0, const CUtensorMap& b1, const moe::GemmParams& prm,
-                 int max_tiles) {
+                 int max_tiles, const CUtensorMap* x = nullptr) {
   const int num_groups = prm.group_offsets ? prm.num_groups : 1;
   const size_t smem = moe::gemm_smem_bytes(num_groups);
-  int grid = max_tiles < L.p->num_sms ? max_tiles : L.p->num_sms;
+  const long long tiles = static_cast<long long>(max_tiles) + (x ? prm.x_tiles : 0);
+  int grid = tiles < L.p->num_sms ? static_cast<int>(tiles) : L.p->num_sms;
   if (grid < 1) grid = 1;
-  L.begin(name, s);
+  moe::GemmParams q = prm;
+  if (!x) q.x_tiles = 0;
+  L.begin(name, s, q.x_tiles > 0 ? "[+shared]" : "");
   launch_pdl(moe::moe_gemm_kernel<MODE>, dim3(grid), dim3(moe::kGemmThreads), smem, s, a, b0,
-             b1, prm);
+             b1, x ? x[0] : a, x ? x[1] : b0, x ? x[2] : b1, q);
   return L.end(name, s);
 }
 
@@ -386,6 +396,10 @@ int moe_plan_set_option(moe_plan_t p, int option, int64_t value) {
     case MOE_OPTION_WIDE_TILES:
       if (value < -1 || value > 1) return fail(MOE_INVALID_ARG, "wide_tiles must be -1, 0 or 1");
       p->wide_tiles = static_cast<int>(value);
+      return MOE_OK;
+    case MOE_OPTION_MERGE_SHARED:
+      if (value < 0 || value > 1) return fail(MOE_INVALID_ARG, "merge_shared must be 0 or 1");
+      p->merge_shared = static_cast<int>(value);
       return MOE_OK;
     default:
       return fail(MOE_INVALID_ARG, "unknown option %d", option);
@@ -505,7 +519,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   cudaStream_t shared_st = shared_forked ? p->side : main_st;
   const bool shared_pair = static_cast<long long>(T) >= p->pair_min_rows_swiglu;
   const int shared_mt2 = static_cast<int>((T + 255) / 256);
-  auto launch_shared = [&]() -> int {
+  auto launch_shared_gate_up = [&]() -> int {
     moe::GemmParams g{};
     g.dense_rows = static_cast<int>(T);
     g.K = d;
@@ -521,6 +535,9 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
                     : !launch_gemm<moe::kEpiSwiGLU>(L, shared_st, "shared_gate_up", mX, mW1s, mW3s,
                                                     g, shared_mt * g.n_tiles))
       return L.status;
+    return MOE_OK;
+  };
+  auto launch_shared_down = [&]() -> int {
     moe::GemmParams h{};
     h.dense_rows = static_cast<int>(T);
     h.K = nsf;
@@ -537,6 +554,10 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
                                                  shared_mt * h.n_tiles))
       return L.status;
     return MOE_OK;
+  };
+  auto launch_shared = [&]() -> int {
+    if (launch_shared_gate_up() != MOE_OK) return L.status;
+    return launch_shared_down();
   };
   if (shared_forked) {
     if (cudaEventRecord(p->fork, main_st) != cudaSuccess ||
@@ -618,6 +639,15 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   const bool routed_pair_swiglu = rows_per_expert >= p->pair_min_rows_swiglu;
   const bool routed_pair = rows_per_expert >= p->pair_min_rows_plain;
   const int expected_mtiles2 = static_cast<int>((A + 255) / 256);
+  // An inline shared expert can instead run as extra dense tiles of the routed
+  // single-CTA launches, spread among the grouped tiles: tensor-bound shared
+  // tiles then overlap the weight streaming of small expert groups, and the
+  // shared GEMMs need no launches (and tails) of their own.
+  const bool merge_ok = p->n_shared > 0 && !shared_forked && !shared_pair && p->merge_shared == 1;
+  const bool merge_gu = merge_ok && !routed_pair_swiglu;
+  const bool merge_dn = merge_gu && !routed_pair;
+  const CUtensorMap xgu[3] = {mX, mW1s, mW3s};
+  const CUtensorMap xdn[3] = {mHs, mW2s, mW2s};
   // 5. grouped gate/up GEMM with the SiLU(gate) * up epilogue
   {
     moe::GemmParams g{};
@@ -632,10 +662,19 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.status = status;
     g.k_splits = 1;
     g.kb_per_split = (d + moe::kBK - 1) / moe::kBK;
+    if (merge_gu) {
+      g.x_tiles = shared_mt * ((nsf + 127) / 128);
+      g.x_rows = static_cast<int>(T);
+      g.x_K = d;
+      g.x_N = nsf;
+      g.x_out = hshared;
+      g.x_ldo = nsf;
+    }
     if (routed_pair_swiglu ? !launch_pair_auto<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1,
                                                          mW3, g, f, expected_mtiles2, max_mtiles2)
                     : !launch_gemm<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1, mW3,
-                                                    g, max_mtiles * g.n_tiles))
+                                                    g, max_mtiles * g.n_tiles,
+                                                    merge_gu ? xgu : nullptr))
       return L.status;
   }
   // 6. grouped down GEMM
@@ -652,15 +691,28 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.status = status;
     g.k_splits = 1;
     g.kb_per_split = (f + moe::kBK - 1) / moe::kBK;
+    if (merge_dn) {
+      g.x_tiles = shared_mt * ((d + 255) / 256);
+      g.x_rows = static_cast<int>(T);
+      g.x_K = nsf;
+      g.x_N = d;
+      g.x_out = yshared;
+      g.x_ldo = d;
+      g.x_out_f32 = 1;
+    }
     if (routed_pair ? !launch_pair_auto<moe::kEpiBF16>(L, main_st, "grouped_down", mH, mW2, mW2, g,
                                                        d, expected_mtiles2, max_mtiles2)
                     : !launch_gemm<moe::kEpiBF16>(L, main_st, "grouped_down", mH, mW2, mW2, g,
-                                                  max_mtiles * g.n_tiles))
+                                                  max_mtiles * g.n_tiles,
+                                                  merge_dn ? xdn : nullptr))
       return L.status;
   }
-  // 7. the shared expert (inline, or joined from the side stream), then the
-  //    weighted combine + shared add with one bf16 rounding
-  if (p->n_shared > 0 && !shared_forked && launch_shared() != MOE_OK) return L.status;
+  // 7. the shared expert (inline, merged, or joined from the side stream), then
+  //    the weighted combine + shared add with one bf16 rounding
+  if (p->n_shared > 0 && !shared_forked) {
+    if (!merge_gu && launch_shared_gate_up() != MOE_OK) return L.status;
+    if (!merge_dn && launch_shared_down() != MOE_OK) return L.status;
+  }
   if (shared_forked && cudaStreamWaitEvent(main_st, p->join, 0) != cudaSuccess)
     return fail(MOE_CUDA_ERROR, "join of the shared-expert stream failed");
   {

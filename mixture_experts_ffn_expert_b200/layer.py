@@ -10,7 +10,8 @@ from typing import Dict, Optional
 
 import torch
 
-from .binding import MOE_OPTION_PAIR_MIN_ROWS, MOE_OPTION_WIDE_TILES, MoEError, Plan
+from .binding import (MOE_OPTION_MERGE_SHARED, MOE_OPTION_PAIR_MIN_ROWS, MOE_OPTION_WIDE_TILES,
+                      MoEError, Plan)
 
 __all__ = ["MoELayer", "MoEError"]
 
@@ -30,7 +31,8 @@ class MoELayer:
     def __init__(self, d: int, f: int, n_routed: int, top_k: int, n_shared: int,
                  renorm: bool, weights: Dict[str, Optional[torch.Tensor]],
                  bias: Optional[torch.Tensor] = None, device=None,
-                 pair_min_rows: Optional[int] = None, wide_tiles: Optional[int] = None):
+                 pair_min_rows: Optional[int] = None, wide_tiles: Optional[int] = None,
+                 merge_shared: Optional[int] = None):
         dev = torch.device(device) if device is not None else torch.device("cuda")
         if dev.type == "cuda" and dev.index is None:
             dev = torch.device("cuda", torch.cuda.current_device())
@@ -43,6 +45,8 @@ class MoELayer:
             self.plan.set_option(MOE_OPTION_PAIR_MIN_ROWS, pair_min_rows)
         if wide_tiles is not None:
             self.plan.set_option(MOE_OPTION_WIDE_TILES, wide_tiles)
+        if merge_shared is not None:
+            self.plan.set_option(MOE_OPTION_MERGE_SHARED, merge_shared)
         self.d, self.f, self.n_routed, self.top_k, self.n_shared = d, f, n_routed, top_k, n_shared
         self.renorm = bool(renorm)
         shapes = {"W_g": (n_routed, d), "W1": (n_routed, f, d), "W3": (n_routed, f, d),

@@ -103,7 +103,7 @@ def check_output(gpu_out: np.ndarray, ref: np.ndarray):
     return rel_l2, max_abs, scale
 
 
-def run_layer(inp, shape, device="cuda", pair_min_rows=None, wide_tiles=None):
+def run_layer(inp, shape, device="cuda", pair_min_rows=None, wide_tiles=None, merge_shared=None):
     """Run the CUDA layer through the C ABI; returns (out (T,d) fp64 numpy, routing dict)."""
     from mixture_experts_ffn_expert_b200.layer import MoELayer
 
@@ -111,7 +111,7 @@ def run_layer(inp, shape, device="cuda", pair_min_rows=None, wide_tiles=None):
                      shape.renorm, {k: inp[k] for k in ("W_g", "W1", "W3", "W2", "W1s",
                                                         "W3s", "W2s")},
                      bias=inp["bias"], device=device, pair_min_rows=pair_min_rows,
-                     wide_tiles=wide_tiles)
+                     wide_tiles=wide_tiles, merge_shared=merge_shared)
     out = layer(inp["x"])
     routing = layer.routing()
     torch.cuda.synchronize()
@@ -119,12 +119,14 @@ def run_layer(inp, shape, device="cuda", pair_min_rows=None, wide_tiles=None):
     return out, routing, layer
 
 
-def full_parity(inp, shape, tokens=None, pair_min_rows=None, wide_tiles=None):
+def full_parity(inp, shape, tokens=None, pair_min_rows=None, wide_tiles=None,
+                merge_shared=None):
     """Routing on all tokens, output on `tokens` (all when None). Returns a summary dict.
     pair_min_rows forces (0) or forbids (huge) the CTA-pair GEMM kernel; wide_tiles
-    forces (1) or forbids (0) its 512-column tiles."""
+    forces (1) or forbids (0) its 512-column tiles; merge_shared forces (1) or
+    forbids (0) the shared expert as extra tiles of the routed GEMM launches."""
     out, routing, layer = run_layer(inp, shape, pair_min_rows=pair_min_rows,
-                                    wide_tiles=wide_tiles)
+                                    wide_tiles=wide_tiles, merge_shared=merge_shared)
     _, idx_ref, n_near = check_routing(inp, routing, shape)
     ref = oracle_out(inp, shape, idx_ref, tokens)
     got = to64(out if tokens is None else out[torch.as_tensor(tokens, device=out.device)])

@@ -71,6 +71,49 @@ def test_pair_and_single_kernels_agree_bitwise(pair_min_rows, wide):
     assert torch.equal(got, ref)
 
 
+MERGE_CASES = [
+    # name, T, d, f, N_r, k, N_s, renorm, bias, expected variant names; the shared
+    # expert is too large for the side stream in all of them
+    ("merged_both", 2048, 256, 640, 32, 2, 2, True, "none",
+     ["grouped_gate_up[+shared]", "grouped_down[+shared]"]),
+    ("merged_ragged", 2000, 320, 576, 40, 3, 3, False, "normal_var0.5",
+     ["grouped_gate_up[+shared]", "grouped_down[+shared]"]),
+    # 256 rows per expert: the routed down projection runs on CTA pairs, so
+    # only the gate/up GEMM carries the shared tiles
+    ("merged_gate_up_only", 2048, 256, 640, 16, 2, 2, True, "none",
+     ["grouped_gate_up[+shared]", "grouped_down[pair]", "shared_down"]),
+]
+
+
+@pytest.mark.parametrize("case", MERGE_CASES, ids=[c[0] for c in MERGE_CASES])
+def test_shared_expert_merged_into_routed_launches(case):
+    name, T, d, f, n, k, ns, renorm, bias, expect = case
+    shape = LayerShape(name, T, d, f, n, k, ns, renorm, bias)
+    inp = make_layer_inputs(shape, seed=7, device="cuda")
+    res = full_parity(inp, shape, merge_shared=1)
+    names = res["layer"].plan.kernel_names()
+    for e in expect:
+        assert e in names, names
+    assert "shared_gate_up" not in names, names
+
+
+@pytest.mark.parametrize("case", MERGE_CASES, ids=[c[0] for c in MERGE_CASES])
+def test_merged_and_separate_shared_expert_agree_bitwise(case):
+    # a merged shared tile runs the same k loop and epilogue as a separate launch
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    name, T, d, f, n, k, ns, renorm, bias, _ = case
+    shape = LayerShape(name, T, d, f, n, k, ns, renorm, bias)
+    inp = make_layer_inputs(shape, seed=8, device="cuda")
+    outs = []
+    for merge in (0, 1):
+        layer = MoELayer(d, f, n, k, ns, renorm, inp, bias=inp["bias"], device="cuda",
+                         merge_shared=merge)
+        outs.append(layer(inp["x"]).clone())
+        torch.cuda.synchronize()
+        assert layer.device_status() == 0
+    assert torch.equal(outs[0], outs[1])
+
+
 def test_default_gemm_variants_on_coarse_shape():
     # defaults: SwiGLU GEMMs on the single-CTA kernel, the routed down projection
     # with many rows per expert and a long reduction on wide CTA pairs
