@@ -87,6 +87,12 @@ __global__ void __launch_bounds__(kRouteThreads)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
 
+    // Selection keys: a NaN score (from NaN or infinite inputs) ranks as -inf,
+    // so the order stays total and every lane agrees on each winner; the
+    // sentinel index of an empty lane loses every tie against a real expert.
+    float key[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) key[i] = v[i] == v[i] ? v[i] : -INFINITY;
     uint32_t taken = 0;
     float sel_sum = 0.0f, my_p = 0.0f;
     int my_e = -1;
@@ -96,8 +102,8 @@ __global__ void __launch_bounds__(kRouteThreads)
 #pragma unroll
       for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;     // ascending within the lane: '>' keeps the lower index
-        if (e < n_routed && !((taken >> i) & 1u) && (v[i] > bv || be == 0x7fffffff)) {
-          bv = v[i];
+        if (e < n_routed && !((taken >> i) & 1u) && (key[i] > bv || be == 0x7fffffff)) {
+          bv = key[i];
           be = e;
         }
       }

@@ -129,6 +129,36 @@ def test_default_gemm_variants_on_coarse_shape():
     assert "grouped_down[pair512]" in names, names
 
 
+def test_non_finite_tokens_keep_routing_in_range():
+    # NaN / infinite activations give NaN router scores; the top-k must still pick
+    # k distinct in-range experts for them (the permutation indexes with these),
+    # and every other token is unaffected
+    from oracle import route_permutation, router_scores, softmax_rows
+    from parity import check_output, oracle_out, reconcile_routing, run_layer, to64
+    T, k, n = 96, 4, 16
+    shape = LayerShape("nonfinite", T, 128, 64, n, k, 1, True, "none")
+    inp = make_layer_inputs(shape, seed=9, device="cuda")
+    x = inp["x"].clone()
+    x[3, 5] = float("nan")
+    x[10, :] = float("inf")
+    x[11, 7] = float("-inf")
+    out, routing, _ = run_layer(dict(inp, x=x), shape)
+    idx = routing["idx"].cpu().numpy().astype(np.int64)
+    assert idx.min() >= 0 and idx.max() < n
+    assert all(len(set(row.tolist())) == k for row in idx)
+    counts, offsets, perm_src, inv_pos = route_permutation(idx, n)
+    np.testing.assert_array_equal(routing["counts"].cpu().numpy(), counts)
+    np.testing.assert_array_equal(routing["offsets"].cpu().numpy(), offsets)
+    np.testing.assert_array_equal(routing["perm_src"].cpu().numpy(), perm_src)
+    np.testing.assert_array_equal(routing["inv_pos"].cpu().numpy(), inv_pos)
+    clean = np.array([t for t in range(T) if t not in (3, 10, 11)])
+    sub = dict(inp, x=x[torch.as_tensor(clean, device=x.device)])
+    p = softmax_rows(router_scores(to64(sub["x"]), to64(inp["W_g"]), None))
+    idx_ref, _ = reconcile_routing(p, idx[clean], k)
+    ref = oracle_out(sub, shape, idx_ref)
+    check_output(to64(out)[clean], ref)
+
+
 def test_tiny_workload_all_outputs():
     shape = WORKLOADS["tiny_t256_d128_f64_e31k7_s1"]
     inp = make_layer_inputs(shape, seed=0, device="cuda")
