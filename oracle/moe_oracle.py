@@ -36,6 +36,12 @@ Readings taken where the pages leave a step open:
 * N_s shared experts are one fused SwiGLU of inner width N_s*f, which equals the
   sum of the N_s separate experts (DSV3 "Official code", "Watch-outs").
 * The routed rows are grouped by expert in ascending (token, slot) order.
+* Capacity (token dropping, WIE glossary "capacity factor / token dropping":
+  each expert has a seat limit per batch, overflow tokens are skipped): with a
+  limit of C seats, an expert keeps the first C (token, slot) pairs routed to it
+  in batch order, i.e. ascending (token, slot); a dropped pair adds nothing to
+  its token's output, the kept gates are not renormalised, and the shared
+  expert still applies to every token.
 
 Every function below is pinned by tests under ``tests/`` against values the
 pages print, closed forms, library routines, or brute force on tiny inputs; the
@@ -241,29 +247,43 @@ def gate_values(p, idx, renorm: bool) -> np.ndarray:
     return g
 
 
-def route_permutation(idx, n_routed: int):
+def route_permutation(idx, n_routed: int, capacity: Optional[int] = None):
     """Group the (token, slot) pairs by expert in stable (token, slot) order.
 
     [DSV3] "How it works": routed outputs are scatter-summed back into the full
     packed batch, so each expert processes the rows of the tokens routed to it.
-    Returns (counts (N_r,), offsets (N_r+1,), perm_src (T*k,), inv_pos (T, k)):
-    expert e owns rows offsets[e] .. offsets[e+1]-1 of the grouped batch, row r
-    of it holds token perm_src[r], and slot j of token t lands in row inv_pos[t, j].
+    Returns (counts (N_r,), offsets (N_r+1,), perm_src (R,), inv_pos (T, k)):
+    counts[e] is the number of pairs routed to expert e; expert e owns rows
+    offsets[e] .. offsets[e+1]-1 of the grouped batch, row r of it holds token
+    perm_src[r], and slot j of token t lands in row inv_pos[t, j].
 
-    Pinned by a brute-force bucket sort and the bijection / sum invariants
-    (tests/test_oracle_routing.py).
+    ``capacity`` (None: unlimited) is the seat limit per expert of [WIE]
+    glossary "capacity factor / token dropping": expert e keeps its first
+    min(counts[e], capacity) pairs in (token, slot) order, the others are
+    dropped (inv_pos -1, no row); offsets then count kept rows and R is their
+    total.
+
+    Pinned by a brute-force bucket sort, the bijection / sum invariants and a
+    seat-by-seat loop for the capacity (tests/test_oracle_routing.py).
     """
     idx = np.asarray(idx, dtype=np.int64)
     T, k = idx.shape
     flat = idx.reshape(-1)
     counts = np.bincount(flat, minlength=n_routed).astype(np.int64)
-    offsets = np.zeros(n_routed + 1, dtype=np.int64)
-    offsets[1:] = np.cumsum(counts)
     # stable sort of the flat (t, j) entries by expert keeps (t, j) order inside a group
     order = np.argsort(flat, kind="stable")
-    perm_src = order // k
-    inv_flat = np.empty(T * k, dtype=np.int64)
-    inv_flat[order] = np.arange(T * k)
+    starts = np.zeros(n_routed, dtype=np.int64)
+    starts[1:] = np.cumsum(counts)[:-1]
+    rank = np.empty(T * k, dtype=np.int64)             # position inside its expert's group
+    rank[order] = np.arange(T * k) - starts[flat[order]]
+    kept = np.ones(T * k, dtype=bool) if capacity is None else rank < capacity
+    kept_counts = counts if capacity is None else np.minimum(counts, capacity)
+    offsets = np.zeros(n_routed + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(kept_counts)
+    order_kept = order[kept[order]]
+    perm_src = order_kept // k
+    inv_flat = np.full(T * k, -1, dtype=np.int64)
+    inv_flat[order_kept] = np.arange(order_kept.size)
     return counts, offsets, perm_src, inv_flat.reshape(T, k)
 
 
@@ -297,7 +317,8 @@ def _expert_getter(experts: ExpertSource):
 
 def moe_layer(x, W_g, bias, experts: ExpertSource, shared, top_k: int, renorm: bool,
               tokens: Optional[Sequence[int]] = None,
-              forced_idx: Optional[np.ndarray] = None) -> dict:
+              forced_idx: Optional[np.ndarray] = None,
+              capacity: Optional[int] = None) -> dict:
     """Forward pass of the layer: shared + sum of gated routed experts, no residual.
 
     [DSV3] eq. (12) without u_t, "Official code": route, run every expert on the
@@ -311,6 +332,8 @@ def moe_layer(x, W_g, bias, experts: ExpertSource, shared, top_k: int, renorm: b
     ``tokens`` restricts the output rows computed (routing always covers all T).
     ``forced_idx`` (T, k) replaces the top-k selection (gates still come from the
     oracle's own probabilities); it is how a second correct selection is scored.
+    ``capacity`` (None: unlimited) is the per-expert seat limit of
+    ``route_permutation``: dropped (token, slot) pairs add nothing.
 
     Returns a dict with p, idx, g, counts, offsets, perm_src, inv_pos, tokens and
     out (len(tokens), d) in fp64. Pinned by the dense brute force on tiny inputs,
@@ -327,7 +350,8 @@ def moe_layer(x, W_g, bias, experts: ExpertSource, shared, top_k: int, renorm: b
         idx = np.asarray(forced_idx, dtype=np.int64)
         assert idx.shape == (T, top_k)
     g = gate_values(p, idx, renorm)
-    counts, offsets, perm_src, inv_pos = route_permutation(idx, n_routed)
+    counts, offsets, perm_src, inv_pos = route_permutation(idx, n_routed, capacity)
+    kept = inv_pos >= 0
 
     rows = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
     out = np.zeros((len(rows), d), dtype=np.float64)
@@ -338,8 +362,9 @@ def moe_layer(x, W_g, bias, experts: ExpertSource, shared, top_k: int, renorm: b
     get = _expert_getter(experts)
     # (row in out, slot) pairs per expert, restricted to the requested tokens
     sel_rows = idx[rows]                                   # (R, k)
+    kept_rows = kept[rows]
     for e in range(n_routed):
-        hit_r, hit_j = np.nonzero(sel_rows == e)
+        hit_r, hit_j = np.nonzero((sel_rows == e) & kept_rows)
         if hit_r.size == 0:
             continue
         W1e, W3e, W2e = get(e)
@@ -350,7 +375,7 @@ def moe_layer(x, W_g, bias, experts: ExpertSource, shared, top_k: int, renorm: b
 
 
 def moe_layer_dense_bruteforce(x, W_g, bias, W1, W3, W2, shared, top_k: int,
-                               renorm: bool) -> np.ndarray:
+                               renorm: bool, capacity: Optional[int] = None) -> np.ndarray:
     """Brute-force evaluation for tiny inputs: every expert on every token.
 
     [SFE] "Why segmentation helps": the layer is sum_{i in S} g_i E_i(x), i.e. a
@@ -358,7 +383,9 @@ def moe_layer_dense_bruteforce(x, W_g, bias, W1, W3, W2, shared, top_k: int,
     selected set. This version uses plain Python loops over scalars (no matrix
     products, no sorting routine) so that it shares no formulation with
     ``moe_layer``: the selection is found by repeatedly taking the first maximum,
-    each expert's SwiGLU is summed element by element.
+    each expert's SwiGLU is summed element by element. With a ``capacity``, the
+    seats are handed out pair by pair in (token, slot) order ([WIE] glossary
+    "capacity factor / token dropping") and a pair without a seat is skipped.
     """
     import math
 
@@ -380,6 +407,7 @@ def moe_layer_dense_bruteforce(x, W_g, bias, W1, W3, W2, shared, top_k: int,
         return [sum(A2[c][i] * h[i] for i in range(inner)) for c in range(d)]
 
     out = np.zeros((T, d), dtype=np.float64)
+    seats_used = [0] * n_routed
     for t in range(T):
         scores = []
         for e in range(n_routed):
@@ -402,7 +430,11 @@ def moe_layer_dense_bruteforce(x, W_g, bias, W1, W3, W2, shared, top_k: int,
             chosen.append(best)
         G = [0.0] * n_routed
         norm = sum(prob[e] for e in chosen) if renorm else 1.0
-        for e in chosen:
+        for e in chosen:                   # slots in order; a full expert skips the pair
+            if capacity is not None:
+                if seats_used[e] >= capacity:
+                    continue
+                seats_used[e] += 1
             G[e] = prob[e] / norm
         acc = [0.0] * d
         for e in range(n_routed):          # dense over all experts

@@ -140,3 +140,24 @@ def test_oracle_on_seeded_tiny_workload_inputs():
     assert np.all(np.isfinite(r["out"]))
     np.testing.assert_allclose(r["g"].sum(1), 1.0, atol=1e-12)
     assert r["idx"].shape == (8, 7) and len(set(map(tuple, np.sort(r["idx"], 1)))) >= 1
+
+
+@pytest.mark.parametrize("capacity", [0, 1, 2, 3])
+def test_capacity_layer_equals_seat_by_seat_bruteforce(capacity):
+    # [WIE] glossary "capacity factor / token dropping": a pair without a seat
+    # is skipped; the brute force hands out seats in plain loops
+    rng = np.random.default_rng(21)
+    T, d, f, n, k, ns = 9, 5, 4, 4, 2, 1
+    x, W_g, b, experts, shared = _tiny(rng, T, d, f, n, ns, bias=True)
+    ref = moe_layer_dense_bruteforce(x, W_g, b, *experts, shared, k, True, capacity=capacity)
+    got = moe_layer(x, W_g, b, experts, shared, k, True, capacity=capacity)["out"]
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_zero_capacity_leaves_only_the_shared_expert():
+    rng = np.random.default_rng(22)
+    x, W_g, b, experts, shared = _tiny(rng, 7, 6, 4, 5, 2)
+    got = moe_layer(x, W_g, b, experts, shared, 2, False, capacity=0)["out"]
+    only_shared = moe_layer(x, W_g, b, tuple(np.zeros_like(a) for a in experts), shared, 2,
+                            False)["out"]
+    np.testing.assert_array_equal(got, only_shared)

@@ -103,3 +103,51 @@ def test_topk_gap_small_example():
     np.testing.assert_allclose(topk_gap(p, 2), [0.15, 0.0])
     np.testing.assert_allclose(topk_gap(p, 1), [0.2, 0.1])
     assert np.all(np.isinf(topk_gap(np.ones((2, 1)), 1)))
+
+
+def _seat_loop(idx, n, capacity):
+    """Seats handed out pair by pair in (token, slot) order ([WIE] glossary
+    "capacity factor / token dropping"): returns kept mask and, per expert, the
+    tokens of its kept pairs in order."""
+    used = [0] * n
+    rows = [[] for _ in range(n)]
+    T, k = idx.shape
+    kept = np.zeros((T, k), dtype=bool)
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            if used[e] < capacity:
+                used[e] += 1
+                kept[t, j] = True
+                rows[e].append(t)
+    return kept, rows
+
+
+@pytest.mark.parametrize("capacity", [0, 1, 2, 5, 1000])
+def test_capacity_keeps_the_first_pairs_in_batch_order(capacity):
+    rng = np.random.default_rng(11)
+    T, k, n = 60, 3, 7
+    # skewed routing so that some experts overflow
+    p = rng.dirichlet(np.linspace(4.0, 0.3, n), size=T)
+    idx = select_topk(p, k)
+    counts, offsets, perm_src, inv_pos = route_permutation(idx, n, capacity)
+    kept, rows = _seat_loop(idx, n, capacity)
+    np.testing.assert_array_equal(counts, np.bincount(idx.reshape(-1), minlength=n))
+    np.testing.assert_array_equal(inv_pos >= 0, kept)
+    np.testing.assert_array_equal(np.diff(offsets), [len(r) for r in rows])
+    np.testing.assert_array_equal(perm_src, [t for r in rows for t in r])
+    assert offsets[-1] == min(T * k, sum(min(c, capacity) for c in counts))
+    # kept pairs land on distinct rows of their expert's group, in (t, j) order
+    for e in range(n):
+        sel = [(t, j) for t in range(T) for j in range(k) if idx[t, j] == e and kept[t, j]]
+        np.testing.assert_array_equal([inv_pos[t, j] for t, j in sel],
+                                      np.arange(offsets[e], offsets[e + 1]))
+
+
+def test_capacity_at_or_above_the_largest_load_drops_nothing():
+    rng = np.random.default_rng(12)
+    idx = select_topk(rng.random((40, 6)), 2)
+    free = route_permutation(idx, 6)
+    capped = route_permutation(idx, 6, int(np.bincount(idx.reshape(-1)).max()))
+    for a, b in zip(free, capped):
+        np.testing.assert_array_equal(a, b)
