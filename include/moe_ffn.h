@@ -91,8 +91,22 @@ int moe_last_status(void);
  *   routed GEMM runs one CTA per tile, compute the matching shared GEMM as extra
  *   tiles of that same launch, spread evenly among the routed tiles (0, the
  *   default: never; 1: whenever possible). Off by default because the merged
- *   launches measured slower on B200 for the DeepSeek-style layer shapes. */
-enum { MOE_OPTION_PAIR_MIN_ROWS = 1, MOE_OPTION_WIDE_TILES = 2, MOE_OPTION_MERGE_SHARED = 3 };
+ *   launches measured slower on B200 for the DeepSeek-style layer shapes.
+ * MOE_OPTION_EXPERT_CAPACITY: seats per expert per forward ("What is an
+ *   'expert,' really?", glossary: capacity factor / token dropping, each expert
+ *   has a seat limit per batch and overflow tokens are skipped). 0 (default):
+ *   unlimited, the layer is dropless. C > 0: expert e keeps the first
+ *   min(count_e, C) of the (token, slot) pairs routed to it, in ascending
+ *   (token, slot) order; a dropped pair adds nothing to its token's output, the
+ *   kept gates are not renormalised and the shared expert still applies. This
+ *   option changes results; the others do not. A capacity factor cf maps to
+ *   C = ceil(cf * T * top_k / N_r). */
+enum {
+  MOE_OPTION_PAIR_MIN_ROWS = 1,
+  MOE_OPTION_WIDE_TILES = 2,
+  MOE_OPTION_MERGE_SHARED = 3,
+  MOE_OPTION_EXPERT_CAPACITY = 4
+};
 int moe_plan_set_option(moe_plan_t plan, int option, int64_t value);
 
 /* Optional per-expert logit bias: device pointer to N_r fp32 values added to
@@ -125,15 +139,19 @@ int moe_forward(moe_plan_t plan, int64_t T, const moe_bf16_t* x,
 /* Copy the routing of the last forward (device to device, enqueued on
  * `stream`): idx (T, top_k) int32 expert ids in slot order (descending
  * probability, ties to the lower index); w (T, top_k) fp32 gates; counts (N_r)
- * int32 rows per expert; offsets (N_r+1) int32 exclusive prefix of counts.
- * Any output may be NULL. T must equal the last forward's T. */
+ * int32 (token, slot) pairs routed to each expert; offsets (N_r+1) int32
+ * exclusive prefix of the rows each expert kept (of counts, unless an expert
+ * capacity dropped pairs). Any output may be NULL. T must equal the last
+ * forward's T. */
 int moe_get_routing(moe_plan_t plan, int64_t T, int32_t* idx, float* w,
                     int32_t* counts, int32_t* offsets, void* stream);
 
 /* Copy the stable permutation of the last forward (device to device):
  * perm_src (T*top_k) int32 token of each grouped row (rows of expert e are
- * offsets[e]..offsets[e+1]-1, in ascending (token, slot) order);
- * inv_pos (T, top_k) int32 grouped row of each (token, slot). NULL skips. */
+ * offsets[e]..offsets[e+1]-1, in ascending (token, slot) order; entries past
+ * offsets[N_r] are unspecified when pairs were dropped);
+ * inv_pos (T, top_k) int32 grouped row of each (token, slot), -1 for a pair
+ * dropped by the expert capacity. NULL skips. */
 int moe_get_permutation(moe_plan_t plan, int64_t T, int32_t* perm_src,
                         int32_t* inv_pos, void* stream);
 

@@ -7,6 +7,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -68,6 +69,8 @@ struct moe_plan {
   // by default: measured on B200 it ran the merged launches at a lower clock
   // under the power cap and lost 5% on the DeepSeek-V3 layer shape.
   int merge_shared = 0;
+  // seats per expert per forward (token dropping); 0: unlimited (dropless)
+  int64_t capacity = 0;
   int device, num_sms;
   const float* bias = nullptr;
   char* ws = nullptr;
@@ -401,6 +404,10 @@ int moe_plan_set_option(moe_plan_t p, int option, int64_t value) {
       if (value < 0 || value > 1) return fail(MOE_INVALID_ARG, "merge_shared must be 0 or 1");
       p->merge_shared = static_cast<int>(value);
       return MOE_OK;
+    case MOE_OPTION_EXPERT_CAPACITY:
+      if (value < 0) return fail(MOE_INVALID_ARG, "expert capacity must be >= 0");
+      p->capacity = value;
+      return MOE_OK;
     default:
       return fail(MOE_INVALID_ARG, "unknown option %d", option);
   }
@@ -620,13 +627,16 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
                0, main_st, chunk_counts, Lw.n_chunks, nr, counts);
     if (!L.end("route_scan", main_st)) return L.status;
   }
-  // 4. offsets + m-tile prefix, stable permutation, 16-byte row copies
+  // 4. offsets + m-tile prefix, stable permutation, 16-byte row copies (with a
+  //    seat limit, only each expert's first `capacity` pairs get rows)
+  const int seat_limit =
+      p->capacity > 0 && p->capacity < INT_MAX ? static_cast<int>(p->capacity) : INT_MAX;
   {
     const size_t smem = size_t(moe::kMaxRouted + nr) * 4 + size_t(2) * Lw.tpc * k * 4;
     L.begin("route_scatter", main_st);
     launch_pdl(moe::route_scatter_kernel, dim3(Lw.n_chunks), dim3(moe::kRouteThreads), smem,
                main_st, (const int*)idx, (const int*)chunk_counts, (const int*)counts,
-               static_cast<int>(T), k, nr, Lw.tpc, Lw.n_chunks, moe::kBM,
+               static_cast<int>(T), k, nr, Lw.tpc, Lw.n_chunks, moe::kBM, seat_limit,
                reinterpret_cast<const uint4*>(x), d / 8, reinterpret_cast<uint4*>(xperm),
                perm_src, inv_pos, offsets, mtiles, mtiles2);
     if (!L.end("route_scatter", main_st)) return L.status;
@@ -635,7 +645,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   const int max_mtiles2 = static_cast<int>((A + 255) / 256 + (A < nr ? A : nr));
   // expected rows per expert against the thresholds (a division: the
   // thresholds may be huge, and a product with N_r could overflow)
-  const long long rows_per_expert = A / nr;
+  const long long rows_per_expert = A / nr < seat_limit ? A / nr : seat_limit;
   const bool routed_pair_swiglu = rows_per_expert >= p->pair_min_rows_swiglu;
   const bool routed_pair = rows_per_expert >= p->pair_min_rows_plain;
   const int expected_mtiles2 = static_cast<int>((A + 255) / 256);

@@ -209,13 +209,18 @@ __device__ __forceinline__ int block_exclusive_scan(int* s, int n, int* tmp) {
 // staged in shared memory by all threads; warp 0 then ranks the (token, slot)
 // entries in order with match-any, so rows inside an expert group follow
 // ascending (t, j); every warp then copies token rows (d_vec 16-byte vectors
-// each) to their k rows, four vectors in flight per lane.
+// each) to their k rows, four vectors in flight per lane. With a seat limit
+// (capacity; INT_MAX when unlimited) an expert keeps its first `capacity` pairs
+// in that order ("What is an expert, really?" glossary, capacity factor / token
+// dropping): offsets and m-tiles count kept rows, a dropped pair gets inv_pos
+// -1 and no row.
 constexpr int kCopyUnroll = 4;
 
 __global__ void __launch_bounds__(kRouteThreads)
     route_scatter_kernel(const int* __restrict__ idx, const int* __restrict__ chunk_base,
                          const int* __restrict__ counts, int T, int top_k, int n_routed,
-                         int tpc, int n_chunks, int tile_rows, const uint4* __restrict__ x,
+                         int tpc, int n_chunks, int tile_rows, int capacity,
+                         const uint4* __restrict__ x,
                          int d_vec, uint4* __restrict__ xperm, int* __restrict__ perm_src,
                          int* __restrict__ inv_pos, int* __restrict__ offsets_out,
                          int* __restrict__ mtiles_out, int* __restrict__ mtiles2_out) {
@@ -237,8 +242,9 @@ __global__ void __launch_bounds__(kRouteThreads)
     s_e[i] = e;
     s_pos[i] = chunk_base[static_cast<long long>(e) * n_chunks + chunk];
   }
+  // an expert keeps at most `capacity` rows: its first pairs in (token, slot) order
   for (int e = threadIdx.x; e < n_routed; e += blockDim.x) {
-    s_off[e] = counts[e];
+    s_off[e] = min(counts[e], capacity);
     s_run[e] = 0;
   }
   __syncthreads();
@@ -253,7 +259,7 @@ __global__ void __launch_bounds__(kRouteThreads)
       int* dst = pass ? mtiles2_out : mtiles_out;
       __syncthreads();
       for (int e = threadIdx.x; e < n_routed; e += blockDim.x)
-        s_run[e] = (counts[e] + rows - 1) / rows;
+        s_run[e] = (min(counts[e], capacity) + rows - 1) / rows;
       __syncthreads();
       const int total_mt = block_exclusive_scan(s_run, n_routed, s_tmp);
       for (int e = threadIdx.x; e < n_routed; e += blockDim.x) {
@@ -273,7 +279,10 @@ __global__ void __launch_bounds__(kRouteThreads)
       const int e = valid ? s_e[i] : -1;
       const uint32_t same = __match_any_sync(0xffffffffu, e);
       const int rank = __popc(same & ((1u << lane) - 1u));
-      if (valid) s_pos[i] += s_off[e] + s_run[e] + rank;
+      if (valid) {
+        const int r = s_pos[i] + s_run[e] + rank;   // place among the expert's pairs
+        s_pos[i] = r < capacity ? s_off[e] + r : -1;  // -1: dropped, no seat left
+      }
       __syncwarp();
       if (valid && lane == 31 - __clz(same)) s_run[e] += __popc(same);
       __syncwarp();
@@ -283,7 +292,7 @@ __global__ void __launch_bounds__(kRouteThreads)
   for (int i = threadIdx.x; i < n_ent; i += blockDim.x) {
     const int pos = s_pos[i];
     inv_pos[ebase + i] = pos;
-    perm_src[pos] = t0 + i / top_k;
+    if (pos >= 0) perm_src[pos] = t0 + i / top_k;
   }
   for (int tl = warp; tl < ntok; tl += kRouteThreads / 32) {
     const uint4* src = x + static_cast<long long>(t0 + tl) * d_vec;
@@ -294,6 +303,7 @@ __global__ void __launch_bounds__(kRouteThreads)
       for (int u = 0; u < kCopyUnroll; ++u)
         if (v0 + 32 * u < d_vec) val[u] = src[v0 + 32 * u];
       for (int j = 0; j < top_k; ++j) {
+        if (pos[j] < 0) continue;
         uint4* dst = xperm + static_cast<long long>(pos[j]) * d_vec;
 #pragma unroll
         for (int u = 0; u < kCopyUnroll; ++u)
@@ -326,7 +336,8 @@ constexpr int kCombineCols = kCombineThreads * kCombineVec;
 // Grid (T, ceil(d_vec / 512)): block = one token and 512 16-byte column vectors,
 // four per thread (strided by 128 so each load instruction is coalesced), all
 // k routed rows of a vector loaded before its FMAs. shared (fp32, (T, d)) may
-// be null when N_s = 0. The slots are added in order after the shared term.
+// be null when N_s = 0. The slots are added in order after the shared term; a
+// dropped slot (inv_pos -1) adds nothing.
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const uint4* __restrict__ Y, const float* __restrict__ shared,
                    const int* __restrict__ inv_pos, const float* __restrict__ gate, int top_k,
@@ -363,14 +374,14 @@ __global__ void __launch_bounds__(kCombineThreads)
 #pragma unroll
       for (int u = 0; u < kCombineVec; ++u) {
         const int v = v0 + u * kCombineThreads;
-        if (j0 + jj < top_k && v < d_vec)
+        if (j0 + jj < top_k && v < d_vec && s_pos[j0 + jj] >= 0)
           y[jj][u] = Y[static_cast<long long>(s_pos[j0 + jj]) * d_vec + v];
       }
 #pragma unroll
     for (int jj = 0; jj < kCombineBatch; ++jj)
 #pragma unroll
       for (int u = 0; u < kCombineVec; ++u)
-        if (j0 + jj < top_k) bf16x8_fma(acc[u], y[jj][u], s_w[j0 + jj]);
+        if (j0 + jj < top_k && s_pos[j0 + jj] >= 0) bf16x8_fma(acc[u], y[jj][u], s_w[j0 + jj]);
   }
 #pragma unroll
   for (int u = 0; u < kCombineVec; ++u) {

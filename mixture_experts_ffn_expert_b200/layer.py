@@ -6,14 +6,25 @@ libmoe_ffn.so. A missing library raises instead of falling back to anything.
 """
 from __future__ import annotations
 
+import math
 from typing import Dict, Optional
 
 import torch
 
-from .binding import (MOE_OPTION_MERGE_SHARED, MOE_OPTION_PAIR_MIN_ROWS, MOE_OPTION_WIDE_TILES,
-                      MoEError, Plan)
+from .binding import (MOE_OPTION_EXPERT_CAPACITY, MOE_OPTION_MERGE_SHARED,
+                      MOE_OPTION_PAIR_MIN_ROWS, MOE_OPTION_WIDE_TILES, MoEError, Plan)
 
-__all__ = ["MoELayer", "MoEError"]
+__all__ = ["MoELayer", "MoEError", "capacity_from_factor"]
+
+
+def capacity_from_factor(factor: float, T: int, top_k: int, n_routed: int) -> int:
+    """Seats per expert for a capacity factor: ceil(factor * T * top_k / N_r), the
+    factor times an expert's share of the batch's T*top_k routed pairs (at
+    least 1). This is the conventional reading of the "capacity factor" of the
+    "What is an expert, really?" glossary, which names it without a formula."""
+    if factor <= 0:
+        raise MoEError(2, "capacity factor must be positive")
+    return max(1, math.ceil(factor * T * top_k / n_routed))
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -25,14 +36,16 @@ class MoELayer:
 
     ``weights`` holds W_g (N_r, d), W1, W3 (N_r, f, d), W2 (N_r, d, f) and, when
     n_shared > 0, W1s, W3s (N_s*f, d), W2s (d, N_s*f), all bf16 contiguous on
-    the device; ``bias`` is an optional fp32 (N_r,) logit bias.
+    the device; ``bias`` is an optional fp32 (N_r,) logit bias. ``capacity``
+    (seats per expert per forward, see ``capacity_from_factor``) turns on token
+    dropping; the other options only select kernels.
     """
 
     def __init__(self, d: int, f: int, n_routed: int, top_k: int, n_shared: int,
                  renorm: bool, weights: Dict[str, Optional[torch.Tensor]],
                  bias: Optional[torch.Tensor] = None, device=None,
                  pair_min_rows: Optional[int] = None, wide_tiles: Optional[int] = None,
-                 merge_shared: Optional[int] = None):
+                 merge_shared: Optional[int] = None, capacity: Optional[int] = None):
         dev = torch.device(device) if device is not None else torch.device("cuda")
         if dev.type == "cuda" and dev.index is None:
             dev = torch.device("cuda", torch.cuda.current_device())
@@ -47,6 +60,10 @@ class MoELayer:
             self.plan.set_option(MOE_OPTION_WIDE_TILES, wide_tiles)
         if merge_shared is not None:
             self.plan.set_option(MOE_OPTION_MERGE_SHARED, merge_shared)
+        # seats per expert per forward (token dropping); None or 0: dropless
+        self.capacity = capacity or 0
+        if capacity:
+            self.plan.set_option(MOE_OPTION_EXPERT_CAPACITY, capacity)
         self.d, self.f, self.n_routed, self.top_k, self.n_shared = d, f, n_routed, top_k, n_shared
         self.renorm = bool(renorm)
         shapes = {"W_g": (n_routed, d), "W1": (n_routed, f, d), "W3": (n_routed, f, d),

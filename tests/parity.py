@@ -51,16 +51,17 @@ def reconcile_routing(p: np.ndarray, gpu_idx: np.ndarray, k: int, tol: float = T
     return idx_ref, int(near.sum())
 
 
-def check_routing(inp, gpu, shape, T=None):
-    """Routing parity on every token. Returns (p, idx_ref, n_near_tie)."""
+def check_routing(inp, gpu, shape, T=None, capacity=None):
+    """Routing parity on every token. Returns (p, idx_ref, n_near_tie). With an
+    expert capacity only the kept rows of perm_src are defined."""
     x = to64(inp["x"])
     p = softmax_rows(router_scores(x, to64(inp["W_g"]), to64(inp["bias"])))
     gpu_idx = gpu["idx"].cpu().numpy().astype(np.int64)
     idx_ref, n_near = reconcile_routing(p, gpu_idx, shape.top_k)
-    counts, offsets, perm_src, inv_pos = route_permutation(idx_ref, shape.n_routed)
+    counts, offsets, perm_src, inv_pos = route_permutation(idx_ref, shape.n_routed, capacity)
     np.testing.assert_array_equal(gpu["counts"].cpu().numpy(), counts)
     np.testing.assert_array_equal(gpu["offsets"].cpu().numpy(), offsets)
-    np.testing.assert_array_equal(gpu["perm_src"].cpu().numpy(), perm_src)
+    np.testing.assert_array_equal(gpu["perm_src"].cpu().numpy()[:perm_src.size], perm_src)
     np.testing.assert_array_equal(gpu["inv_pos"].cpu().numpy(), inv_pos)
     g = np.take_along_axis(p, idx_ref, 1)
     if shape.renorm:
@@ -71,7 +72,7 @@ def check_routing(inp, gpu, shape, T=None):
     return p, idx_ref, n_near
 
 
-def oracle_out(inp, shape, idx_ref, tokens=None):
+def oracle_out(inp, shape, idx_ref, tokens=None, capacity=None):
     """Oracle output for `tokens` (all when None), streaming one expert at a time."""
     W1, W3, W2 = inp["W1"], inp["W3"], inp["W2"]
 
@@ -82,7 +83,8 @@ def oracle_out(inp, shape, idx_ref, tokens=None):
     if shape.n_shared > 0:
         shared = (to64(inp["W1s"]), to64(inp["W3s"]), to64(inp["W2s"]))
     r = moe_layer(to64(inp["x"]), to64(inp["W_g"]), to64(inp["bias"]), expert, shared,
-                  shape.top_k, shape.renorm, tokens=tokens, forced_idx=idx_ref)
+                  shape.top_k, shape.renorm, tokens=tokens, forced_idx=idx_ref,
+                  capacity=capacity)
     return r["out"]
 
 
@@ -103,7 +105,8 @@ def check_output(gpu_out: np.ndarray, ref: np.ndarray):
     return rel_l2, max_abs, scale
 
 
-def run_layer(inp, shape, device="cuda", pair_min_rows=None, wide_tiles=None, merge_shared=None):
+def run_layer(inp, shape, device="cuda", pair_min_rows=None, wide_tiles=None, merge_shared=None,
+              capacity=None):
     """Run the CUDA layer through the C ABI; returns (out (T,d) fp64 numpy, routing dict)."""
     from mixture_experts_ffn_expert_b200.layer import MoELayer
 
@@ -111,7 +114,7 @@ def run_layer(inp, shape, device="cuda", pair_min_rows=None, wide_tiles=None, me
                      shape.renorm, {k: inp[k] for k in ("W_g", "W1", "W3", "W2", "W1s",
                                                         "W3s", "W2s")},
                      bias=inp["bias"], device=device, pair_min_rows=pair_min_rows,
-                     wide_tiles=wide_tiles, merge_shared=merge_shared)
+                     wide_tiles=wide_tiles, merge_shared=merge_shared, capacity=capacity)
     out = layer(inp["x"])
     routing = layer.routing()
     torch.cuda.synchronize()
@@ -120,15 +123,17 @@ def run_layer(inp, shape, device="cuda", pair_min_rows=None, wide_tiles=None, me
 
 
 def full_parity(inp, shape, tokens=None, pair_min_rows=None, wide_tiles=None,
-                merge_shared=None):
+                merge_shared=None, capacity=None):
     """Routing on all tokens, output on `tokens` (all when None). Returns a summary dict.
     pair_min_rows forces (0) or forbids (huge) the CTA-pair GEMM kernel; wide_tiles
     forces (1) or forbids (0) its 512-column tiles; merge_shared forces (1) or
-    forbids (0) the shared expert as extra tiles of the routed GEMM launches."""
+    forbids (0) the shared expert as extra tiles of the routed GEMM launches;
+    capacity sets the seats per expert (token dropping)."""
     out, routing, layer = run_layer(inp, shape, pair_min_rows=pair_min_rows,
-                                    wide_tiles=wide_tiles, merge_shared=merge_shared)
-    _, idx_ref, n_near = check_routing(inp, routing, shape)
-    ref = oracle_out(inp, shape, idx_ref, tokens)
+                                    wide_tiles=wide_tiles, merge_shared=merge_shared,
+                                    capacity=capacity)
+    _, idx_ref, n_near = check_routing(inp, routing, shape, capacity=capacity)
+    ref = oracle_out(inp, shape, idx_ref, tokens, capacity=capacity)
     got = to64(out if tokens is None else out[torch.as_tensor(tokens, device=out.device)])
     rel_l2, max_abs, scale = check_output(got, ref)
     return {"near_ties": n_near, "rel_l2": rel_l2, "max_abs": max_abs, "max_ref": scale,

@@ -85,3 +85,23 @@ def test_valid_plan_without_gpu_fails_loudly(lib):
         pytest.skip("a GPU is present")
     assert not lib.moe_plan_create(128, 64, 31, 7, 1, 1)
     assert lib.moe_last_status() == 4
+
+
+def test_capacity_from_factor():
+    # seats = ceil(factor * T * k / N_r), at least one
+    from mixture_experts_ffn_expert_b200.layer import MoEError, capacity_from_factor
+    assert capacity_from_factor(1.0, 4096, 8, 256) == 128
+    assert capacity_from_factor(1.25, 4096, 8, 256) == 160
+    assert capacity_from_factor(1.0, 100, 3, 7) == 43          # 300 / 7 = 42.86
+    assert capacity_from_factor(0.001, 10, 1, 64) == 1
+    with pytest.raises(MoEError):
+        capacity_from_factor(0.0, 10, 1, 4)
+
+
+def test_option_ids_match_the_header():
+    import mixture_experts_ffn_expert_b200.binding as B
+    hdr = open(os.path.join(os.path.dirname(__file__), "..", "include", "moe_ffn.h")).read()
+    found = dict(re.findall(r"(MOE_OPTION_[A-Z_]+)\s*=\s*(\d+)", hdr))
+    assert found, "no option ids in the header"
+    for name, value in found.items():
+        assert getattr(B, name) == int(value), name

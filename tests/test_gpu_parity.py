@@ -183,6 +183,44 @@ def test_full_size_workloads(name, n_tokens):
     torch.cuda.empty_cache()
 
 
+CAPACITY_CASES = [
+    # name, T, d, f, N_r, k, N_s, renorm, bias, seats per expert, pair_min_rows
+    ("cap_one_seat", 200, 128, 64, 16, 2, 1, True, "none", 1, None),
+    ("cap_skewed", 1000, 256, 128, 64, 6, 1, True, "zipf1.1", 64, None),
+    ("cap_all_overflow_raw", 600, 384, 320, 6, 2, 1, False, "none", 150, None),
+    ("cap_pairs", 600, 384, 320, 6, 2, 1, True, "normal_var0.5", 170, 0),
+    ("cap_no_drop", 300, 128, 64, 8, 2, 0, True, "none", 10000, None),
+]
+
+
+@pytest.mark.parametrize("case", CAPACITY_CASES, ids=[c[0] for c in CAPACITY_CASES])
+def test_expert_capacity_drops_the_later_pairs(case):
+    # "What is an expert, really?" glossary, capacity factor / token dropping
+    name, T, d, f, n, k, ns, renorm, bias, cap, pmr = case
+    shape = LayerShape(name, T, d, f, n, k, ns, renorm, bias)
+    inp = make_layer_inputs(shape, seed=10, device="cuda")
+    res = full_parity(inp, shape, capacity=cap, pair_min_rows=pmr)
+    r = res["layer"].routing()
+    counts = r["counts"].cpu().numpy()
+    dropped = int((r["inv_pos"].cpu().numpy() < 0).sum())
+    assert dropped == int(np.maximum(counts - cap, 0).sum())
+    assert int(r["offsets"][-1]) == T * k - dropped
+
+
+def test_capacity_from_factor_on_the_deepseek_v3_shape():
+    from mixture_experts_ffn_expert_b200.layer import capacity_from_factor
+    shape = WORKLOADS["dsv3_prefill_t4096_d7168_f2048_e256k8_s1"]
+    inp = make_layer_inputs(shape, seed=0, device="cuda")
+    cap = capacity_from_factor(1.0, shape.T, shape.top_k, shape.n_routed)
+    assert cap == 128
+    tokens = np.sort(np.random.default_rng(77).choice(shape.T, size=24, replace=False))
+    res = full_parity(inp, shape, tokens=tokens, capacity=cap)
+    inv = res["layer"].routing()["inv_pos"].cpu().numpy()
+    assert (inv < 0).any()          # the skewed bias overflows some experts
+    del inp
+    torch.cuda.empty_cache()
+
+
 def test_zero_tokens_is_a_noop():
     from mixture_experts_ffn_expert_b200.layer import MoELayer
     shape = WORKLOADS["tiny_t256_d128_f64_e31k7_s1"]
@@ -235,6 +273,10 @@ def test_error_paths_on_device():
     assert e.value.status == 2
     with pytest.raises(MoEError) as e:
         plan.forward(-1, *args)
+    assert e.value.status == 2
+    from mixture_experts_ffn_expert_b200.binding import MOE_OPTION_EXPERT_CAPACITY
+    with pytest.raises(MoEError) as e:          # negative seat limit
+        plan.set_option(MOE_OPTION_EXPERT_CAPACITY, -1)
     assert e.value.status == 2
     plan.forward(T, *args)
     torch.cuda.synchronize()
