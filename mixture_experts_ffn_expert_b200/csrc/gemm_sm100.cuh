@@ -15,8 +15,9 @@
 //    counts, so no host synchronisation is needed to learn the group sizes;
 //    within a group the m-blocks are innermost so the CTAs running at the same
 //    time share one weight tile through L2;
-//  * warp 0: TMA producer (128B-swizzled boxes, no cluster multicast), a
-//    kStages-deep shared-memory ring guarded by full/empty mbarriers;
+//  * warps 0 and 6: TMA producers taking alternate stages of a kStages-deep
+//    shared-memory ring guarded by full/empty mbarriers (128B-swizzled boxes,
+//    no cluster multicast); the CTA-pair kernel has warp 0 only;
 //  * warp 1: allocates 512 TMEM columns, one thread issues
 //    tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) and commits; a
 //    tile that owns at most 64 rows (a small expert group) uses M=64 instead,
@@ -45,7 +46,15 @@ constexpr int kBTileBytes = kBN * kBK * 2;     // 32 KB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kNumAcc = 2;
 constexpr int kTmemCols = kNumAcc * kBN;       // 512: the whole TMEM of the SM
-constexpr int kGemmThreads = 192;
+// Single-CTA kernel: warps 0 and 6 are TMA producers taking alternate stages,
+// warp 1 issues MMAs, warps 2..5 run the epilogue. Measured on B200 with
+// per-role cycle counters: one producer thread spends ~400 cycles per stage
+// issuing its three TMA loads (the expect-tx arrive is ~60), against 512
+// cycles of MMAs per stage, so a single producer left the tensor pipe waiting.
+// The CTA-pair kernel issues two loads per CTA per stage and keeps one producer.
+constexpr int kGemmThreads = 224;
+constexpr int kProducer2Warp = 6;
+constexpr int kPairThreads = 192;
 constexpr int kEpiThreads = 128;
 
 enum EpiMode : int { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiF32 = 2 };
@@ -228,10 +237,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     kb_end = P.k_splits > 1 ? min(nkb, kb_begin + P.kb_per_split) : nkb;
   };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    int s = 0;
-    uint32_t ph = 0;
+  if (warp == 0 || warp == kProducer2Warp) {
+    // ------------------------------------------------------------ TMA producers
+    // Both walk the tile and k-block sequence; producer `pid` fills the
+    // k-blocks it (counted over the CTA's tiles) with it % 2 == pid, i.e.
+    // alternate stages of the ring, so their issue latencies overlap.
+    const int pid = warp == 0 ? 0 : 1;
+    int it = 0;
     uint32_t issued_mask = 0, issued_par = 0;  // per stage: issued at least once / last parity
     bool ok = true;
     // Grouped GEMMs stream a weight tile (evict first) when its group has a
@@ -251,7 +263,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const CUtensorMap* mB1 = ex ? &tmB1x : &tmB1;
       int kb_begin, kb_end;
       kb_range(tc, ex, kb_begin, kb_end);
-      for (int kb = kb_begin; kb < kb_end; ++kb) {
+      for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
+        if ((it & 1) != pid) continue;
+        const int s = it % kStages;
+        const uint32_t ph = static_cast<uint32_t>(it / kStages) & 1u;
         ok = mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, s_abort);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) {
@@ -279,7 +294,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
         issued_mask |= 1u << s;
         issued_par = (issued_par & ~(1u << s)) | (ph << s);
-        if (++s == kStages) { s = 0; ph ^= 1u; }
       }
     }
     if (!ok && lane == 0) {
@@ -496,7 +510,7 @@ __host__ __device__ constexpr int pair_tile_cols(int mode, int nw) {
 }
 
 template <int MODE, int NW>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kPairThreads, 1)
     moe_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB0,
                          const __grid_constant__ CUtensorMap tmB1, const GemmParams P) {

@@ -238,7 +238,7 @@ bool launch_gemm_pair(Launcher& L, cudaStream_t s, const char* name, const CUten
   if (pairs < 1) pairs = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
-  cfg.blockDim = dim3(moe::kGemmThreads);
+  cfg.blockDim = dim3(moe::kPairThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
