@@ -180,7 +180,21 @@ def kernel_work(name, shape, T, touched):
 
 
 # ----------------------------------------------------------------- oracle (CPU)
-def oracle_sample_run(inp, shape, tokens, expert_cache):
+def oracle_experts(inp_host, shape, budget_bytes=16 << 30):
+    """Expert e -> its fp64 (W1, W3, W2) for the oracle. The bf16 -> fp64 widening is
+    input preparation, not the oracle's work: done once, outside any timed region,
+    when all experts fit in budget_bytes (the coarse layer: 11.3 GB); otherwise per
+    call, and then it is part of the timed oracle run. Returns (fn, converted_once)."""
+    import torch
+    keys = ("W1", "W3", "W2")
+    if 8 * 3 * shape.d * shape.f * shape.n_routed <= budget_bytes:
+        conv = [tuple(inp_host[k][e].to(torch.float64).numpy() for k in keys)
+                for e in range(shape.n_routed)]
+        return (lambda e: conv[e]), True
+    return (lambda e: tuple(inp_host[k][e].to(torch.float64).numpy() for k in keys)), False
+
+
+def oracle_sample_run(inp, shape, tokens, expert):
     """Run the fp64 oracle on the rows `tokens` of x; returns seconds."""
     import numpy as np
     import torch
@@ -189,12 +203,6 @@ def oracle_sample_run(inp, shape, tokens, expert_cache):
     x = inp["x"][torch.as_tensor(tokens)].to(torch.float64).numpy()
     wg = inp["W_g"].to(torch.float64).numpy()
     bias = None if inp["bias"] is None else inp["bias"].to(torch.float64).numpy()
-
-    def expert(e):
-        w1, w3, w2 = expert_cache(e)
-        return (w1.to(torch.float64).numpy(), w3.to(torch.float64).numpy(),
-                w2.to(torch.float64).numpy())
-
     shared = None
     if shape.n_shared > 0:
         shared = tuple(inp[k].to(torch.float64).numpy() for k in ("W1s", "W3s", "W2s"))
@@ -221,16 +229,15 @@ def cpu_threads():
     return len(os.sched_getaffinity(0))
 
 
-def timed_oracle(inp_host, shape, target_s, max_tokens=None):
+def timed_oracle(inp_host, shape, target_s, expert, max_tokens=None):
     """Grow a seeded token sample until one oracle run costs about target_s."""
     import numpy as np
     rng = np.random.default_rng(0)
     T = shape.T if max_tokens is None else max_tokens
     order = rng.permutation(T)
-    cache = lambda e: (inp_host["W1"][e], inp_host["W3"][e], inp_host["W2"][e])  # noqa: E731
     n = min(8, T)
     while True:
-        dt = oracle_sample_run(inp_host, shape, np.sort(order[:n]), cache)
+        dt = oracle_sample_run(inp_host, shape, np.sort(order[:n]), expert)
         if dt >= 0.6 * target_s or n >= T:
             return n, dt
         n = min(T, max(n + 1, int(n * min(8.0, max(2.0, target_s / max(dt, 1e-3))))))
@@ -249,18 +256,18 @@ def run_reference(args, info):
         shape = shape.with_tokens(args.tokens)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = host_copy_of_inputs(make_layer_inputs(shape, seed=0, device=dev))
-    # size one step to about (a few minutes) / (steps + warmup)
-    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
-    n_tok, _ = timed_oracle(inp, shape, per_step)
+    expert, once = oracle_experts(inp, shape)
+    # size one step to about (two minutes) / (steps + warmup)
+    per_step = max(0.25, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    n_tok, _ = timed_oracle(inp, shape, per_step, expert)
     import numpy as np
     rng = np.random.default_rng(1)
-    cache = lambda e: (inp["W1"][e], inp["W3"][e], inp["W2"][e])  # noqa: E731
     for _ in range(args.warmup):
-        oracle_sample_run(inp, shape, np.sort(rng.choice(shape.T, n_tok, replace=False)), cache)
+        oracle_sample_run(inp, shape, np.sort(rng.choice(shape.T, n_tok, replace=False)), expert)
     times = []
     for _ in range(args.steps):
         times.append(oracle_sample_run(inp, shape,
-                                       np.sort(rng.choice(shape.T, n_tok, replace=False)), cache))
+                                       np.sort(rng.choice(shape.T, n_tok, replace=False)), expert))
     total = sum(times)
     value = n_tok * args.steps / total
     cores = cpu_threads()
@@ -272,7 +279,9 @@ def run_reference(args, info):
         "config": workload_config(shape, args),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"{n_tok} seeded tokens of T={shape.T} per step (routing and "
-                                   f"experts for those tokens only)"},
+                                   f"experts for those tokens only; expert weights widened to "
+                                   f"fp64 {'once, outside the timing' if once else 'inside each run'}"
+                                   f")"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -467,10 +476,13 @@ def run_ours(args, info):
     cpu = None
     if not args.no_cpu_baseline and info.rank == 0 and info.world_size == 1:
         inp_host = host_copy_of_inputs(inp)
-        n_tok, dt = timed_oracle(inp_host, shape, args.cpu_seconds)
+        expert, once = oracle_experts(inp_host, shape)
+        n_tok, dt = timed_oracle(inp_host, shape, args.cpu_seconds, expert)
         cpu = {"value": n_tok / dt, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
                "sample": f"{n_tok} seeded tokens of T={T} (routing and experts for those "
-                         f"tokens), one run of {dt:.1f} s"}
+                         f"tokens; expert weights widened to fp64 "
+                         f"{'once, outside the timing' if once else 'inside the run'}), "
+                         f"one run of {dt:.1f} s"}
 
     return {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": info.world_size,
