@@ -221,6 +221,18 @@ def test_capacity_from_factor_on_the_deepseek_v3_shape():
     torch.cuda.empty_cache()
 
 
+def test_many_tokens_routing_and_sampled_outputs():
+    # 65536 tokens x 8 slots: 512 routing chunks, 524288 grouped rows (int32 row
+    # indices well past 2^16, offsets past 2^18); routing is checked on every token
+    shape = LayerShape("many_tokens", 65536, 256, 128, 64, 8, 1, True, "normal_var0.5")
+    inp = make_layer_inputs(shape, seed=12, device="cuda")
+    tokens = np.sort(np.random.default_rng(5).choice(shape.T, size=256, replace=False))
+    res = full_parity(inp, shape, tokens=tokens)
+    assert res["near_ties"] <= shape.T * shape.top_k // 50
+    del inp
+    torch.cuda.empty_cache()
+
+
 def test_zero_tokens_is_a_noop():
     from mixture_experts_ffn_expert_b200.layer import MoELayer
     shape = WORKLOADS["tiny_t256_d128_f64_e31k7_s1"]
