@@ -633,8 +633,14 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
       p->capacity > 0 && p->capacity < INT_MAX ? static_cast<int>(p->capacity) : INT_MAX;
   {
     const size_t smem = size_t(moe::kMaxRouted + nr) * 4 + size_t(2) * Lw.tpc * k * 4;
+    // few chunks (small T): split the row copy into column slices of at least
+    // 32 vectors so that about two blocks per SM copy
+    int slices = (2 * p->num_sms) / Lw.n_chunks;
+    const int max_slices = d / 8 / 32;
+    if (slices > max_slices) slices = max_slices;
+    if (slices < 1) slices = 1;
     L.begin("route_scatter", main_st);
-    launch_pdl(moe::route_scatter_kernel, dim3(Lw.n_chunks), dim3(moe::kRouteThreads), smem,
+    launch_pdl(moe::route_scatter_kernel, dim3(Lw.n_chunks, slices), dim3(moe::kRouteThreads), smem,
                main_st, (const int*)idx, (const int*)chunk_counts, (const int*)counts,
                static_cast<int>(T), k, nr, Lw.tpc, Lw.n_chunks, moe::kBM, seat_limit,
                reinterpret_cast<const uint4*>(x), d / 8, reinterpret_cast<uint4*>(xperm),

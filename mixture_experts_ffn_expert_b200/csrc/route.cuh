@@ -213,7 +213,8 @@ __device__ __forceinline__ int block_exclusive_scan(int* s, int n, int* tmp) {
 // (capacity; INT_MAX when unlimited) an expert keeps its first `capacity` pairs
 // in that order ("What is an expert, really?" glossary, capacity factor / token
 // dropping): offsets and m-tiles count kept rows, a dropped pair gets inv_pos
-// -1 and no row.
+// -1 and no row. Grid (n_chunks, column slices): every block ranks its chunk;
+// the blocks of slice 0 write the permutation, block (0, 0) the offsets.
 constexpr int kCopyUnroll = 4;
 
 __global__ void __launch_bounds__(kRouteThreads)
@@ -249,7 +250,7 @@ __global__ void __launch_bounds__(kRouteThreads)
   }
   __syncthreads();
   const int total = block_exclusive_scan(s_off, n_routed, s_tmp);
-  if (blockIdx.x == 0) {
+  if (blockIdx.x == 0 && blockIdx.y == 0) {
     // publish offsets and the m-tile prefix for the grouped GEMMs
     for (int e = threadIdx.x; e < n_routed; e += blockDim.x) offsets_out[e] = s_off[e];
     if (threadIdx.x == 0) offsets_out[n_routed] = total;
@@ -289,25 +290,31 @@ __global__ void __launch_bounds__(kRouteThreads)
     }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < n_ent; i += blockDim.x) {
-    const int pos = s_pos[i];
-    inv_pos[ebase + i] = pos;
-    if (pos >= 0) perm_src[pos] = t0 + i / top_k;
-  }
+  if (blockIdx.y == 0)
+    for (int i = threadIdx.x; i < n_ent; i += blockDim.x) {
+      const int pos = s_pos[i];
+      inv_pos[ebase + i] = pos;
+      if (pos >= 0) perm_src[pos] = t0 + i / top_k;
+    }
+  // blockIdx.y selects a column slice of the rows (several slices when the
+  // batch has few chunks, so that the copy still spreads over the SMs)
+  const int span = (d_vec + gridDim.y - 1) / gridDim.y;
+  const int v_begin = blockIdx.y * span;
+  const int v_end = min(d_vec, v_begin + span);
   for (int tl = warp; tl < ntok; tl += kRouteThreads / 32) {
     const uint4* src = x + static_cast<long long>(t0 + tl) * d_vec;
     const int* pos = s_pos + tl * top_k;
-    for (int v0 = lane; v0 < d_vec; v0 += 32 * kCopyUnroll) {
+    for (int v0 = v_begin + lane; v0 < v_end; v0 += 32 * kCopyUnroll) {
       uint4 val[kCopyUnroll];
 #pragma unroll
       for (int u = 0; u < kCopyUnroll; ++u)
-        if (v0 + 32 * u < d_vec) val[u] = src[v0 + 32 * u];
+        if (v0 + 32 * u < v_end) val[u] = src[v0 + 32 * u];
       for (int j = 0; j < top_k; ++j) {
         if (pos[j] < 0) continue;
         uint4* dst = xperm + static_cast<long long>(pos[j]) * d_vec;
 #pragma unroll
         for (int u = 0; u < kCopyUnroll; ++u)
-          if (v0 + 32 * u < d_vec) dst[v0 + 32 * u] = val[u];
+          if (v0 + 32 * u < v_end) dst[v0 + 32 * u] = val[u];
       }
     }
   }

@@ -29,6 +29,7 @@ SMALL = [
     ("wide_router", 96, 256, 64, 512, 10, 1, True, "zipf1.1"),      # 16 scores per lane, 2 n-tiles
     ("max_router", 64, 128, 32, 1024, 32, 0, True, "none"),         # N_r and k at their limits
     ("skewed_groups", 1000, 256, 128, 64, 6, 1, True, "zipf1.1"),
+    ("sliced_row_copy", 40, 1024, 64, 12, 3, 1, True, "none"),      # few chunks: 4 column slices
 ]
 
 
