@@ -100,12 +100,20 @@ int moe_last_status(void);
  *   (token, slot) order; a dropped pair adds nothing to its token's output, the
  *   kept gates are not renormalised and the shared expert still applies. This
  *   option changes results; the others do not. A capacity factor cf maps to
- *   C = ceil(cf * T * top_k / N_r). */
+ *   C = ceil(cf * T * top_k / N_r).
+ * MOE_OPTION_TEST_WAIT_TIMEOUT: test hook for the failure path, not for normal
+ *   use. Value 1 arms it for the next forward only: if that forward runs the
+ *   routed gate/up GEMM on the one-CTA-per-tile kernel, one CTA withholds the
+ *   loads of its first pipeline stage, its MMA warp's bounded wait (2 s) expires,
+ *   and the kernel sets the device status to MOE_DEVICE_TIMEOUT, drains its
+ *   copies, frees its tensor memory and returns; that forward's output is
+ *   invalid, the context stays usable. No fault, trap or unbounded wait. */
 enum {
   MOE_OPTION_PAIR_MIN_ROWS = 1,
   MOE_OPTION_WIDE_TILES = 2,
   MOE_OPTION_MERGE_SHARED = 3,
-  MOE_OPTION_EXPERT_CAPACITY = 4
+  MOE_OPTION_EXPERT_CAPACITY = 4,
+  MOE_OPTION_TEST_WAIT_TIMEOUT = 100
 };
 int moe_plan_set_option(moe_plan_t plan, int option, int64_t value);
 

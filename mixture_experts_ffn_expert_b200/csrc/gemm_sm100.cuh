@@ -84,6 +84,10 @@ struct GemmParams {
   void* x_out;
   long long x_ldo;
   int x_out_f32;             // plain epilogue: store fp32 instead of bf16
+  // Test hook (0 in normal use): CTA 0 of the single-CTA kernel withholds the
+  // loads of its first stage, so that its MMA warp's bounded wait expires and
+  // the kernel takes its timeout path (status word, drain, TMEM release).
+  int test_withhold;
 };
 
 // Dynamic shared memory the kernel needs for a given number of groups.
@@ -265,6 +269,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       kb_range(tc, ex, kb_begin, kb_end);
       for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
         if ((it & 1) != pid) continue;
+        if (P.test_withhold && blockIdx.x == 0 && it == 0) continue;   // test hook
         const int s = it % kStages;
         const uint32_t ph = static_cast<uint32_t>(it / kStages) & 1u;
         ok = mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, s_abort);

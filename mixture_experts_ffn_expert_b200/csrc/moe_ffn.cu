@@ -71,6 +71,9 @@ struct moe_plan {
   int merge_shared = 0;
   // seats per expert per forward (token dropping); 0: unlimited (dropless)
   int64_t capacity = 0;
+  // one-shot test hook: the next forward's routed gate/up GEMM (single-CTA
+  // kernel) lets one bounded wait expire
+  int test_withhold = 0;
   int device, num_sms;
   const float* bias = nullptr;
   char* ws = nullptr;
@@ -404,6 +407,10 @@ int moe_plan_set_option(moe_plan_t p, int option, int64_t value) {
       if (value < 0 || value > 1) return fail(MOE_INVALID_ARG, "merge_shared must be 0 or 1");
       p->merge_shared = static_cast<int>(value);
       return MOE_OK;
+    case MOE_OPTION_TEST_WAIT_TIMEOUT:
+      if (value < 0 || value > 1) return fail(MOE_INVALID_ARG, "test hook must be 0 or 1");
+      p->test_withhold = static_cast<int>(value);
+      return MOE_OK;
     case MOE_OPTION_EXPERT_CAPACITY:
       if (value < 0) return fail(MOE_INVALID_ARG, "expert capacity must be >= 0");
       p->capacity = value;
@@ -678,6 +685,10 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.status = status;
     g.k_splits = 1;
     g.kb_per_split = (d + moe::kBK - 1) / moe::kBK;
+    if (!routed_pair_swiglu) {
+      g.test_withhold = p->test_withhold;
+      p->test_withhold = 0;
+    }
     if (merge_gu) {
       g.x_tiles = shared_mt * ((nsf + 127) / 128);
       g.x_rows = static_cast<int>(T);

@@ -297,6 +297,35 @@ def test_error_paths_on_device():
     plan.close()
 
 
+def test_bounded_wait_timeout_sets_status_and_context_recovers():
+    # the failure path without a fault: the one-shot test hook makes one CTA of
+    # the gate/up GEMM withhold a stage's loads, so its MMA warp's bounded wait
+    # (2 s) expires; the kernel must report MOE_DEVICE_TIMEOUT and leave the
+    # context usable
+    import time
+    from mixture_experts_ffn_expert_b200.binding import MOE_OPTION_TEST_WAIT_TIMEOUT
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    shape = WORKLOADS["tiny_t256_d128_f64_e31k7_s1"]
+    inp = make_layer_inputs(shape, seed=0, device="cuda")
+    layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
+                     shape.renorm, inp, bias=inp["bias"], device="cuda")
+    ref = layer(inp["x"]).clone()
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    layer.plan.set_option(MOE_OPTION_TEST_WAIT_TIMEOUT, 1)
+    t0 = time.perf_counter()
+    layer(inp["x"])
+    torch.cuda.synchronize()
+    waited = time.perf_counter() - t0
+    assert layer.device_status() == 6          # MOE_DEVICE_TIMEOUT
+    assert layer.device_status() == 0          # reading clears it
+    assert 1.5 < waited < 30.0, waited         # one bounded wait, not a hang
+    again = layer(inp["x"])                    # the hook was one-shot
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    assert torch.equal(again, ref)
+
+
 @pytest.mark.parametrize("name", ["decode_t128_d2048_f512_e512k10_s1", "tiny_t256_d128_f64_e31k7_s1"])
 def test_cuda_graph_replay_matches_stream_launch(name):
     # the whole forward (including the shared expert's forked stream, when used)
