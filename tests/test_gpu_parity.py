@@ -234,6 +234,38 @@ def test_many_tokens_routing_and_sampled_outputs():
     torch.cuda.empty_cache()
 
 
+POISON_CASES = [
+    # name, T, d, f, N_r, k, N_s, renorm, bias, capacity, pair_min_rows
+    ("poison_ragged", 600, 384, 320, 6, 2, 1, True, "none", None, None),
+    ("poison_pairs", 600, 384, 320, 6, 2, 1, True, "none", None, 0),
+    ("poison_capacity", 1000, 256, 128, 64, 6, 1, True, "zipf1.1", 40, None),
+    ("poison_decode_like", 128, 2048, 512, 512, 10, 1, True, "zipf1.1", None, None),
+]
+
+
+@pytest.mark.parametrize("case", POISON_CASES, ids=[c[0] for c in POISON_CASES])
+def test_poisoned_workspace_and_output_are_fully_overwritten(case):
+    # every scratch byte 0xFF (NaN as bf16 / fp32, -1 as int32) and out NaN before
+    # the forward: a kernel reading scratch that no kernel wrote, or leaving part
+    # of out unwritten, shows up as NaN or a parity failure
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    from parity import check_output, check_routing, oracle_out, to64
+    name, T, d, f, n, k, ns, renorm, bias, cap, pmr = case
+    shape = LayerShape(name, T, d, f, n, k, ns, renorm, bias)
+    inp = make_layer_inputs(shape, seed=13, device="cuda")
+    layer = MoELayer(d, f, n, k, ns, renorm, inp, bias=inp["bias"], device="cuda",
+                     capacity=cap, pair_min_rows=pmr)
+    layer.ensure_workspace(T)
+    layer.workspace[256:].fill_(0xFF)          # the first 256 bytes hold the status word
+    out = torch.full_like(inp["x"], float("nan"))
+    layer(inp["x"], out)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    assert torch.isfinite(out).all()
+    _, idx_ref, _ = check_routing(inp, layer.routing(), shape, capacity=cap)
+    check_output(to64(out), oracle_out(inp, shape, idx_ref, capacity=cap))
+
+
 def test_zero_tokens_is_a_noop():
     from mixture_experts_ffn_expert_b200.layer import MoELayer
     shape = WORKLOADS["tiny_t256_d128_f64_e31k7_s1"]
