@@ -36,6 +36,13 @@ Readings taken where the pages leave a step open:
 * N_s shared experts are one fused SwiGLU of inner width N_s*f, which equals the
   sum of the N_s separate experts (DSV3 "Official code", "Watch-outs").
 * The routed rows are grouped by expert in ascending (token, slot) order.
+* Bias placement: by default the per-expert bias is a logit bias (it moves both
+  the selection and the gates). The selection-only variant (the survey's
+  "selection-only load-balance bias"; DSV3 "How it works" names a load-balance
+  bias on the routed centroids without defining it) adds the bias to the scores
+  only to choose the top k; the gates are then the softmax of the unbiased
+  scores over all N_r experts (raw), or those probabilities renormalised over
+  the selected set. Ties in the biased scores go to the lower index.
 * Capacity (token dropping, WIE glossary "capacity factor / token dropping":
   each expert has a seat limit per batch, overflow tokens are skipped): with a
   limit of C seats, an expert keeps the first C (token, slot) pairs routed to it
@@ -65,6 +72,7 @@ __all__ = [
     "softmax_rows",
     "select_topk",
     "gate_values",
+    "routing_probabilities",
     "route_permutation",
     "topk_gap",
     "moe_layer",
@@ -315,10 +323,25 @@ def _expert_getter(experts: ExpertSource):
     return lambda e: (W1[e], W3[e], W2[e])
 
 
+def routing_probabilities(x, W_g, bias, bias_selection_only: bool = False):
+    """(p_select, p_gate): the probabilities the top-k ranks and the ones the gates
+    take. With a logit bias (default) both are softmax(x W_g^T + b); with a
+    selection-only bias p_select = softmax(x W_g^T + b) and p_gate = softmax(x W_g^T).
+    Ranking by softmax(s + b) is ranking by s + b (softmax is increasing).
+    Pinned by tests/test_oracle_routing.py (a forcing bias keeps the unbiased gate;
+    no bias makes both modes equal) and by the scalar brute force.
+    """
+    p_sel = softmax_rows(router_scores(x, W_g, bias))
+    if not bias_selection_only or bias is None:
+        return p_sel, p_sel
+    return p_sel, softmax_rows(router_scores(x, W_g, None))
+
+
 def moe_layer(x, W_g, bias, experts: ExpertSource, shared, top_k: int, renorm: bool,
               tokens: Optional[Sequence[int]] = None,
               forced_idx: Optional[np.ndarray] = None,
-              capacity: Optional[int] = None) -> dict:
+              capacity: Optional[int] = None,
+              bias_selection_only: bool = False) -> dict:
     """Forward pass of the layer: shared + sum of gated routed experts, no residual.
 
     [DSV3] eq. (12) without u_t, "Official code": route, run every expert on the
@@ -334,6 +357,8 @@ def moe_layer(x, W_g, bias, experts: ExpertSource, shared, top_k: int, renorm: b
     oracle's own probabilities); it is how a second correct selection is scored.
     ``capacity`` (None: unlimited) is the per-expert seat limit of
     ``route_permutation``: dropped (token, slot) pairs add nothing.
+    ``bias_selection_only`` moves the bias out of the gates (see
+    ``routing_probabilities``); the returned p is the gate probability.
 
     Returns a dict with p, idx, g, counts, offsets, perm_src, inv_pos, tokens and
     out (len(tokens), d) in fp64. Pinned by the dense brute force on tiny inputs,
@@ -343,9 +368,9 @@ def moe_layer(x, W_g, bias, experts: ExpertSource, shared, top_k: int, renorm: b
     x = _f64(x)
     T, d = x.shape
     n_routed = np.asarray(W_g).shape[0]
-    p = softmax_rows(router_scores(x, W_g, bias))
+    p_sel, p = routing_probabilities(x, W_g, bias, bias_selection_only)
     if forced_idx is None:
-        idx = select_topk(p, top_k)
+        idx = select_topk(p_sel, top_k)
     else:
         idx = np.asarray(forced_idx, dtype=np.int64)
         assert idx.shape == (T, top_k)
@@ -375,7 +400,8 @@ def moe_layer(x, W_g, bias, experts: ExpertSource, shared, top_k: int, renorm: b
 
 
 def moe_layer_dense_bruteforce(x, W_g, bias, W1, W3, W2, shared, top_k: int,
-                               renorm: bool, capacity: Optional[int] = None) -> np.ndarray:
+                               renorm: bool, capacity: Optional[int] = None,
+                               bias_selection_only: bool = False) -> np.ndarray:
     """Brute-force evaluation for tiny inputs: every expert on every token.
 
     [SFE] "Why segmentation helps": the layer is sum_{i in S} g_i E_i(x), i.e. a
@@ -386,6 +412,8 @@ def moe_layer_dense_bruteforce(x, W_g, bias, W1, W3, W2, shared, top_k: int,
     each expert's SwiGLU is summed element by element. With a ``capacity``, the
     seats are handed out pair by pair in (token, slot) order ([WIE] glossary
     "capacity factor / token dropping") and a pair without a seat is skipped.
+    With ``bias_selection_only`` the biased scores choose the experts and the
+    gates come from the unbiased scores.
     """
     import math
 
@@ -409,23 +437,25 @@ def moe_layer_dense_bruteforce(x, W_g, bias, W1, W3, W2, shared, top_k: int,
     out = np.zeros((T, d), dtype=np.float64)
     seats_used = [0] * n_routed
     for t in range(T):
-        scores = []
-        for e in range(n_routed):
-            s = sum(Wg[e][c] * x[t][c] for c in range(d))
-            if bias is not None:
-                s += float(bias[e])
-            scores.append(s)
-        mx = max(scores)
-        ex = [math.exp(s - mx) for s in scores]
-        tot = sum(ex)
-        prob = [v / tot for v in ex]
+        raw = [sum(Wg[e][c] * x[t][c] for c in range(d)) for e in range(n_routed)]
+        scores = [raw[e] + (float(bias[e]) if bias is not None else 0.0)
+                  for e in range(n_routed)]
+
+        def probs(v):
+            mx = max(v)
+            ex = [math.exp(a - mx) for a in v]
+            tot = sum(ex)
+            return [a / tot for a in ex]
+
+        prob_sel = probs(scores)
+        prob = probs(raw) if bias_selection_only else prob_sel
         chosen = []
         for _ in range(top_k):
             best = None
             for e in range(n_routed):      # first maximum wins: lower index on ties
                 if e in chosen:
                     continue
-                if best is None or prob[e] > prob[best]:
+                if best is None or prob_sel[e] > prob_sel[best]:
                     best = e
             chosen.append(best)
         G = [0.0] * n_routed

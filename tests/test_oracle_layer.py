@@ -161,3 +161,18 @@ def test_zero_capacity_leaves_only_the_shared_expert():
     only_shared = moe_layer(x, W_g, b, tuple(np.zeros_like(a) for a in experts), shared, 2,
                             False)["out"]
     np.testing.assert_array_equal(got, only_shared)
+
+
+@pytest.mark.parametrize("renorm", [True, False])
+def test_selection_only_bias_layer_equals_bruteforce(renorm):
+    rng = np.random.default_rng(23)
+    T, d, f, n, k, ns = 8, 5, 4, 6, 2, 1
+    x, W_g, b, experts, shared = _tiny(rng, T, d, f, n, ns, bias=True)
+    b = b * 3.0                     # large enough to change some selections
+    ref = moe_layer_dense_bruteforce(x, W_g, b, *experts, shared, k, renorm,
+                                     bias_selection_only=True)
+    got = moe_layer(x, W_g, b, experts, shared, k, renorm, bias_selection_only=True)["out"]
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    # and it differs from the logit-bias layer (the bias really left the gates)
+    logit = moe_layer(x, W_g, b, experts, shared, k, renorm)["out"]
+    assert np.abs(logit - got).max() > 1e-6

@@ -151,3 +151,33 @@ def test_capacity_at_or_above_the_largest_load_drops_nothing():
     capped = route_permutation(idx, 6, int(np.bincount(idx.reshape(-1)).max()))
     for a, b in zip(free, capped):
         np.testing.assert_array_equal(a, b)
+
+
+def test_selection_only_bias_keeps_the_unbiased_gate():
+    # a bias that forces expert 3 into every selection: as a logit bias its gate is
+    # ~1, as a selection-only bias the gate is expert 3's unbiased probability
+    from oracle import routing_probabilities
+    rng = np.random.default_rng(31)
+    x = rng.normal(size=(20, 6))
+    W_g = rng.normal(size=(5, 6))
+    bias = np.array([0.0, 0.0, 0.0, 60.0, 0.0])
+    p_sel, p_gate = routing_probabilities(x, W_g, bias, bias_selection_only=True)
+    idx = select_topk(p_sel, 2)
+    assert np.all(idx[:, 0] == 3)
+    unbiased = softmax_rows(router_scores(x, W_g))
+    np.testing.assert_array_equal(p_gate, unbiased)
+    g = gate_values(p_gate, idx, False)
+    np.testing.assert_allclose(g[:, 0], unbiased[:, 3], rtol=0, atol=0)
+    assert np.all(g[:, 0] < 0.99)
+    p_logit, p_logit_gate = routing_probabilities(x, W_g, bias)
+    assert p_logit is p_logit_gate and np.all(p_logit[:, 3] > 0.999)
+
+
+def test_selection_only_without_bias_is_the_plain_router():
+    from oracle import routing_probabilities
+    rng = np.random.default_rng(32)
+    x, W_g = rng.normal(size=(7, 4)), rng.normal(size=(6, 4))
+    a = routing_probabilities(x, W_g, None, bias_selection_only=True)
+    b = routing_probabilities(x, W_g, None)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
