@@ -101,6 +101,12 @@ int moe_last_status(void);
  *   kept gates are not renormalised and the shared expert still applies. This
  *   option changes results; the others do not. A capacity factor cf maps to
  *   C = ceil(cf * T * top_k / N_r).
+ * MOE_OPTION_BIAS_SELECTION_ONLY: 0 (default): the logit bias set with
+ *   moe_plan_set_logit_bias is added to the router scores for both the top-k
+ *   selection and the gates. 1: it only chooses the experts (the selection-only
+ *   load-balance bias "Shared Expert (DeepSeek-V3)" mentions for the routed
+ *   centroids); the gates are the softmax of the unbiased scores over all N_r
+ *   experts, renormalised over the selected ones when the plan renormalises.
  * MOE_OPTION_TEST_WAIT_TIMEOUT: test hook for the failure path, not for normal
  *   use. Value 1 arms it for the next forward only: if that forward runs the
  *   routed gate/up GEMM on the one-CTA-per-tile kernel, one CTA withholds the
@@ -113,6 +119,7 @@ enum {
   MOE_OPTION_WIDE_TILES = 2,
   MOE_OPTION_MERGE_SHARED = 3,
   MOE_OPTION_EXPERT_CAPACITY = 4,
+  MOE_OPTION_BIAS_SELECTION_ONLY = 5,
   MOE_OPTION_TEST_WAIT_TIMEOUT = 100
 };
 int moe_plan_set_option(moe_plan_t plan, int option, int64_t value);

@@ -26,6 +26,7 @@ MOE_OPTION_PAIR_MIN_ROWS = 1
 MOE_OPTION_WIDE_TILES = 2
 MOE_OPTION_MERGE_SHARED = 3
 MOE_OPTION_EXPERT_CAPACITY = 4
+MOE_OPTION_BIAS_SELECTION_ONLY = 5
 MOE_OPTION_TEST_WAIT_TIMEOUT = 100
 
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_INVALID_CONFIG", 2: "MOE_INVALID_ARG",

@@ -71,6 +71,8 @@ struct moe_plan {
   int merge_shared = 0;
   // seats per expert per forward (token dropping); 0: unlimited (dropless)
   int64_t capacity = 0;
+  // 1: the logit bias only chooses the experts, the gates come from unbiased scores
+  int bias_select_only = 0;
   // one-shot test hook: the next forward's routed gate/up GEMM (single-CTA
   // kernel) lets one bounded wait expire
   int test_withhold = 0;
@@ -411,6 +413,10 @@ int moe_plan_set_option(moe_plan_t p, int option, int64_t value) {
       if (value < 0 || value > 1) return fail(MOE_INVALID_ARG, "test hook must be 0 or 1");
       p->test_withhold = static_cast<int>(value);
       return MOE_OK;
+    case MOE_OPTION_BIAS_SELECTION_ONLY:
+      if (value < 0 || value > 1) return fail(MOE_INVALID_ARG, "bias selection-only must be 0 or 1");
+      p->bias_select_only = static_cast<int>(value);
+      return MOE_OK;
     case MOE_OPTION_EXPERT_CAPACITY:
       if (value < 0) return fail(MOE_INVALID_ARG, "expert capacity must be >= 0");
       p->capacity = value;
@@ -608,7 +614,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   launch_pdl(moe::route_topk_kernel<N, S>, dim3(Lw.n_chunks), dim3(moe::kRouteThreads),     \
              smem, main_st, (const float*)scores, Lw.lds, sp,                               \
              static_cast<long long>(T) * Lw.lds, p->bias, static_cast<int>(T), nr, k,       \
-             p->renorm, Lw.tpc, Lw.n_chunks, idx, gate, chunk_counts)
+             p->renorm, p->bias_select_only, Lw.tpc, Lw.n_chunks, idx, gate, chunk_counts)
 #define MOE_TOPK_S(N)                                                                       \
   if (sp <= 1) MOE_TOPK(N, 1);                                                              \
   else if (sp <= 2) MOE_TOPK(N, 2);                                                         \

@@ -40,7 +40,8 @@ template <int NPL, int MAXS>
 __global__ void __launch_bounds__(kRouteThreads)
     route_topk_kernel(const float* __restrict__ scores, int lds, int splits,
                       long long split_stride, const float* __restrict__ bias, int T,
-                      int n_routed, int top_k, int renorm, int tpc, int n_chunks,
+                      int n_routed, int top_k, int renorm, int bias_select_only, int tpc,
+                      int n_chunks,
                       int* __restrict__ idx, float* __restrict__ gate,
                       int* __restrict__ chunk_counts) {
   extern __shared__ int s_hist[];               // [n_routed]
@@ -71,11 +72,16 @@ __global__ void __launch_bounds__(kRouteThreads)
       for (int sp = 1; sp < MAXS; ++sp) a += part[sp][i];
       v[i] = a;
     }
+    // The biased scores rank the experts; the gates are the softmax of the
+    // biased scores (logit bias) or of the unbiased ones (selection-only bias).
     float m = -INFINITY;
+    float key[NPL];
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
       const int e = lane + 32 * i;
-      v[i] = e < n_routed ? v[i] + (bias ? bias[e] : 0.0f) : -INFINITY;
+      const float b = (bias && e < n_routed) ? bias[e] : 0.0f;
+      key[i] = e < n_routed ? v[i] + b : -INFINITY;
+      v[i] = e < n_routed ? (bias_select_only ? v[i] : key[i]) : -INFINITY;
       m = fmaxf(m, v[i]);
     }
 #pragma unroll
@@ -90,9 +96,8 @@ __global__ void __launch_bounds__(kRouteThreads)
     // Selection keys: a NaN score (from NaN or infinite inputs) ranks as -inf,
     // so the order stays total and every lane agrees on each winner; the
     // sentinel index of an empty lane loses every tie against a real expert.
-    float key[NPL];
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) key[i] = v[i] == v[i] ? v[i] : -INFINITY;
+    for (int i = 0; i < NPL; ++i) key[i] = key[i] == key[i] ? key[i] : -INFINITY;
     uint32_t taken = 0;
     float sel_sum = 0.0f, my_p = 0.0f;
     int my_e = -1;
@@ -114,7 +119,13 @@ __global__ void __launch_bounds__(kRouteThreads)
         if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
       }
       if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      const float p = expf(bv - m) / sum;
+      // the winner's gate score, from the lane that holds it
+      float gw = 0.0f;
+#pragma unroll
+      for (int i = 0; i < NPL; ++i)
+        if (i == (be >> 5)) gw = v[i];
+      gw = __shfl_sync(0xffffffffu, gw, be & 31);
+      const float p = expf(gw - m) / sum;
       sel_sum += p;
       if (lane == j) { my_p = p; my_e = be; }
     }

@@ -11,8 +11,9 @@ from typing import Dict, Optional
 
 import torch
 
-from .binding import (MOE_OPTION_EXPERT_CAPACITY, MOE_OPTION_MERGE_SHARED,
-                      MOE_OPTION_PAIR_MIN_ROWS, MOE_OPTION_WIDE_TILES, MoEError, Plan)
+from .binding import (MOE_OPTION_BIAS_SELECTION_ONLY, MOE_OPTION_EXPERT_CAPACITY,
+                      MOE_OPTION_MERGE_SHARED, MOE_OPTION_PAIR_MIN_ROWS, MOE_OPTION_WIDE_TILES,
+                      MoEError, Plan)
 
 __all__ = ["MoELayer", "MoEError", "capacity_from_factor"]
 
@@ -38,14 +39,16 @@ class MoELayer:
     n_shared > 0, W1s, W3s (N_s*f, d), W2s (d, N_s*f), all bf16 contiguous on
     the device; ``bias`` is an optional fp32 (N_r,) logit bias. ``capacity``
     (seats per expert per forward, see ``capacity_from_factor``) turns on token
-    dropping; the other options only select kernels.
+    dropping; ``bias_selection_only`` makes the bias choose experts without
+    entering the gates; the other options only select kernels.
     """
 
     def __init__(self, d: int, f: int, n_routed: int, top_k: int, n_shared: int,
                  renorm: bool, weights: Dict[str, Optional[torch.Tensor]],
                  bias: Optional[torch.Tensor] = None, device=None,
                  pair_min_rows: Optional[int] = None, wide_tiles: Optional[int] = None,
-                 merge_shared: Optional[int] = None, capacity: Optional[int] = None):
+                 merge_shared: Optional[int] = None, capacity: Optional[int] = None,
+                 bias_selection_only: bool = False):
         dev = torch.device(device) if device is not None else torch.device("cuda")
         if dev.type == "cuda" and dev.index is None:
             dev = torch.device("cuda", torch.cuda.current_device())
@@ -64,6 +67,9 @@ class MoELayer:
         self.capacity = capacity or 0
         if capacity:
             self.plan.set_option(MOE_OPTION_EXPERT_CAPACITY, capacity)
+        self.bias_selection_only = bool(bias_selection_only)
+        if bias_selection_only:
+            self.plan.set_option(MOE_OPTION_BIAS_SELECTION_ONLY, 1)
         self.d, self.f, self.n_routed, self.top_k, self.n_shared = d, f, n_routed, top_k, n_shared
         self.renorm = bool(renorm)
         shapes = {"W_g": (n_routed, d), "W1": (n_routed, f, d), "W3": (n_routed, f, d),

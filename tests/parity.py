@@ -12,7 +12,8 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from oracle import moe_layer, route_permutation, router_scores, select_topk, softmax_rows
+from oracle import (moe_layer, route_permutation, router_scores, routing_probabilities,
+                    select_topk, softmax_rows)
 
 TIE_TOL = 1e-5
 REL_L2_TOL = 1e-2
@@ -51,13 +52,15 @@ def reconcile_routing(p: np.ndarray, gpu_idx: np.ndarray, k: int, tol: float = T
     return idx_ref, int(near.sum())
 
 
-def check_routing(inp, gpu, shape, T=None, capacity=None):
+def check_routing(inp, gpu, shape, T=None, capacity=None, bias_selection_only=False):
     """Routing parity on every token. Returns (p, idx_ref, n_near_tie). With an
-    expert capacity only the kept rows of perm_src are defined."""
+    expert capacity only the kept rows of perm_src are defined. The near-tie rule
+    applies to the probabilities the selection ranks; the gates are compared with
+    the gate probabilities (different only for a selection-only bias)."""
     x = to64(inp["x"])
-    p = softmax_rows(router_scores(x, to64(inp["W_g"]), to64(inp["bias"])))
+    p_sel, p = routing_probabilities(x, to64(inp["W_g"]), to64(inp["bias"]), bias_selection_only)
     gpu_idx = gpu["idx"].cpu().numpy().astype(np.int64)
-    idx_ref, n_near = reconcile_routing(p, gpu_idx, shape.top_k)
+    idx_ref, n_near = reconcile_routing(p_sel, gpu_idx, shape.top_k)
     counts, offsets, perm_src, inv_pos = route_permutation(idx_ref, shape.n_routed, capacity)
     np.testing.assert_array_equal(gpu["counts"].cpu().numpy(), counts)
     np.testing.assert_array_equal(gpu["offsets"].cpu().numpy(), offsets)
@@ -72,7 +75,7 @@ def check_routing(inp, gpu, shape, T=None, capacity=None):
     return p, idx_ref, n_near
 
 
-def oracle_out(inp, shape, idx_ref, tokens=None, capacity=None):
+def oracle_out(inp, shape, idx_ref, tokens=None, capacity=None, bias_selection_only=False):
     """Oracle output for `tokens` (all when None), streaming one expert at a time."""
     W1, W3, W2 = inp["W1"], inp["W3"], inp["W2"]
 
@@ -84,7 +87,7 @@ def oracle_out(inp, shape, idx_ref, tokens=None, capacity=None):
         shared = (to64(inp["W1s"]), to64(inp["W3s"]), to64(inp["W2s"]))
     r = moe_layer(to64(inp["x"]), to64(inp["W_g"]), to64(inp["bias"]), expert, shared,
                   shape.top_k, shape.renorm, tokens=tokens, forced_idx=idx_ref,
-                  capacity=capacity)
+                  capacity=capacity, bias_selection_only=bias_selection_only)
     return r["out"]
 
 
@@ -106,7 +109,7 @@ def check_output(gpu_out: np.ndarray, ref: np.ndarray):
 
 
 def run_layer(inp, shape, device="cuda", pair_min_rows=None, wide_tiles=None, merge_shared=None,
-              capacity=None):
+              capacity=None, bias_selection_only=False):
     """Run the CUDA layer through the C ABI; returns (out (T,d) fp64 numpy, routing dict)."""
     from mixture_experts_ffn_expert_b200.layer import MoELayer
 
@@ -114,7 +117,8 @@ def run_layer(inp, shape, device="cuda", pair_min_rows=None, wide_tiles=None, me
                      shape.renorm, {k: inp[k] for k in ("W_g", "W1", "W3", "W2", "W1s",
                                                         "W3s", "W2s")},
                      bias=inp["bias"], device=device, pair_min_rows=pair_min_rows,
-                     wide_tiles=wide_tiles, merge_shared=merge_shared, capacity=capacity)
+                     wide_tiles=wide_tiles, merge_shared=merge_shared, capacity=capacity,
+                     bias_selection_only=bias_selection_only)
     out = layer(inp["x"])
     routing = layer.routing()
     torch.cuda.synchronize()
@@ -123,17 +127,20 @@ def run_layer(inp, shape, device="cuda", pair_min_rows=None, wide_tiles=None, me
 
 
 def full_parity(inp, shape, tokens=None, pair_min_rows=None, wide_tiles=None,
-                merge_shared=None, capacity=None):
+                merge_shared=None, capacity=None, bias_selection_only=False):
     """Routing on all tokens, output on `tokens` (all when None). Returns a summary dict.
     pair_min_rows forces (0) or forbids (huge) the CTA-pair GEMM kernel; wide_tiles
     forces (1) or forbids (0) its 512-column tiles; merge_shared forces (1) or
     forbids (0) the shared expert as extra tiles of the routed GEMM launches;
-    capacity sets the seats per expert (token dropping)."""
+    capacity sets the seats per expert (token dropping); bias_selection_only keeps
+    the bias out of the gates."""
     out, routing, layer = run_layer(inp, shape, pair_min_rows=pair_min_rows,
                                     wide_tiles=wide_tiles, merge_shared=merge_shared,
-                                    capacity=capacity)
-    _, idx_ref, n_near = check_routing(inp, routing, shape, capacity=capacity)
-    ref = oracle_out(inp, shape, idx_ref, tokens, capacity=capacity)
+                                    capacity=capacity, bias_selection_only=bias_selection_only)
+    _, idx_ref, n_near = check_routing(inp, routing, shape, capacity=capacity,
+                                       bias_selection_only=bias_selection_only)
+    ref = oracle_out(inp, shape, idx_ref, tokens, capacity=capacity,
+                     bias_selection_only=bias_selection_only)
     got = to64(out if tokens is None else out[torch.as_tensor(tokens, device=out.device)])
     rel_l2, max_abs, scale = check_output(got, ref)
     return {"near_ties": n_near, "rel_l2": rel_l2, "max_abs": max_abs, "max_ref": scale,

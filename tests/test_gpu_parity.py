@@ -208,6 +208,39 @@ def test_expert_capacity_drops_the_later_pairs(case):
     assert int(r["offsets"][-1]) == T * k - dropped
 
 
+SELECTION_ONLY_CASES = [
+    # name, T, d, f, N_r, k, N_s, renorm, bias
+    ("selonly_normal_renorm", 600, 256, 128, 64, 6, 1, True, "normal_var0.5"),
+    ("selonly_zipf_raw", 500, 256, 128, 128, 8, 1, False, "zipf1.1"),
+    ("selonly_top1_raw", 300, 128, 64, 16, 1, 0, False, "normal_var0.5"),  # renormalised top-1 is always 1
+]
+
+
+@pytest.mark.parametrize("case", SELECTION_ONLY_CASES, ids=[c[0] for c in SELECTION_ONLY_CASES])
+def test_selection_only_bias(case):
+    name, T, d, f, n, k, ns, renorm, bias = case
+    shape = LayerShape(name, T, d, f, n, k, ns, renorm, bias)
+    inp = make_layer_inputs(shape, seed=14, device="cuda")
+    res = full_parity(inp, shape, bias_selection_only=True)
+    assert res["near_ties"] <= max(2, T * k // 20)
+    # the same selections as the logit-bias layer, different gates
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    logit = MoELayer(d, f, n, k, ns, renorm, inp, bias=inp["bias"], device="cuda")
+    logit(inp["x"])
+    a, b = res["layer"].routing(), logit.routing()
+    same_sel = (a["idx"] == b["idx"]).float().mean().item()
+    assert same_sel > 0.99
+    assert not torch.allclose(a["w"], b["w"])
+
+
+def test_selection_only_bias_on_the_decode_shape():
+    shape = WORKLOADS["decode_t128_d2048_f512_e512k10_s1"]
+    inp = make_layer_inputs(shape, seed=0, device="cuda")
+    full_parity(inp, shape, bias_selection_only=True)
+    del inp
+    torch.cuda.empty_cache()
+
+
 def test_capacity_from_factor_on_the_deepseek_v3_shape():
     from mixture_experts_ffn_expert_b200.layer import capacity_from_factor
     shape = WORKLOADS["dsv3_prefill_t4096_d7168_f2048_e256k8_s1"]
