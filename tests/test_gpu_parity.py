@@ -299,6 +299,39 @@ def test_poisoned_workspace_and_output_are_fully_overwritten(case):
     check_output(to64(out), oracle_out(inp, shape, idx_ref, capacity=cap))
 
 
+def _random_cases(n=14, seed=2024):
+    """Seeded random layer shapes within the library's limits (d, f multiples of
+    8, N_r <= 1024, k <= 32), with random bias modes, capacities and kernels."""
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(n):
+        n_r = int(rng.choice([1, 2, 5, 8, 17, 33, 64, 100, 257]))
+        k = int(rng.integers(1, min(n_r, 16) + 1))
+        T = int(rng.choice([1, 2, 7, 64, 129, 300, 777, 2000]))
+        d = 8 * int(rng.integers(1, 97))
+        f = 8 * int(rng.integers(1, 97))
+        ns = int(rng.integers(0, 4))
+        renorm = bool(rng.integers(0, 2))
+        bias = str(rng.choice(["none", "normal_var0.5", "zipf1.1"]))
+        sel_only = bias != "none" and bool(rng.integers(0, 2))
+        cap = int(rng.integers(1, max(2, T * k // n_r + 2))) if rng.random() < 0.3 else None
+        pmr = 0 if rng.random() < 0.3 else None
+        cases.append((f"rand{i}_T{T}_d{d}_f{f}_e{n_r}k{k}_s{ns}", T, d, f, n_r, k, ns, renorm,
+                      bias, sel_only, cap, pmr))
+    return cases
+
+
+RANDOM_CASES = _random_cases()
+
+
+@pytest.mark.parametrize("case", RANDOM_CASES, ids=[c[0] for c in RANDOM_CASES])
+def test_random_shapes_all_outputs(case):
+    name, T, d, f, n, k, ns, renorm, bias, sel_only, cap, pmr = case
+    shape = LayerShape(name, T, d, f, n, k, ns, renorm, bias)
+    inp = make_layer_inputs(shape, seed=15, device="cuda")
+    full_parity(inp, shape, capacity=cap, pair_min_rows=pmr, bias_selection_only=sel_only)
+
+
 def test_zero_tokens_is_a_noop():
     from mixture_experts_ffn_expert_b200.layer import MoELayer
     shape = WORKLOADS["tiny_t256_d128_f64_e31k7_s1"]
