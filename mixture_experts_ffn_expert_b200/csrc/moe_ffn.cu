@@ -646,9 +646,10 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
       p->capacity > 0 && p->capacity < INT_MAX ? static_cast<int>(p->capacity) : INT_MAX;
   {
     const size_t smem = size_t(moe::kMaxRouted + nr) * 4 + size_t(2) * Lw.tpc * k * 4;
-    // few chunks (small T): split the row copy into column slices of at least
-    // 32 vectors so that about two blocks per SM copy
-    int slices = (2 * p->num_sms) / Lw.n_chunks;
+    // split the row copy into column slices of at least 32 vectors so that
+    // about four blocks per SM copy (one block per chunk leaves most SMs with
+    // one or two resident blocks, too few loads in flight)
+    int slices = (4 * p->num_sms) / Lw.n_chunks;
     const int max_slices = d / 8 / 32;
     if (slices > max_slices) slices = max_slices;
     if (slices < 1) slices = 1;

@@ -347,12 +347,13 @@ __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
 }
 
 constexpr int kCombineThreads = 128;
-constexpr int kCombineVec = 4;                 // 16-byte column vectors per thread
+constexpr int kCombineVec = 2;                 // 16-byte column vectors per thread
 constexpr int kCombineBatch = 4;               // routed rows loaded before any FMA
 constexpr int kCombineCols = kCombineThreads * kCombineVec;
 
-// Grid (T, ceil(d_vec / 512)): block = one token and 512 16-byte column vectors,
-// four per thread (strided by 128 so each load instruction is coalesced), all
+// Grid (T, ceil(d_vec / 256)): block = one token and 256 16-byte column vectors,
+// two per thread (strided by 128 so each load instruction is coalesced; two
+// rather than four keeps registers low enough for eight resident blocks), all
 // k routed rows of a vector loaded before its FMAs. shared (fp32, (T, d)) may
 // be null when N_s = 0. The slots are added in order after the shared term; a
 // dropped slot (inv_pos -1) adds nothing.
