@@ -499,6 +499,7 @@ def run_ours(args, info):
         "clocks": clock_info,
         "kernels_ms": {k: round(v, 4) for k, v in kavg.items()},
         "routing": {"touched_experts": touched, "max_rows": int(counts.max()),
+                    "p99_rows": float(counts.float().quantile(0.99)),
                     "median_rows": float(counts.float().median()),
                     "min_rows": int(counts.min())},
     }
