@@ -29,7 +29,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-DEFAULT_WORKLOAD = "coarse_t4096_d4096_f14336_e8k2_s0"
+DEFAULT_WORKLOAD = "dsv3_prefill_t4096_d7168_f2048_e256k8_s1"
 METRIC = "MoE-layer tokens/s at 1 B200; TFLOP/s vs bf16 peak (HBM GB/s when weight-bound)"
 L2_FLUSH_BYTES = 256 << 20          # twice the 126 MB L2
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -50,6 +50,10 @@ def parse_args(argv=None):
                     help="time plain stream launches instead of CUDA-graph replays")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU seconds of the oracle sample")
+    ap.add_argument("--per-workload", choices=["all", "none"], default="all",
+                    help="also measure the other four workloads (per_workload in the line)")
+    ap.add_argument("--min-seconds", type=float, default=0.25,
+                    help="least device time of each per-workload timed region")
     return ap.parse_args(argv)
 
 
@@ -95,12 +99,14 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    def __init__(self, device_index: int, period_s: float = 0.02, probe: bool = False):
         self.idx, self.period = device_index, period_s
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self._stop = threading.Event()
         self._thread = None
         self.ok = False
+        if probe:          # a sampler that samples nothing (untimed probe runs)
+            return
         try:
             import pynvml
             import torch
@@ -152,31 +158,6 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
                 "samples": len(self.samples), "source": "nvml" if self.ok else "unavailable"}
-
-
-# ----------------------------------------------------------------- work accounting
-def kernel_work(name, shape, T, touched):
-    """(flops, bytes) the kernel cannot avoid: its inputs, outputs and weights."""
-    d, f, n, k = shape.d, shape.f, shape.n_routed, shape.top_k
-    A, nsf = T * k, shape.n_shared * shape.f
-    name, _, tag = name.partition("[")  # GEMM variant tags do not change the work,
-    merged = "+shared" in tag          # except a shared GEMM merged into the launch
-    table = {
-        "router_gemm": (2 * T * d * n, 2 * n * d + 2 * T * d + 4 * T * n),
-        "route_topk": (0, 4 * T * n + 8 * A),
-        "route_scan": (0, 0),
-        "route_scatter": (0, 2 * T * d + 2 * A * d + 12 * A),
-        "grouped_gate_up": (4 * A * d * f, touched * 4 * d * f + 2 * A * d + 2 * A * f),
-        "grouped_down": (2 * A * d * f, touched * 2 * d * f + 2 * A * f + 2 * A * d),
-        "shared_gate_up": (4 * T * d * nsf, 4 * nsf * d + 2 * T * d + 2 * T * nsf),
-        "shared_down": (2 * T * d * nsf, 2 * nsf * d + 2 * T * nsf + 4 * T * d),
-        "combine": (0, 2 * A * d + (4 * T * d if nsf else 0) + 2 * T * d + 8 * A),
-    }
-    fl, by = table.get(name, (0, 0))
-    if merged:
-        sf, sb = table["shared_" + name.split("_", 1)[1]]
-        fl, by = fl + sf, by + sb
-    return fl, by
 
 
 # ----------------------------------------------------------------- oracle (CPU)
@@ -235,7 +216,7 @@ def timed_oracle(inp_host, shape, target_s, expert, max_tokens=None):
     rng = np.random.default_rng(0)
     T = shape.T if max_tokens is None else max_tokens
     order = rng.permutation(T)
-    n = min(8, T)
+    n = 1
     while True:
         dt = oracle_sample_run(inp_host, shape, np.sort(order[:n]), expert)
         if dt >= 0.6 * target_s or n >= T:
@@ -296,17 +277,54 @@ def workload_config(shape, args):
                   "weights also exceed L2"}
 
 
-def run_ours(args, info):
+def timed_steps(step, flush, stream, steps, info, clocks):
+    """Device time (ms, max over ranks) of `steps` calls of step(), L2 flushed
+    between them outside the per-step events; clocks sampled meanwhile."""
     import torch
-    from mixture_experts_ffn_expert_b200.inputs import WORKLOADS, make_layer_inputs
-    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
     from mixture_experts_ffn_expert_b200 import replicas
+    replicas.barrier(info)
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+        flush.fill_(1)
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    replicas.barrier(info)
+    return sum(a.elapsed_time(b) for a, b in ev), clock_info
 
-    dev = torch.device("cuda", info.local_rank)
-    torch.cuda.set_device(dev)
-    shape = WORKLOADS[args.workload]
-    if args.tokens:
-        shape = shape.with_tokens(args.tokens)
+
+def roofline_of(flops, nbytes, seconds, peaks, peak_src):
+    """Achieved rate against the bound that limits (flops, bytes) at the measured
+    peaks. A tensor fraction uses the burst bf16 peak (each timed region here is
+    far shorter than the seconds-long loop the sustained figure comes from)."""
+    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    if flops and t_tensor >= t_hbm:
+        ach, peak = flops / seconds / 1e12, peaks["bf16_tflops"]
+        return {"bound": "tensor", "achieved": round(ach, 2), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(ach / peak, 4), "peak_source": f"{peak_src} (bf16 burst)",
+                "frac_of_sustained_peak": round(ach / peaks["bf16_tflops_sustained"], 4)}
+    ach, peak = nbytes / seconds / 1e9, peaks["hbm_gbs"]
+    return {"bound": "hbm", "achieved": round(ach, 2), "peak": peak, "unit": "GB/s",
+            "frac": round(ach / peak, 4), "peak_source": f"{peak_src} (HBM copy)"}
+
+
+def measure_workload(shape, args, info, dev, steps, headline):
+    """One workload: warm-up, CUDA-graph capture, `steps` timed replays (None: at
+    least --steps and at least --min-seconds of device time, estimated from a
+    3-step run), a pass of plain launches with per-kernel events, and (headline
+    only) the end-to-end leg and the oracle baseline. Returns a dict."""
+    import torch
+    from mixture_experts_ffn_expert_b200 import replicas
+    from mixture_experts_ffn_expert_b200.inputs import make_layer_inputs
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    from mixture_experts_ffn_expert_b200.metrics import kernel_work, layer_bytes, layer_flops
+
     T = shape.T
     inp = make_layer_inputs(shape, seed=0, device=dev)
     layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
@@ -316,7 +334,8 @@ def run_ours(args, info):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    for _ in range(max(args.warmup, 3)):
+    warm = max(args.warmup, 3)
+    for _ in range(warm):
         layer(x, out)
         flush.fill_(1)
     torch.cuda.synchronize(dev)
@@ -349,28 +368,27 @@ def run_ours(args, info):
         else:
             layer(x, out)
 
-    # ---- timed region: device time of K steps, max over ranks
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    clocks = ClockSampler(dev.index if dev.index is not None else 0)
-    replicas.barrier(info)
-    torch.cuda.synchronize(dev)
-    clocks.start()
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-        flush.fill_(1)
-    torch.cuda.synchronize(dev)
-    replicas.barrier(info)
-    local_ms = sum(a.elapsed_time(b) for a, b in ev)
+    if steps is None:
+        # all ranks take the same count (the largest estimate)
+        probe_ms, _ = timed_steps(step, flush, stream, 3, info, ClockSampler(-1, probe=True))
+        est = replicas.max_over_ranks(probe_ms, info, device=dev) / 3 / 1e3
+        steps = int(min(5000, max(args.steps, -(-args.min_seconds // max(est, 1e-6)))))
 
-    # ---- per-kernel times: the same number of plain launches with events
-    #      recorded around every kernel on the stream it runs on
+    # ---- timed region: device time of `steps` steps, max over ranks
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    local_ms, clock_info = timed_steps(step, flush, stream, steps, info, clocks)
+    total_ms = replicas.max_over_ranks(local_ms, info, device=dev)
+    ms_per_step = total_ms / steps
+    value = info.world_size * T * steps / (total_ms / 1e3)
+
+    # ---- per-kernel times: plain launches with events recorded around every
+    #      kernel on the stream it runs on (the events between kernels break the
+    #      programmatic-launch overlap, so these are shares, not absolutes)
     layer.plan.enable_timing(True)
     ktimes = {}
     names = None
-    for i in range(args.steps):
+    n_k = max(3, min(steps, 50))
+    for i in range(n_k):
         layer(x, out)
         flush.fill_(1)
         if names is None:
@@ -381,44 +399,45 @@ def run_ours(args, info):
     for name, t in zip(names, layer.plan.kernel_times(back=0)):
         ktimes.setdefault(name, []).append(t)
     torch.cuda.synchronize(dev)
-    clock_info = clocks.stop()
     layer.plan.enable_timing(False)
     assert layer.device_status() == 0, "a kernel reported a bounded-wait timeout"
-    total_ms = replicas.max_over_ranks(local_ms, info, device=dev)
-    ms_per_step = total_ms / args.steps
-    value = info.world_size * T * args.steps / (total_ms / 1e3)
 
-    # ---- per-kernel times and the dominant kernel's roofline
+    # ---- rooflines: the layer as a whole, and its dominant kernel
     peaks, peak_src = load_peaks()
     kavg = {k: sum(v) / len(v) for k, v in ktimes.items()}
+    ksum = sum(kavg.values())
     dominant = max(kavg, key=kavg.get)
     flops, nbytes = kernel_work(dominant, shape, T, touched)
-    t_dom = kavg[dominant] / 1e3
-    t_tensor = flops / (peaks["bf16_tflops_sustained"] * 1e12)
-    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
-    if flops and t_tensor >= t_hbm:
-        achieved, peak, unit, bound = flops / t_dom / 1e12, peaks["bf16_tflops_sustained"], \
-            "TFLOP/s", "tensor"
-    else:
-        achieved, peak, unit, bound = nbytes / t_dom / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
-    roofline = {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
-                "frac": round(achieved / peak, 4), "kernel": dominant,
-                "peak_source": f"{peak_src} ({'bf16 sustained' if bound == 'tensor' else 'HBM copy'})",
-                "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": nbytes,
-                "avg_launch_ms": round(kavg[dominant], 4),
-                "traffic": profiled_traffic(dominant.split("[")[0], shape.name)}
-    if bound == "tensor":
-        roofline["frac_of_burst_peak"] = round(achieved / peaks["bf16_tflops"], 4)
-    layer_flops = (2 * T * shape.d * shape.n_routed + 6 * T * shape.top_k * shape.d * shape.f
-                   + 6 * T * shape.d * shape.n_shared * shape.f)
+    kroof = roofline_of(flops, nbytes, kavg[dominant] / 1e3, peaks, peak_src)
+    kroof.update({"kernel": dominant, "algorithmic_flops_per_launch": flops,
+                  "algorithmic_bytes_per_launch": nbytes,
+                  "avg_launch_ms": round(kavg[dominant], 4),
+                  "traffic": profiled_traffic(dominant.split("[")[0], shape.name)})
+    lflops, lbytes = layer_flops(shape), layer_bytes(shape, touched)
+    lroof = roofline_of(lflops, lbytes, ms_per_step / 1e3, peaks, peak_src)
+    lroof.update({"algorithmic_flops_per_step": lflops, "algorithmic_bytes_per_step": lbytes})
+    mhz = clock_info.get("sm_mhz")
+    res = {
+        "value": value, "ms_per_step": ms_per_step, "steps": steps,
+        "tflops": lflops / (ms_per_step / 1e3) / 1e12 * info.world_size,
+        "layer_roofline": lroof, "roofline": kroof, "clocks": clock_info,
+        "sm_kcycles_per_step": round(ms_per_step * mhz, 1) if mhz else None,
+        "gpu_launches_per_step": launches_per_step,
+        "kernels_ms": {k: round(v, 4) for k, v in kavg.items()},
+        "kernel_shares": {k: round(v / ksum, 4) for k, v in kavg.items()},
+        "routing": {"touched_experts": touched, "max_rows": int(counts.max()),
+                    "p99_rows": float(counts.float().quantile(0.99)),
+                    "median_rows": float(counts.float().median()),
+                    "min_rows": int(counts.min())},
+        "step_launch": "cuda graph replay" if graph is not None else "stream launches",
+    }
 
     # ---- end to end through the public API with pinned host buffers: every
     #      step copies its x in from pinned host memory and its output back out;
     #      the copies run on their own streams, double-buffered, so the copy-in
     #      of step i+1 and the copy-out of step i-1 overlap the forward of step i
-    e2e = None
-    if not args.no_e2e:
-        n_e2e = max(3, min(args.steps, 50))
+    if headline and not args.no_e2e:
+        n_e2e = max(3, min(steps, 50))
         x_host = [x.cpu().pin_memory() for _ in range(2)]
         out_host = [torch.empty_like(x_host[0]).pin_memory() for _ in range(2)]
         x_dev = [torch.empty_like(x) for _ in range(2)]
@@ -463,46 +482,95 @@ def run_ours(args, info):
         stop.record(stream)          # after the last copy-out
         torch.cuda.synchronize(dev)
         e_ms = replicas.max_over_ranks(start.elapsed_time(stop), info, device=dev)
-        e2e = {"value": info.world_size * T * n_e2e / (e_ms / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": x_host[0].numel() * x_host[0].element_size(),
-               "d2h_bytes_per_step": out_host[0].numel() * out_host[0].element_size(),
-               "steps": n_e2e,
-               "path": "pinned host x -> device (copy stream), moe_forward, device -> pinned "
-                       "host out (copy stream); double-buffered so copies overlap forwards; "
-                       "plain stream launches, no L2 flush (each step's x arrives by copy, "
-                       "so it is partly L2-resident when the forward starts, as in use)"}
+        res["e2e"] = {"value": info.world_size * T * n_e2e / (e_ms / 1e3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": x_host[0].numel() * x_host[0].element_size(),
+                      "d2h_bytes_per_step": out_host[0].numel() * out_host[0].element_size(),
+                      "steps": n_e2e,
+                      "path": "pinned host x -> device (copy stream), moe_forward, device -> "
+                              "pinned host out (copy stream); double-buffered so copies overlap "
+                              "forwards; plain stream launches, no L2 flush (each step's x "
+                              "arrives by copy, so it is partly L2-resident when the forward "
+                              "starts, as in use)"}
 
     # ---- CPU baseline: the oracle on a bounded sample, rank 0 at N=1 only
-    cpu = None
-    if not args.no_cpu_baseline and info.rank == 0 and info.world_size == 1:
+    if headline and not args.no_cpu_baseline and info.rank == 0 and info.world_size == 1:
         inp_host = host_copy_of_inputs(inp)
+        del inp
         expert, once = oracle_experts(inp_host, shape)
         n_tok, dt = timed_oracle(inp_host, shape, args.cpu_seconds, expert)
-        cpu = {"value": n_tok / dt, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
-               "sample": f"{n_tok} seeded tokens of T={T} (routing and experts for those "
-                         f"tokens; expert weights widened to fp64 "
-                         f"{'once, outside the timing' if once else 'inside the run'}), "
-                         f"one run of {dt:.1f} s"}
+        res["cpu_baseline"] = {
+            "value": n_tok / dt, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{n_tok} seeded tokens of T={T} (routing and experts for those "
+                      f"tokens; expert weights widened to fp64 "
+                      f"{'once, outside the timing' if once else 'inside the run'}), "
+                      f"one run of {dt:.1f} s"}
+        del inp_host
+    return res
 
-    return {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": info.world_size,
-        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+
+PER_WORKLOAD_KEYS = ("value", "ms_per_step", "steps", "tflops", "layer_roofline", "roofline",
+                     "sm_kcycles_per_step", "gpu_launches_per_step", "kernel_shares", "routing")
+
+
+def run_ours(args, info):
+    import gc
+    import torch
+    from mixture_experts_ffn_expert_b200.inputs import WORKLOADS
+
+    dev = torch.device("cuda", info.local_rank)
+    torch.cuda.set_device(dev)
+    shape = WORKLOADS[args.workload]
+    if args.tokens:
+        shape = shape.with_tokens(args.tokens)
+
+    head = measure_workload(shape, args, info, dev, args.steps, headline=True)
+    per = {}
+    if args.per_workload == "all":
+        per[shape.name] = {k: head[k] for k in PER_WORKLOAD_KEYS}
+        per[shape.name]["clocks"] = head["clocks"]
+        for name, other in WORKLOADS.items():
+            if name == shape.name:
+                continue
+            gc.collect()
+            torch.cuda.empty_cache()
+            r = measure_workload(other, args, info, dev, None, headline=False)
+            per[name] = {k: r[k] for k in PER_WORKLOAD_KEYS}
+            per[name]["clocks"] = r["clocks"]
+            per[name]["config"] = workload_config(other, args)
+            del r
+    gc.collect()
+    torch.cuda.empty_cache()
+
+    out = {
+        "metric": METRIC, "value": head["value"], "unit": "tokens/s",
+        "n_gpus": info.world_size, "steps": args.steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init weights scaled 1/sqrt(fan_in))",
         "config": workload_config(shape, args),
-        "tflops": layer_flops / (ms_per_step / 1e3) / 1e12 * info.world_size,
-        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps,
-        "step_launch": "cuda graph replay" if graph is not None else "stream launches",
-        "kernel_times_from": f"{args.steps} plain forwards after the timed region, CUDA events "
-                             "around each kernel on its own stream",
-        "clocks": clock_info,
-        "kernels_ms": {k: round(v, 4) for k, v in kavg.items()},
-        "routing": {"touched_experts": touched, "max_rows": int(counts.max()),
-                    "p99_rows": float(counts.float().quantile(0.99)),
-                    "median_rows": float(counts.float().median()),
-                    "min_rows": int(counts.min())},
+        "tflops": head["tflops"], "roofline": head["roofline"],
+        "layer_roofline": head["layer_roofline"],
+        "cpu_baseline": head.get("cpu_baseline"), "e2e": head.get("e2e"),
+        "gpu_launches": head["gpu_launches_per_step"] * args.steps,
+        "step_launch": head["step_launch"],
+        "clocks": head["clocks"], "sm_kcycles_per_step": head["sm_kcycles_per_step"],
+        "kernels_ms": head["kernels_ms"],
+        "kernels_ms_basis": "plain stream launches with CUDA events around each kernel on its "
+                            "own stream, after the timed region; the events break the "
+                            "programmatic-launch overlap, so use them as shares only",
+        "kernel_shares": head["kernel_shares"],
+        "routing": head["routing"],
     }
+    if per:
+        out["per_workload"] = per
+        out["per_workload_basis"] = (
+            "every workload of the layer's five configurations, measured the same way as the "
+            "headline (CUDA-graph replays, L2 flushed between steps, device time); steps per "
+            "workload >= --steps and >= --min-seconds of device time; layer_roofline = the "
+            "layer's algorithmic FLOPs or bytes per step / ms_per_step against the measured "
+            "bf16 burst peak or HBM copy bandwidth, whichever bounds the layer; "
+            "sm_kcycles_per_step = ms_per_step x median SM MHz (compare across clock states)")
+    return out
 
 
 def main(argv=None):

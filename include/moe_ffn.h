@@ -99,8 +99,15 @@ int moe_last_status(void);
  *   min(count_e, C) of the (token, slot) pairs routed to it, in ascending
  *   (token, slot) order; a dropped pair adds nothing to its token's output, the
  *   kept gates are not renormalised and the shared expert still applies. This
- *   option changes results; the others do not. A capacity factor cf maps to
- *   C = ceil(cf * T * top_k / N_r).
+ *   option changes results; the others do not (setting it turns the capacity
+ *   factor below off).
+ * MOE_OPTION_CAPACITY_FACTOR_PERMILLE: the same token dropping stated as the
+ *   glossary's capacity factor cf, passed in thousandths (1000 = 1.0; 0, the
+ *   default, turns it off). A forward over T tokens then gives each expert
+ *   C = max(1, ceil(cf * T * top_k / N_r)) seats - the factor times an
+ *   expert's even share of the batch's T*top_k routed pairs (the glossary
+ *   names the factor without a formula; this is the conventional one). Setting
+ *   it turns MOE_OPTION_EXPERT_CAPACITY off. moe_plan_capacity_seats reports C.
  * MOE_OPTION_BIAS_SELECTION_ONLY: 0 (default): the logit bias set with
  *   moe_plan_set_logit_bias is added to the router scores for both the top-k
  *   selection and the gates. 1: it only chooses the experts (the selection-only
@@ -120,6 +127,7 @@ enum {
   MOE_OPTION_MERGE_SHARED = 3,
   MOE_OPTION_EXPERT_CAPACITY = 4,
   MOE_OPTION_BIAS_SELECTION_ONLY = 5,
+  MOE_OPTION_CAPACITY_FACTOR_PERMILLE = 6,
   MOE_OPTION_TEST_WAIT_TIMEOUT = 100
 };
 int moe_plan_set_option(moe_plan_t plan, int option, int64_t value);
@@ -170,10 +178,13 @@ int moe_get_routing(moe_plan_t plan, int64_t T, int32_t* idx, float* w,
 int moe_get_permutation(moe_plan_t plan, int64_t T, int32_t* perm_src,
                         int32_t* inv_pos, void* stream);
 
-/* Read (synchronously) and clear the plan's device status word: MOE_OK, or
- * MOE_DEVICE_TIMEOUT if a kernel abandoned a bounded wait since the last
- * read. Kernels never spin without a bound; a timeout means the forward's
- * output is invalid. */
+/* Read (synchronously) and clear the plan's device status: MOE_OK, or
+ * MOE_DEVICE_TIMEOUT if a kernel abandoned a bounded wait since the last read.
+ * It covers the forwards that ran on the plan's workspace and, when this plan
+ * has run moe_forward_noalloc since the last read, the status word of the
+ * static scratch those forwards share (one word for every plan of the
+ * process: a read through any plan that used it clears it). Kernels never spin
+ * without a bound; a timeout means that forward's output is invalid. */
 int moe_plan_device_status(moe_plan_t plan);
 
 /* Timing: when enabled, moe_forward records a CUDA event on its stream before
@@ -191,22 +202,23 @@ int moe_plan_kernel_times(moe_plan_t plan, int back, float* ms, int cap);
 const char* moe_plan_kernel_name(moe_plan_t plan, int i);
 
 /* Forward for callers that cannot allocate device memory - for instance a
- * plugin whose host application owns the whole device-memory budget, or a
- * latency-critical loop where cudaMalloc would synchronise the device. The
- * pages have no counterpart of this call; it is a deployment convenience.
- * Same arguments and result as moe_forward, but the scratch the layer needs
- * lives in one static device array of 32 MiB inside the library (held on
- * every GPU that loads the library until the process exits) instead of the
- * plan's workspace; the caller passes only inputs and outputs, and nothing is
- * allocated by the call. T whose scratch would exceed 32 MiB is rejected with
+ * plugin whose host application owns the whole device-memory budget through
+ * its own pool, or a latency-critical loop where cudaMalloc would synchronise
+ * the device. The pages have no counterpart of this call; it is a deployment
+ * convenience. Same arguments and result as moe_forward, but the scratch the
+ * layer needs lives in one static device array of 32 MiB inside the library
+ * (held on every GPU that loads the library until the process exits) instead
+ * of the plan's workspace; the caller passes only inputs and outputs, and the
+ * call allocates nothing. T whose scratch would exceed 32 MiB is rejected with
  * MOE_WORKSPACE_TOO_SMALL before anything is enqueued (the 512-expert decode
  * shape d=2048, f=512, N_r=512, k=10, N_s=1 needs about 13 MiB at T=128).
- * The first call on a device looks up the array's device address (with that
- * device current); make that first call before any stream capture. All calls
- * share the one array and it keeps the last call's contents: two calls that
- * overlap on the GPU (different streams, plans or threads) race, so keep them
- * on one stream. Timing events are not recorded, and moe_get_routing /
- * moe_get_permutation / moe_plan_device_status do not see these forwards. */
+ * moe_plan_create looks up the array's device address (with the plan's device
+ * current), so the call itself makes no lookup. All calls share the one array
+ * and it keeps the last call's contents: two calls that overlap on the GPU
+ * (different streams, plans or threads) race, so keep them on one stream.
+ * Timing events are not recorded. The plan's routing, permutation, launch
+ * count and kernel-name getters keep describing the last moe_forward; a
+ * bounded-wait timeout is reported by moe_plan_device_status. */
 int moe_forward_noalloc(moe_plan_t plan, int64_t T, const moe_bf16_t* x,
                         const moe_bf16_t* W_g, const moe_bf16_t* W1,
                         const moe_bf16_t* W3, const moe_bf16_t* W2,
@@ -215,6 +227,11 @@ int moe_forward_noalloc(moe_plan_t plan, int64_t T, const moe_bf16_t* x,
 
 /* Number of kernels the last forward of this plan launched. */
 int moe_plan_last_launch_count(moe_plan_t plan);
+
+/* Seats per expert a forward over T tokens gives each expert under the plan's
+ * capacity options (0: unlimited, the layer is dropless); a negative
+ * moe_status on a NULL plan or negative T. Host only, enqueues nothing. */
+int64_t moe_plan_capacity_seats(moe_plan_t plan, int64_t T);
 
 void moe_plan_destroy(moe_plan_t plan);
 

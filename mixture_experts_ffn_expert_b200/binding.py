@@ -20,13 +20,14 @@ EXPORTED_SYMBOLS = [
     "moe_plan_set_workspace", "moe_forward", "moe_get_routing", "moe_get_permutation",
     "moe_plan_device_status", "moe_plan_enable_timing", "moe_plan_kernel_times",
     "moe_plan_kernel_name", "moe_plan_last_launch_count", "moe_plan_destroy", "moe_strerror",
-    "moe_last_error", "moe_forward_noalloc", "moe_plan_set_option",
+    "moe_last_error", "moe_forward_noalloc", "moe_plan_set_option", "moe_plan_capacity_seats",
 ]
 MOE_OPTION_PAIR_MIN_ROWS = 1
 MOE_OPTION_WIDE_TILES = 2
 MOE_OPTION_MERGE_SHARED = 3
 MOE_OPTION_EXPERT_CAPACITY = 4
 MOE_OPTION_BIAS_SELECTION_ONLY = 5
+MOE_OPTION_CAPACITY_FACTOR_PERMILLE = 6
 MOE_OPTION_TEST_WAIT_TIMEOUT = 100
 
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_INVALID_CONFIG", 2: "MOE_INVALID_ARG",
@@ -71,6 +72,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_plan_kernel_times": (_i, [_vp, _i, ctypes.POINTER(ctypes.c_float), _i]),
         "moe_plan_kernel_name": (ctypes.c_char_p, [_vp, _i]),
         "moe_plan_last_launch_count": (_i, [_vp]),
+        "moe_plan_capacity_seats": (_i64, [_vp, _i64]),
         "moe_plan_destroy": (None, [_vp]),
         "moe_strerror": (ctypes.c_char_p, [_i]),
         "moe_last_error": (ctypes.c_char_p, []),
@@ -153,6 +155,13 @@ class Plan:
 
     def last_launch_count(self) -> int:
         return int(self.lib.moe_plan_last_launch_count(self.handle))
+
+    def capacity_seats(self, T: int) -> int:
+        """Seats per expert a forward over T tokens uses (0: dropless)."""
+        n = int(self.lib.moe_plan_capacity_seats(self.handle, T))
+        if n < 0:
+            _check(self.lib, -n)
+        return n
 
     def close(self) -> None:
         if getattr(self, "handle", None):

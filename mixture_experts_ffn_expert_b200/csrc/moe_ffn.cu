@@ -71,6 +71,9 @@ struct moe_plan {
   int merge_shared = 0;
   // seats per expert per forward (token dropping); 0: unlimited (dropless)
   int64_t capacity = 0;
+  // capacity factor in thousandths: seats = ceil(factor * T * top_k / N_r) per
+  // forward over T tokens; 0: off (capacity above applies)
+  int64_t capacity_permille = 0;
   // 1: the logit bias only chooses the experts, the gates come from unbiased scores
   int bias_select_only = 0;
   // one-shot test hook: the next forward's routed gate/up GEMM (single-CTA
@@ -93,6 +96,11 @@ struct moe_plan {
   // the shared expert runs on a forked stream, concurrently with the routing
   cudaStream_t side = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
+  // device address of the allocation-free forward's static scratch in this
+  // plan's context (looked up at plan creation), and whether a forward of this
+  // plan has used it since moe_plan_device_status last read its status word
+  void* noalloc_scratch = nullptr;
+  bool noalloc_used = false;
 };
 
 namespace {
@@ -333,6 +341,52 @@ int set_kernel_attributes() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Seats per expert for a forward over T tokens: the explicit capacity, or the
+// capacity factor times an expert's even share of the T*top_k routed pairs,
+// rounded up (at least 1); 0 means unlimited.
+int64_t capacity_seats(const moe_plan* p, int64_t T) {
+  if (p->capacity_permille > 0) {
+    const int64_t num = p->capacity_permille * T * p->top_k;
+    const int64_t den = 1000LL * p->n_routed;
+    const int64_t c = (num + den - 1) / den;
+    return c < 1 ? 1 : c;
+  }
+  return p->capacity;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Static scratch of the allocation-free forward (moe_forward_noalloc).
+//
+// Some callers cannot allocate device memory at all: a plugin inside a host
+// application that owns the whole device-memory budget through its own pool,
+// or a latency-critical loop where cudaMalloc would synchronise the device.
+// For them the layer's scratch lives in one file-scope device array instead
+// of a caller workspace. Every GPU that loads this library holds the array
+// (kNoAllocScratchBytes) until the process exits.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;   // 32 MiB
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the array in the current device's context. In host code
+// the array's name only stands in for the symbol, so the address is looked up
+// with the plan's device current, when the plan is created, and kept in the
+// plan (which is bound to that context).
+int noalloc_scratch_address(void** out) {
+  void* ptr = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+  if (e != cudaSuccess || !ptr) {
+    cudaGetLastError();
+    return fail(MOE_CUDA_ERROR, "cudaGetSymbolAddress of the static scratch failed: %s",
+                cudaGetErrorString(e));
+  }
+  *out = ptr;
+  return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -389,6 +443,10 @@ moe_plan_t moe_plan_create(int d, int f, int n_routed, int top_k, int n_shared, 
     moe_plan_destroy(p);
     return nullptr;
   }
+  if (noalloc_scratch_address(&p->noalloc_scratch) != MOE_OK) {
+    moe_plan_destroy(p);
+    return nullptr;
+  }
   return p;
 }
 
@@ -420,6 +478,13 @@ int moe_plan_set_option(moe_plan_t p, int option, int64_t value) {
     case MOE_OPTION_EXPERT_CAPACITY:
       if (value < 0) return fail(MOE_INVALID_ARG, "expert capacity must be >= 0");
       p->capacity = value;
+      p->capacity_permille = 0;
+      return MOE_OK;
+    case MOE_OPTION_CAPACITY_FACTOR_PERMILLE:
+      if (value < 0 || value > (1LL << 20))
+        return fail(MOE_INVALID_ARG, "capacity factor (permille) must be in [0, 2^20]");
+      p->capacity_permille = value;
+      p->capacity = 0;
       return MOE_OK;
     default:
       return fail(MOE_INVALID_ARG, "unknown option %d", option);
@@ -642,8 +707,8 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   }
   // 4. offsets + m-tile prefix, stable permutation, 16-byte row copies (with a
   //    seat limit, only each expert's first `capacity` pairs get rows)
-  const int seat_limit =
-      p->capacity > 0 && p->capacity < INT_MAX ? static_cast<int>(p->capacity) : INT_MAX;
+  const int64_t seats = capacity_seats(p, T);
+  const int seat_limit = seats > 0 && seats < INT_MAX ? static_cast<int>(seats) : INT_MAX;
   {
     const size_t smem = size_t(moe::kMaxRouted + nr) * 4 + size_t(2) * Lw.tpc * k * 4;
     // split the row copy into column slices of at least 32 vectors so that
@@ -805,12 +870,22 @@ int moe_get_permutation(moe_plan_t p, int64_t T, int32_t* perm_src, int32_t* inv
 
 int moe_plan_device_status(moe_plan_t p) {
   if (!p) return fail(MOE_INVALID_ARG, "null plan");
-  if (!p->ws) return MOE_OK;
-  int v = 0;
-  cudaError_t e = cudaMemcpy(&v, p->ws, sizeof(int), cudaMemcpyDeviceToHost);
-  if (e == cudaSuccess) e = cudaMemset(p->ws, 0, sizeof(int));
-  if (e != cudaSuccess) return fail(MOE_CUDA_ERROR, "device status read: %s", cudaGetErrorString(e));
-  if (v != MOE_OK) return fail(v, "a kernel gave up a bounded wait (device status %d)", v);
+  // the plan's workspace, and the static scratch when this plan's allocation-free
+  // forwards have used it since the last read
+  void* words[2] = {p->ws, p->noalloc_used ? p->noalloc_scratch : nullptr};
+  int worst = MOE_OK;
+  for (void* w : words) {
+    if (!w) continue;
+    int v = 0;
+    cudaError_t e = cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemset(w, 0, sizeof(int));
+    if (e != cudaSuccess)
+      return fail(MOE_CUDA_ERROR, "device status read: %s", cudaGetErrorString(e));
+    if (v != MOE_OK) worst = v;
+  }
+  p->noalloc_used = false;
+  if (worst != MOE_OK)
+    return fail(worst, "a kernel gave up a bounded wait (device status %d)", worst);
   return MOE_OK;
 }
 
@@ -848,48 +923,12 @@ const char* moe_plan_kernel_name(moe_plan_t p, int i) {
 
 int moe_plan_last_launch_count(moe_plan_t p) { return p ? p->n_launch : 0; }
 
-}  // extern "C"
-
-// ---------------------------------------------------------------------------
-// Forward without caller-provided scratch.
-//
-// Some callers cannot allocate device memory at all: a plugin inside a host
-// application that owns the whole device-memory budget through its own pool,
-// or a latency-critical loop where cudaMalloc would synchronise the device.
-// For them the layer's scratch lives in one file-scope device array instead
-// of a caller workspace. Every GPU that loads this library holds the array
-// (kNoAllocScratchBytes) until the process exits.
-namespace {
-
-constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;   // 32 MiB
-constexpr int kNoAllocMaxDevices = 64;
-
-static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
-
-std::mutex g_noalloc_mutex;
-void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
-
-// Device address of the array on the current device. In host code the
-// array's name only stands in for the symbol, so the address is looked up once
-// per device (with that device current) and cached.
-int noalloc_scratch(int dev, void** out) {
-  if (dev < 0 || dev >= kNoAllocMaxDevices)
-    return fail(MOE_UNSUPPORTED, "device %d is beyond the %d devices supported", dev,
-                kNoAllocMaxDevices);
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_ptr[dev]) {
-    void* ptr = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess || !ptr)
-      return fail(MOE_CUDA_ERROR, "cudaGetSymbolAddress of the static scratch failed: %s",
-                  cudaGetErrorString(e));
-    g_noalloc_ptr[dev] = ptr;
-  }
-  *out = g_noalloc_ptr[dev];
-  return MOE_OK;
+int64_t moe_plan_capacity_seats(moe_plan_t p, int64_t T) {
+  if (!p || T < 0) return -fail(MOE_INVALID_ARG, "null plan or negative T");
+  return capacity_seats(p, T);
 }
 
-}  // namespace
+}  // extern "C"
 
 extern "C" {
 
@@ -905,29 +944,32 @@ int moe_forward_noalloc(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_
                 "T=%lld needs %zu bytes of scratch; the static scratch of moe_forward_noalloc "
                 "holds %zu bytes (use moe_forward with a caller workspace)",
                 (long long)T, need, kNoAllocScratchBytes);
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev != p->device)
-    return fail(MOE_INVALID_ARG, "plan was created on device %d, current device is %d",
-                p->device, dev);
-  void* scratch = nullptr;
-  int rc = noalloc_scratch(dev, &scratch);
-  if (rc != MOE_OK) return rc;
-  // The status word is the only scratch that must start at zero.
-  cudaError_t e = cudaMemsetAsync(scratch, 0, 256, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return fail(MOE_CUDA_ERROR, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+  if (!p->noalloc_scratch)
+    return fail(MOE_CUDA_ERROR, "the plan has no address for the static scratch");
   // Run the regular forward on the static scratch, with timing off so that no
-  // events are created, then give the plan its own workspace back.
+  // events are created, then give the plan back its own workspace and the state
+  // its getters report (routing, permutation, launch count and kernel names
+  // keep describing the last moe_forward, whose routing is still in the
+  // plan's workspace). The status word at the start of the scratch is not
+  // cleared here: a bounded-wait timeout stays visible to moe_plan_device_status.
   char* saved_ws = p->ws;
   const size_t saved_bytes = p->ws_bytes;
   const bool saved_timing = p->timing;
-  p->ws = static_cast<char*>(scratch);
+  const int64_t saved_T = p->last_T;
+  const int saved_launch = p->n_launch;
+  char saved_names[kMaxKernels][48];
+  memcpy(saved_names, p->names, sizeof(saved_names));
+  p->ws = static_cast<char*>(p->noalloc_scratch);
   p->ws_bytes = kNoAllocScratchBytes;
   p->timing = false;
-  rc = moe_forward(p, T, x, W_g, W1, W3, W2, W1s, W3s, W2s, out, stream);
+  const int rc = moe_forward(p, T, x, W_g, W1, W3, W2, W1s, W3s, W2s, out, stream);
   p->ws = saved_ws;
   p->ws_bytes = saved_bytes;
   p->timing = saved_timing;
-  p->last_T = -1;   // the routing getters read the plan's own workspace only
+  p->last_T = saved_T;
+  p->n_launch = saved_launch;
+  memcpy(p->names, saved_names, sizeof(saved_names));
+  if (rc == MOE_OK && T > 0) p->noalloc_used = true;
   return rc;
 }
 

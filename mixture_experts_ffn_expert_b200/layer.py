@@ -6,26 +6,15 @@ libmoe_ffn.so. A missing library raises instead of falling back to anything.
 """
 from __future__ import annotations
 
-import math
 from typing import Dict, Optional
 
 import torch
 
-from .binding import (MOE_OPTION_BIAS_SELECTION_ONLY, MOE_OPTION_EXPERT_CAPACITY,
-                      MOE_OPTION_MERGE_SHARED, MOE_OPTION_PAIR_MIN_ROWS, MOE_OPTION_WIDE_TILES,
-                      MoEError, Plan)
+from .binding import (MOE_OPTION_BIAS_SELECTION_ONLY, MOE_OPTION_CAPACITY_FACTOR_PERMILLE,
+                      MOE_OPTION_EXPERT_CAPACITY, MOE_OPTION_MERGE_SHARED,
+                      MOE_OPTION_PAIR_MIN_ROWS, MOE_OPTION_WIDE_TILES, MoEError, Plan)
 
-__all__ = ["MoELayer", "MoEError", "capacity_from_factor"]
-
-
-def capacity_from_factor(factor: float, T: int, top_k: int, n_routed: int) -> int:
-    """Seats per expert for a capacity factor: ceil(factor * T * top_k / N_r), the
-    factor times an expert's share of the batch's T*top_k routed pairs (at
-    least 1). This is the conventional reading of the "capacity factor" of the
-    "What is an expert, really?" glossary, which names it without a formula."""
-    if factor <= 0:
-        raise MoEError(2, "capacity factor must be positive")
-    return max(1, math.ceil(factor * T * top_k / n_routed))
+__all__ = ["MoELayer", "MoEError"]
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -38,9 +27,10 @@ class MoELayer:
     ``weights`` holds W_g (N_r, d), W1, W3 (N_r, f, d), W2 (N_r, d, f) and, when
     n_shared > 0, W1s, W3s (N_s*f, d), W2s (d, N_s*f), all bf16 contiguous on
     the device; ``bias`` is an optional fp32 (N_r,) logit bias. ``capacity``
-    (seats per expert per forward, see ``capacity_from_factor``) turns on token
-    dropping; ``bias_selection_only`` makes the bias choose experts without
-    entering the gates; the other options only select kernels.
+    (seats per expert per forward) or ``capacity_factor`` (the library gives each
+    expert ceil(factor * T * top_k / N_r) seats per forward over T tokens) turns
+    on token dropping; ``bias_selection_only`` makes the bias choose experts
+    without entering the gates; the other options only select kernels.
     """
 
     def __init__(self, d: int, f: int, n_routed: int, top_k: int, n_shared: int,
@@ -48,7 +38,7 @@ class MoELayer:
                  bias: Optional[torch.Tensor] = None, device=None,
                  pair_min_rows: Optional[int] = None, wide_tiles: Optional[int] = None,
                  merge_shared: Optional[int] = None, capacity: Optional[int] = None,
-                 bias_selection_only: bool = False):
+                 bias_selection_only: bool = False, capacity_factor: Optional[float] = None):
         dev = torch.device(device) if device is not None else torch.device("cuda")
         if dev.type == "cuda" and dev.index is None:
             dev = torch.device("cuda", torch.cuda.current_device())
@@ -64,9 +54,15 @@ class MoELayer:
         if merge_shared is not None:
             self.plan.set_option(MOE_OPTION_MERGE_SHARED, merge_shared)
         # seats per expert per forward (token dropping); None or 0: dropless
-        self.capacity = capacity or 0
+        if capacity and capacity_factor:
+            raise MoEError(2, "give either capacity or capacity_factor, not both")
         if capacity:
             self.plan.set_option(MOE_OPTION_EXPERT_CAPACITY, capacity)
+        if capacity_factor:
+            if capacity_factor <= 0:
+                raise MoEError(2, "capacity factor must be positive")
+            self.plan.set_option(MOE_OPTION_CAPACITY_FACTOR_PERMILLE,
+                                 int(round(capacity_factor * 1000)))
         self.bias_selection_only = bool(bias_selection_only)
         if bias_selection_only:
             self.plan.set_option(MOE_OPTION_BIAS_SELECTION_ONLY, 1)
@@ -134,6 +130,10 @@ class MoELayer:
                               r["offsets"].data_ptr(), stream)
         self.plan.get_permutation(T, r["perm_src"].data_ptr(), r["inv_pos"].data_ptr(), stream)
         return r
+
+    def capacity_seats(self, T: int) -> int:
+        """Seats per expert a forward over T tokens uses (0: dropless)."""
+        return self.plan.capacity_seats(T)
 
     def device_status(self) -> int:
         return self.plan.device_status()

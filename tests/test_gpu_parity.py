@@ -12,7 +12,7 @@ import torch
 
 from mixture_experts_ffn_expert_b200.inputs import LayerShape, WORKLOADS, make_layer_inputs
 
-from parity import full_parity
+from parity import check_output, check_routing, full_parity, oracle_out, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -244,17 +244,45 @@ def test_selection_only_bias_on_the_decode_shape():
     torch.cuda.empty_cache()
 
 
-def test_capacity_from_factor_on_the_deepseek_v3_shape():
-    from mixture_experts_ffn_expert_b200.layer import capacity_from_factor
+def test_capacity_factor_seats_computed_by_the_library():
+    # the glossary's capacity factor passed through the C ABI (thousandths); the
+    # seats are ceil(cf * T * k / N_r), at least one, written out here by hand
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    shape = LayerShape("cf", 8, 128, 64, 256, 8, 0, True, "none")
+    inp = make_layer_inputs(shape, seed=0, device="cuda")
+    for cf, T, want in [(1.0, 4096, 128), (1.25, 4096, 160), (0.001, 10, 1), (0.5, 1000, 16)]:
+        layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, 0, True, inp,
+                         device="cuda", capacity_factor=cf)
+        assert layer.capacity_seats(T) == want, (cf, T)
+    shape7 = LayerShape("cf7", 8, 128, 64, 7, 3, 0, True, "none")
+    inp7 = make_layer_inputs(shape7, seed=0, device="cuda")
+    layer = MoELayer(128, 64, 7, 3, 0, True, inp7, device="cuda", capacity_factor=1.0)
+    assert layer.capacity_seats(100) == 43            # 300 / 7 = 42.86, rounded up
+    layer = MoELayer(128, 64, 7, 3, 0, True, inp7, device="cuda", capacity=5)
+    assert layer.capacity_seats(100) == 5
+    layer = MoELayer(128, 64, 7, 3, 0, True, inp7, device="cuda")
+    assert layer.capacity_seats(100) == 0
+
+
+def test_capacity_factor_on_the_deepseek_v3_shape():
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
     shape = WORKLOADS["dsv3_prefill_t4096_d7168_f2048_e256k8_s1"]
     inp = make_layer_inputs(shape, seed=0, device="cuda")
-    cap = capacity_from_factor(1.0, shape.T, shape.top_k, shape.n_routed)
+    cap = -(-shape.T * shape.top_k // shape.n_routed)        # factor 1.0: 128 seats
     assert cap == 128
+    layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
+                     shape.renorm, inp, bias=inp["bias"], device="cuda", capacity_factor=1.0)
+    assert layer.capacity_seats(shape.T) == cap
+    out = layer(inp["x"])
+    routing = layer.routing()
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    _, idx_ref, _ = check_routing(inp, routing, shape, capacity=cap)
     tokens = np.sort(np.random.default_rng(77).choice(shape.T, size=24, replace=False))
-    res = full_parity(inp, shape, tokens=tokens, capacity=cap)
-    inv = res["layer"].routing()["inv_pos"].cpu().numpy()
-    assert (inv < 0).any()          # the skewed bias overflows some experts
-    del inp
+    ref = oracle_out(inp, shape, idx_ref, tokens, capacity=cap)
+    check_output(to64(out[torch.as_tensor(tokens, device=out.device)]), ref)
+    assert (routing["inv_pos"].cpu().numpy() < 0).any()   # the skewed bias overflows some experts
+    del inp, layer
     torch.cuda.empty_cache()
 
 
