@@ -56,7 +56,10 @@ typedef enum {
   MOE_WORKSPACE_TOO_SMALL = 3,
   MOE_CUDA_ERROR = 4,       /* a CUDA runtime/driver call or launch failed */
   MOE_UNSUPPORTED = 5,      /* valid layer the kernels do not cover */
-  MOE_DEVICE_TIMEOUT = 6    /* a kernel gave up a bounded wait (see moe_plan_device_status) */
+  MOE_DEVICE_TIMEOUT = 6,   /* a kernel gave up a bounded wait (see moe_plan_device_status) */
+  MOE_DEVICE_INCONSISTENT = 7 /* the permutation kernel found routing totals that do not add
+                                 up (scratch overwritten during a forward); that forward wrote
+                                 no grouped rows and dropped every routed slot */
 } moe_status;
 
 /* Create a plan for one layer shape.
@@ -114,6 +117,23 @@ int moe_last_status(void);
  *   load-balance bias "Shared Expert (DeepSeek-V3)" mentions for the routed
  *   centroids); the gates are the softmax of the unbiased scores over all N_r
  *   experts, renormalised over the selected ones when the plan renormalises.
+ * MOE_OPTION_FUSED_ROUTER: -1 (default) computes the router in one kernel
+ *   (scores on the tensor core, softmax, top-k, gates and the expert
+ *   histogram of each 128-token tile, with its K range split over a cluster of
+ *   up to 8 CTAs) whenever N_r <= 512, else in two (a split-K scores GEMM, then
+ *   softmax + top-k); 0 always uses the two-kernel router; 1 is the same as -1.
+ *   Both give the same selection up to fp32 rounding of the scores.
+ * MOE_OPTION_SWIGLU_TILE_COLS: output columns of one tile of the routed
+ *   gate/up GEMM when it runs one CTA per tile: 0 (default) chooses 64 when the
+ *   expected rows per expert (T*top_k/N_r) are below 32 - the weight-streaming
+ *   decode regime, where twice as many, shorter tiles leave a shorter last
+ *   wave - and 128 otherwise; 64 or 128 force it.
+ * MOE_OPTION_SHARED_CONCURRENT: where a shared expert too large for the
+ *   routing phase runs. -1 (default): beside the routed GEMMs, on a second
+ *   stream and a few SMs (the routed GEMMs keep the rest), when those stream
+ *   weights (fewer than 192 expected rows per expert); else after them on the
+ *   caller's stream. 1: always beside them; 0: never. Small shared experts
+ *   always run beside the routing kernels.
  * MOE_OPTION_TEST_WAIT_TIMEOUT: test hook for the failure path, not for normal
  *   use. Value 1 arms it for the next forward only: if that forward runs the
  *   routed gate/up GEMM on the one-CTA-per-tile kernel, one CTA withholds the
@@ -128,6 +148,9 @@ enum {
   MOE_OPTION_EXPERT_CAPACITY = 4,
   MOE_OPTION_BIAS_SELECTION_ONLY = 5,
   MOE_OPTION_CAPACITY_FACTOR_PERMILLE = 6,
+  MOE_OPTION_FUSED_ROUTER = 7,
+  MOE_OPTION_SWIGLU_TILE_COLS = 8,
+  MOE_OPTION_SHARED_CONCURRENT = 9,
   MOE_OPTION_TEST_WAIT_TIMEOUT = 100
 };
 int moe_plan_set_option(moe_plan_t plan, int option, int64_t value);
@@ -179,7 +202,9 @@ int moe_get_permutation(moe_plan_t plan, int64_t T, int32_t* perm_src,
                         int32_t* inv_pos, void* stream);
 
 /* Read (synchronously) and clear the plan's device status: MOE_OK, or
- * MOE_DEVICE_TIMEOUT if a kernel abandoned a bounded wait since the last read.
+ * MOE_DEVICE_TIMEOUT if a kernel abandoned a bounded wait since the last read
+ * (MOE_DEVICE_INCONSISTENT if the permutation kernel found inconsistent routing
+ * state).
  * It covers the forwards that ran on the plan's workspace and, when this plan
  * has run moe_forward_noalloc since the last read, the status word of the
  * static scratch those forwards share (one word for every plan of the

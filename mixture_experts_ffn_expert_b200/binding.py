@@ -28,11 +28,14 @@ MOE_OPTION_MERGE_SHARED = 3
 MOE_OPTION_EXPERT_CAPACITY = 4
 MOE_OPTION_BIAS_SELECTION_ONLY = 5
 MOE_OPTION_CAPACITY_FACTOR_PERMILLE = 6
+MOE_OPTION_FUSED_ROUTER = 7
+MOE_OPTION_SWIGLU_TILE_COLS = 8
+MOE_OPTION_SHARED_CONCURRENT = 9
 MOE_OPTION_TEST_WAIT_TIMEOUT = 100
 
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_INVALID_CONFIG", 2: "MOE_INVALID_ARG",
                 3: "MOE_WORKSPACE_TOO_SMALL", 4: "MOE_CUDA_ERROR", 5: "MOE_UNSUPPORTED",
-                6: "MOE_DEVICE_TIMEOUT"}
+                6: "MOE_DEVICE_TIMEOUT", 7: "MOE_DEVICE_INCONSISTENT"}
 
 
 class MoEError(RuntimeError):

@@ -90,10 +90,25 @@ struct GemmParams {
   int test_withhold;
 };
 
+// Single-CTA kernel shapes: BN accumulator columns per tile (MMA N). BN = 256
+// is the default; BN = 128 (SwiGLU only: 64 gate + 64 up columns, 64 output
+// columns per tile) halves the weight bytes per tile, so that weight-streaming
+// launches with few rows per expert split into more, shorter tiles and their
+// last wave is shorter, and it keeps four accumulators in TMEM.
+template <int BN>
+struct SingleCfg {
+  static constexpr int kBBytes = BN * kBK * 2;                // B rows per stage
+  static constexpr int kStage = kATileBytes + kBBytes;        // 48 KB (256), 32 KB (128)
+  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kAcc = 512 / BN;                       // accumulators in TMEM
+  static constexpr int kHalfRows = BN / 2;                    // rows of one SwiGLU B box
+};
+
 // Dynamic shared memory the kernel needs for a given number of groups.
+template <int BN = 256>
 __host__ __device__ constexpr size_t gemm_smem_bytes(int num_groups) {
-  return 1024 /* alignment slack */ + size_t(kStages) * kStageBytes + 256 /* barriers */ +
-         size_t(2) * (num_groups + 1) * sizeof(int);
+  return 1024 /* alignment slack */ + size_t(SingleCfg<BN>::kStages) * SingleCfg<BN>::kStage +
+         256 /* barriers */ + size_t(2) * (num_groups + 1) * sizeof(int);
 }
 
 struct TileCoord {
@@ -162,12 +177,18 @@ __device__ __forceinline__ void raise_timeout(volatile int* s_abort, int* status
 }
 
 
-template <int MODE>
+template <int MODE, int BN = 256>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmA2,
                     const __grid_constant__ CUtensorMap tmB0x, const __grid_constant__ CUtensorMap tmB1x,
                     const GemmParams P) {
+  static_assert(BN == 256 || (BN == 128 && MODE == kEpiSwiGLU), "BN 128 is a SwiGLU shape");
+  using Cfg = SingleCfg<BN>;
+  constexpr int kStages = Cfg::kStages;
+  constexpr int kStageBytes = Cfg::kStage;
+  constexpr int kNumAcc = Cfg::kAcc;
+  constexpr int kHalfBytes = Cfg::kHalfRows * kBK * 2;       // one SwiGLU B box
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -285,15 +306,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int k0 = kb * kBK;
           mbar_arrive_expect_tx(fb, kStageBytes);
           tma_load_2d(a_dst, mA, fb, k0, tc.row0);
+          // SwiGLU: BN/2 rows of W1 then the same rows of W3; plain: two
+          // 128-row boxes of the one weight
           const CUtensorMap* b1 = MODE == kEpiSwiGLU ? mB1 : mB0;
-          const int n0 = MODE == kEpiSwiGLU ? tc.n_blk * 128 : tc.n_blk * 256;
+          const int n0 = MODE == kEpiSwiGLU ? tc.n_blk * (BN / 2) : tc.n_blk * 256;
           const int n1 = MODE == kEpiSwiGLU ? n0 : n0 + 128;
+          const uint32_t b_hi = b_dst + (MODE == kEpiSwiGLU ? kHalfBytes : kBHalfBytes);
           if (stream) {
             tma_load_3d_hint(b_dst, mB0, fb, k0, n0, z, once);
-            tma_load_3d_hint(b_dst + kBHalfBytes, b1, fb, k0, n1, z, once);
+            tma_load_3d_hint(b_hi, b1, fb, k0, n1, z, once);
           } else {
             tma_load_3d(b_dst, mB0, fb, k0, n0, z);
-            tma_load_3d(b_dst + kBHalfBytes, b1, fb, k0, n1, z);
+            tma_load_3d(b_hi, b1, fb, k0, n1, z);
           }
         }
         __syncwarp();
@@ -311,8 +335,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t idesc128 = idesc_bf16_f32(kBM, kBN);
-    constexpr uint32_t idesc64 = idesc_bf16_f32(64, kBN);
+    constexpr uint32_t idesc128 = idesc_bf16_f32(kBM, BN);
+    constexpr uint32_t idesc64 = idesc_bf16_f32(64, BN);
     int s = 0;
     uint32_t ph = 0;
     int acc = 0;
@@ -328,7 +352,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after_sync();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
       for (int kb = kb_begin; kb < kb_end; ++kb) {
         ok = mbar_wait(smem_u32(&full_bar[s]), ph, s_abort);
         ok = __all_sync(0xffffffffu, ok);
@@ -384,20 +408,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after_sync();
-      const uint32_t tbase = lane_base + static_cast<uint32_t>(acc * kBN);
+      const uint32_t tbase = lane_base + static_cast<uint32_t>(acc * BN);
       const bool m64 = tc.rows <= 64;
       const int r = m64 ? quarter * 16 + lane : quarter * 32 + lane;   // tile row of this thread
       const bool row_ok = (!m64 || lane < 16) && r < tc.rows;
       const long long grow = static_cast<long long>(tc.row0) + r;
       if (MODE == kEpiSwiGLU) {
-        const int col0 = tc.n_blk * 128;
+        const int col0 = tc.n_blk * (BN / 2);
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(out_base);
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
+        for (int c = 0; c < BN / 2; c += 32) {
           if (col0 + c >= n_valid) break;              // warp-uniform
           uint32_t g[32], u[32];
           tmem_ld_32cols(tbase + c, g);
-          tmem_ld_32cols(tbase + 128 + c, u);
+          tmem_ld_32cols(tbase + BN / 2 + c, u);
           tmem_ld_wait();
           if (row_ok) {
 #pragma unroll

@@ -18,6 +18,7 @@
 #include "moe_ffn.h"
 #include "gemm_sm100.cuh"
 #include "route.cuh"
+#include "router_sm100.cuh"
 
 namespace {
 
@@ -41,15 +42,21 @@ constexpr int kMaxKernels = 16;
 constexpr int kTimingRing = 4;   // event sets: forward i records into set i % kTimingRing
 
 struct Layout {
-  size_t status, scores, idx, gate, chunk_counts, counts, offsets, mtiles, mtiles2, perm_src,
-      inv_pos;
+  size_t status, ticket, scores, idx, gate, chunk_counts, sub_base, counts, offsets, mtiles,
+      mtiles2, perm_src, inv_pos;
   size_t xperm, hidden, yrouted, hshared, yshared, total;
   int lds;            // row stride of the fp32 router scores
-  int tpc;            // tokens per routing chunk
+  int tpc;            // tokens per routing chunk (a block of route_scatter)
   int n_chunks;
+  int n_base;         // columns of chunk_counts: n_chunks, or the fused router's tiles
   int router_splits;  // split-K factor of the router GEMM (partials summed by route_topk)
   int router_kb_per;  // k-blocks per split
+  bool fused;         // router scores + softmax + top-k in one kernel (route_fused)
+  moe::RouterParams rt;   // its launch shape (sizes only; pointers set per forward)
+  size_t rt_smem;         // its dynamic shared memory
 };
+
+constexpr size_t kRouterMinSmem = 116 * 1024;   // one fused-router CTA per SM (see below)
 
 }  // namespace
 
@@ -69,6 +76,18 @@ struct moe_plan {
   // by default: measured on B200 it ran the merged launches at a lower clock
   // under the power cap and lost 5% on the DeepSeek-V3 layer shape.
   int merge_shared = 0;
+  // output columns of a single-CTA routed SwiGLU tile: 0 automatic (64 when
+  // the expected rows per expert are below 32, the weight-streaming regime,
+  // else 128), 64 or 128
+  int swiglu_tile_cols = 0;
+  // shared expert beside weight-streaming routed GEMMs: -1 automatic, 0 never, 1 always.
+  // Measured on B200 (DeepSeek-V3-shaped prefill): beside the routed GEMMs on 16
+  // SMs the layer took 7.09 ms per step against 6.19 ms inline (the capped
+  // routed GEMMs slowed more than the shared GEMMs saved), so automatic means never.
+  int shared_concurrent = -1;
+  // router: -1 automatic (the fused router whenever N_r <= 512), 0 the split
+  // router (scores GEMM, then softmax + top-k), 1 fused whenever supported
+  int fused_router = -1;
   // seats per expert per forward (token dropping); 0: unlimited (dropless)
   int64_t capacity = 0;
   // capacity factor in thousandths: seats = ceil(factor * T * top_k / N_r) per
@@ -105,18 +124,88 @@ struct moe_plan {
 
 namespace {
 
+// Launch shape of the fused router for T tokens (see router_sm100.cuh): the
+// cluster size CS splits each 128-token tile's K range; CS is at least N_r/64
+// so that one CTA's scores (128/CS tokens x N_r fp32) fit in 32 KB, and grows
+// (up to 8, and up to the number of K blocks) until the grid covers about
+// three quarters of the SMs.
+moe::RouterParams router_shape(const moe_plan* p, int64_t T, size_t* smem) {
+  moe::RouterParams r{};
+  const int nr = p->n_routed;
+  const int mt = static_cast<int>((T + moe::kBM - 1) / moe::kBM);
+  const int num_kb = (p->d + moe::kBK - 1) / moe::kBK;
+  int cs = nr <= 64 ? 1 : (nr <= 128 ? 2 : (nr <= 256 ? 4 : 8));
+  while (cs < moe::kRtMaxCluster && static_cast<long long>(mt) * cs < (3LL * p->num_sms) / 4 &&
+         cs < num_kb)
+    cs *= 2;
+  auto up = [](int v, int m) { return (v + m - 1) / m * m; };
+  r.T = static_cast<int>(T);
+  r.d = p->d;
+  r.n_routed = nr;
+  r.top_k = p->top_k;
+  r.renorm = p->renorm;
+  r.bias_select_only = p->bias_select_only;
+  r.cs = cs;
+  r.num_kb = num_kb;
+  r.kb_per = (num_kb + cs - 1) / cs;
+  r.own_rows = moe::kBM / cs;
+  r.n_chunks = mt;                 // one chunk of the histogram per 128-token tile
+  r.n_acc = nr > 256 ? 2 : 1;
+  r.mma_n0 = up(nr < 256 ? nr : 256, 16);
+  r.mma_n1 = r.n_acc > 1 ? up(nr - 256, 16) : 0;
+  r.ncols0 = up(nr < 256 ? nr : 256, 32);
+  r.ncols1 = r.n_acc > 1 ? up(nr - 256, 32) : 0;
+  r.box_rows = r.mma_n0 < 128 ? r.mma_n0 : 128;
+  r.nbox0 = (r.mma_n0 + r.box_rows - 1) / r.box_rows;
+  r.nbox1 = r.n_acc > 1 ? (r.mma_n1 + r.box_rows - 1) / r.box_rows : 0;
+  const int box_bytes = r.box_rows * moe::kBK * 2;
+  r.b_acc1_off = moe::kATileBytes + r.nbox0 * box_bytes;
+  r.stage_bytes = moe::kATileBytes + (r.nbox0 + r.nbox1) * box_bytes;
+  int stages = (160 * 1024) / r.stage_bytes;
+  if (stages > r.kb_per + 1) stages = r.kb_per + 1;
+  stages = stages < 2 ? 2 : (stages > moe::kRtMaxStages ? moe::kRtMaxStages : stages);
+  r.stages = stages;
+  const int exch = moe::kBM * ((r.ncols0 > r.ncols1 ? r.ncols0 : r.ncols1) + 4) * 4;
+  const int ring = stages * r.stage_bytes;
+  r.ring_bytes = up(ring > exch ? ring : exch, 1024);
+  r.lds = up(nr, 32);
+  int cols = 32;
+  while (cols < r.ncols0) cols *= 2;
+  r.tmem_cols = r.n_acc > 1 ? 512 : cols;
+  // fold the chunk scan into the router's last cluster while there are few
+  // chunks (one thread per expert walks them)
+  r.fold_scan = r.n_chunks <= 64 ? 1 : 0;
+  // at least kRouterMinSmem so that two router CTAs never share an SM: each
+  // allocates tensor memory and waits at cluster barriers, and two clusters
+  // interleaved on two SMs could otherwise wait on each other's allocation
+  size_t bytes = moe::router_smem_bytes(r.ring_bytes, r.own_rows, r.lds, nr);
+  *smem = bytes < kRouterMinSmem ? kRouterMinSmem : bytes;
+  return r;
+}
+
 Layout make_layout(const moe_plan* p, int64_t T) {
   Layout L{};
   const int64_t A = T * p->top_k;
   const int nsf = p->n_shared * p->f;
-  // chunking of the routing kernels: about two chunks per SM, 8..128 tokens each
-  int64_t tpc = (T + 2 * p->num_sms - 1) / (2 * p->num_sms);
-  tpc = tpc < 8 ? 8 : (tpc > 128 ? 128 : tpc);
-  L.tpc = static_cast<int>(tpc);
-  L.n_chunks = static_cast<int>((T + tpc - 1) / tpc);
+  L.fused = p->fused_router != 0 && p->n_routed <= moe::kRtMaxExperts;
   L.lds = static_cast<int>(align_up(p->n_routed, 8));
-  // split-K of the router GEMM so that it occupies most SMs even for few tokens
-  {
+  if (L.fused) {
+    // the router's histogram has one column per 128-token tile, plus each CTA's
+    // offsets inside its tile: route_scatter's chunks are the CTAs' token ranges
+    L.rt = router_shape(p, T, &L.rt_smem);
+    L.tpc = L.rt.own_rows;
+    L.n_chunks = L.rt.n_chunks * L.rt.cs;
+    L.n_base = L.rt.n_chunks;
+    L.router_splits = 0;
+    L.router_kb_per = 0;
+  } else {
+    // chunking of the routing kernels: about two chunks per SM, 8..128 tokens each
+    int64_t tpc = (T + 2 * p->num_sms - 1) / (2 * p->num_sms);
+    tpc = tpc < 8 ? 8 : (tpc > 128 ? 128 : tpc);
+    L.tpc = static_cast<int>(tpc);
+    L.n_chunks = static_cast<int>((T + tpc - 1) / tpc);
+    L.n_base = L.n_chunks;
+    // split-K of the router GEMM so that it occupies most SMs even for few tokens
     const int64_t tiles = ((T + moe::kBM - 1) / moe::kBM) * ((p->n_routed + moe::kBN - 1) / moe::kBN);
     const int num_kb = (p->d + moe::kBK - 1) / moe::kBK;
     // at most 8 splits, and at most 128 partial scores held per lane in route_topk
@@ -130,11 +219,13 @@ Layout make_layout(const moe_plan* p, int64_t T) {
   }
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
-  L.status = take(256);
-  L.scores = take(size_t(L.router_splits) * T * L.lds * 4);
+  L.status = take(256);          // status word at +0, router ticket at +64
+  L.ticket = L.status + 64;
+  L.scores = take(L.fused ? 0 : size_t(L.router_splits) * T * L.lds * 4);
   L.idx = take(size_t(A) * 4);
   L.gate = take(size_t(A) * 4);
-  L.chunk_counts = take(size_t(p->n_routed) * (L.n_chunks > 0 ? L.n_chunks : 1) * 4);
+  L.chunk_counts = take(size_t(p->n_routed) * (L.n_base > 0 ? L.n_base : 1) * 4);
+  L.sub_base = take(L.fused ? size_t(p->n_routed) * (L.n_chunks > 0 ? L.n_chunks : 1) * 4 : 0);
   L.counts = take(size_t(p->n_routed) * 4);
   L.offsets = take(size_t(p->n_routed + 1) * 4);
   L.mtiles = take(size_t(p->n_routed + 1) * 4);
@@ -171,13 +262,14 @@ EncodeTiledFn encode_fn() {
 }
 
 // bf16 matrix (rows, cols) row-major, optionally stacked `batch` times; box of
-// 64 columns (128 B, one swizzle row) x 128 rows, 128-byte swizzle, zero fill.
-bool make_map(CUtensorMap* m, const void* base, uint64_t batch, uint64_t rows, uint64_t cols) {
+// 64 columns (128 B, one swizzle row) x box_rows rows, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* m, const void* base, uint64_t batch, uint64_t rows, uint64_t cols,
+              uint32_t box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {cols, rows, batch};
   cuuint64_t strides[2] = {cols * 2, rows * cols * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   const cuuint32_t rank = batch > 0 ? 3 : 2;
   if (batch == 0) dims[2] = 1;
@@ -192,6 +284,7 @@ struct Launcher {
   moe_plan* p;
   cudaStream_t st;     // the caller's stream
   int status = MOE_OK;
+  int grid_cap = INT_MAX;   // most CTAs a GEMM launch may use (SMs left to a concurrent one)
 
   void begin(const char* name, cudaStream_t s, const char* variant = "") {
     if (p->n_launch < kMaxKernels) {
@@ -246,7 +339,7 @@ bool launch_gemm_pair(Launcher& L, cudaStream_t s, const char* name, const CUten
                       int max_tiles) {
   const int num_groups = prm.group_offsets ? prm.num_groups : 1;
   const size_t smem = moe::gemm_pair_smem_bytes<NW>(num_groups);
-  int pairs = L.p->num_sms / 2;
+  int pairs = (L.p->num_sms < L.grid_cap ? L.p->num_sms : L.grid_cap) / 2;
   if (max_tiles < pairs) pairs = max_tiles;
   if (pairs < 1) pairs = 1;
   cudaLaunchConfig_t cfg = {};
@@ -291,22 +384,24 @@ bool launch_pair_auto(Launcher& L, cudaStream_t s, const char* name, const CUten
   return launch_gemm_pair<MODE, 1>(L, s, name, a, b0, b1, prm, max_mtiles * prm.n_tiles);
 }
 
-// Single-CTA GEMM. x (optional) holds the A, B0, B1 maps of the extra dense
-// problem that prm.x_tiles describes; max_tiles bounds the grouped tiles only.
-template <int MODE>
+// Single-CTA GEMM with BN accumulator columns per tile. x (optional) holds the
+// A, B0, B1 maps of the extra dense problem that prm.x_tiles describes;
+// max_tiles bounds the grouped tiles only.
+template <int MODE, int BN = 256>
 bool launch_gemm(Launcher& L, cudaStream_t s, const char* name, const CUtensorMap& a,
                  const CUtensorMap& b0, const CUtensorMap& b1, const moe::GemmParams& prm,
                  int max_tiles, const CUtensorMap* x = nullptr) {
   const int num_groups = prm.group_offsets ? prm.num_groups : 1;
-  const size_t smem = moe::gemm_smem_bytes(num_groups);
+  const size_t smem = moe::gemm_smem_bytes<BN>(num_groups);
   const long long tiles = static_cast<long long>(max_tiles) + (x ? prm.x_tiles : 0);
-  int grid = tiles < L.p->num_sms ? static_cast<int>(tiles) : L.p->num_sms;
+  const int sms = L.p->num_sms < L.grid_cap ? L.p->num_sms : L.grid_cap;
+  int grid = tiles < sms ? static_cast<int>(tiles) : sms;
   if (grid < 1) grid = 1;
   moe::GemmParams q = prm;
   if (!x) q.x_tiles = 0;
-  L.begin(name, s, q.x_tiles > 0 ? "[+shared]" : "");
-  launch_pdl(moe::moe_gemm_kernel<MODE>, dim3(grid), dim3(moe::kGemmThreads), smem, s, a, b0,
-             b1, x ? x[0] : a, x ? x[1] : b0, x ? x[2] : b1, q);
+  L.begin(name, s, q.x_tiles > 0 ? "[+shared]" : (BN == 128 ? "[n64]" : ""));
+  launch_pdl(moe::moe_gemm_kernel<MODE, BN>, dim3(grid), dim3(moe::kGemmThreads), smem, s, a,
+             b0, b1, x ? x[0] : a, x ? x[1] : b0, x ? x[2] : b1, q);
   return L.end(name, s);
 }
 
@@ -327,6 +422,11 @@ int set_kernel_attributes() {
     if (e != cudaSuccess)
       return fail(MOE_CUDA_ERROR, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
   const size_t smem = moe::gemm_smem_bytes(moe::kMaxRouted);
+  const cudaError_t e0 = cudaFuncSetAttribute(
+      moe::moe_gemm_kernel<moe::kEpiSwiGLU, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      int(moe::gemm_smem_bytes<128>(moe::kMaxRouted)));
+  if (e0 != cudaSuccess)
+    return fail(MOE_CUDA_ERROR, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e0));
   cudaError_t e1 = cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiSwiGLU>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   cudaError_t e2 = cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiBF16>,
@@ -336,7 +436,42 @@ int set_kernel_attributes() {
   if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess)
     return fail(MOE_CUDA_ERROR, "cudaFuncSetAttribute failed: %s",
                 cudaGetErrorString(e1 != cudaSuccess ? e1 : (e2 != cudaSuccess ? e2 : e3)));
+  const int rsm = 227 * 1024;
+  const cudaError_t er[5] = {cudaFuncSetAttribute(moe::route_fused_kernel<1>, attr, rsm),
+                             cudaFuncSetAttribute(moe::route_fused_kernel<2>, attr, rsm),
+                             cudaFuncSetAttribute(moe::route_fused_kernel<4>, attr, rsm),
+                             cudaFuncSetAttribute(moe::route_fused_kernel<8>, attr, rsm),
+                             cudaFuncSetAttribute(moe::route_fused_kernel<16>, attr, rsm)};
+  for (cudaError_t e : er)
+    if (e != cudaSuccess)
+      return fail(MOE_CUDA_ERROR, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
   return MOE_OK;
+}
+
+// Fused router launch: clusters of rt.cs CTAs, one cluster per 128-token tile.
+cudaError_t launch_router(const Layout& Lw, const moe::RouterParams& rt, const CUtensorMap& mX,
+                          const CUtensorMap& mWg, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  const int mt = (rt.T + moe::kBM - 1) / moe::kBM;
+  cfg.gridDim = dim3(static_cast<unsigned>(mt * rt.cs));
+  cfg.blockDim = dim3(moe::kRtThreads);
+  cfg.dynamicSmemBytes = Lw.rt_smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(rt.cs);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const int npl = (rt.n_routed + 31) / 32;
+  if (npl <= 1) return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<1>, mX, mWg, rt);
+  if (npl <= 2) return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<2>, mX, mWg, rt);
+  if (npl <= 4) return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<4>, mX, mWg, rt);
+  if (npl <= 8) return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<8>, mX, mWg, rt);
+  return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<16>, mX, mWg, rt);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -480,6 +615,20 @@ int moe_plan_set_option(moe_plan_t p, int option, int64_t value) {
       p->capacity = value;
       p->capacity_permille = 0;
       return MOE_OK;
+    case MOE_OPTION_SHARED_CONCURRENT:
+      if (value < -1 || value > 1)
+        return fail(MOE_INVALID_ARG, "shared_concurrent must be -1, 0 or 1");
+      p->shared_concurrent = static_cast<int>(value);
+      return MOE_OK;
+    case MOE_OPTION_SWIGLU_TILE_COLS:
+      if (value != 0 && value != 64 && value != 128)
+        return fail(MOE_INVALID_ARG, "swiglu tile columns must be 0, 64 or 128");
+      p->swiglu_tile_cols = static_cast<int>(value);
+      return MOE_OK;
+    case MOE_OPTION_FUSED_ROUTER:
+      if (value < -1 || value > 1) return fail(MOE_INVALID_ARG, "fused_router must be -1, 0 or 1");
+      p->fused_router = static_cast<int>(value);
+      return MOE_OK;
     case MOE_OPTION_CAPACITY_FACTOR_PERMILLE:
       if (value < 0 || value > (1LL << 20))
         return fail(MOE_INVALID_ARG, "capacity factor (permille) must be in [0, 2^20]");
@@ -564,6 +713,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   int* idx = reinterpret_cast<int*>(ws + Lw.idx);
   float* gate = reinterpret_cast<float*>(ws + Lw.gate);
   int* chunk_counts = reinterpret_cast<int*>(ws + Lw.chunk_counts);
+  int* sub_base = Lw.fused ? reinterpret_cast<int*>(ws + Lw.sub_base) : nullptr;
   int* counts = reinterpret_cast<int*>(ws + Lw.counts);
   int* offsets = reinterpret_cast<int*>(ws + Lw.offsets);
   int* mtiles = reinterpret_cast<int*>(ws + Lw.mtiles);
@@ -599,8 +749,29 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   // a larger one would take SMs from the routing chain, so it runs inline on
   // the main stream after the routed GEMMs instead.
   const int shared_mt = static_cast<int>((T + 127) / 128);
-  const bool shared_forked =
+  // seats per expert and the expected rows per expert group (a division: the
+  // thresholds may be huge, and a product with N_r could overflow)
+  const int64_t seats = capacity_seats(p, T);
+  const int seat_limit = seats > 0 && seats < INT_MAX ? static_cast<int>(seats) : INT_MAX;
+  const long long rows_per_expert = A / nr < seat_limit ? A / nr : seat_limit;
+  const bool shared_small =
       p->n_shared > 0 && shared_mt * ((nsf + 127) / 128) <= p->num_sms / 2;
+  // A larger shared expert runs beside the routed GEMMs when those stream
+  // weights (few rows per expert: their tensor pipes idle most of the time):
+  // forked at the start onto shared_sms SMs, sized so that its tensor-bound
+  // work takes about as long as the routed weight stream on the other SMs
+  // (at about 253 FLOP per HBM byte, the measured B200 ridge); the routed
+  // GEMMs are capped to the remaining SMs.
+  int shared_sms = 0;
+  if (p->n_shared > 0 && !shared_small &&
+      p->shared_concurrent == 1) {
+    const double t_sh = 6.0 * double(T) * d * nsf / 253.0;
+    const double t_r = 6.0 * double(d) * f * (A < nr ? A : nr);
+    int sm = static_cast<int>(1.5 * p->num_sms * t_sh / (t_sh + t_r)) + 1;
+    sm = sm < 8 ? 8 : (sm > p->num_sms / 4 ? p->num_sms / 4 : sm);
+    shared_sms = sm;
+  }
+  const bool shared_forked = shared_small || shared_sms > 0;
   cudaStream_t shared_st = shared_forked ? p->side : main_st;
   const bool shared_pair = static_cast<long long>(T) >= p->pair_min_rows_swiglu;
   const int shared_mt2 = static_cast<int>((T + 255) / 256);
@@ -648,10 +819,32 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     if (cudaEventRecord(p->fork, main_st) != cudaSuccess ||
         cudaStreamWaitEvent(p->side, p->fork, 0) != cudaSuccess)
       return fail(MOE_CUDA_ERROR, "fork of the shared-expert stream failed");
+    if (shared_sms > 0) L.grid_cap = shared_sms;
     if (launch_shared() != MOE_OK) return L.status;
+    L.grid_cap = INT_MAX;
     if (cudaEventRecord(p->join, p->side) != cudaSuccess)
       return fail(MOE_CUDA_ERROR, "join record of the shared-expert stream failed");
   }
+  if (Lw.fused) {
+    // 1-3. fused router: scores on the tensor core, softmax, top-k, gates, the
+    //      chunk histogram and (when small) its scan, in one launch
+    CUtensorMap mWgR;
+    // rank-2 map (the kernel issues 2-D loads), boxes of rt.box_rows expert rows
+    if (!make_map(&mWgR, W_g, 0, nr, d, static_cast<uint32_t>(Lw.rt.box_rows)))
+      return fail(MOE_CUDA_ERROR, "cuTensorMapEncodeTiled rejected the router map");
+    moe::RouterParams rt = Lw.rt;
+    rt.bias = p->bias;
+    rt.idx = idx;
+    rt.gate = gate;
+    rt.tile_counts = chunk_counts;
+    rt.sub_base = sub_base;
+    rt.counts = counts;
+    rt.ticket = reinterpret_cast<int*>(ws + Lw.ticket);
+    rt.status = status;
+    L.begin("route_fused", main_st);
+    launch_router(Lw, rt, mX, mWgR, main_st);
+    if (!L.end("route_fused", main_st)) return L.status;
+  } else {
   // 1. router scores s = x W_g^T (fp32 partial sums of a split-K), dense over T rows
   {
     moe::GemmParams g{};
@@ -697,18 +890,18 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
 #undef MOE_TOPK
     if (!L.end("route_topk", main_st)) return L.status;
   }
-  // 3. per-expert prefix over chunks and expert totals (one warp per expert)
-  {
+  }
+  // 3. per-expert prefix over chunks and expert totals (one warp per expert),
+  //    unless the fused router's last CTA did it
+  if (!(Lw.fused && Lw.rt.fold_scan)) {
     const int warps = moe::kRouteThreads / 32;
     L.begin("route_scan", main_st);
     launch_pdl(moe::route_scan_kernel, dim3((nr + warps - 1) / warps), dim3(moe::kRouteThreads),
-               0, main_st, chunk_counts, Lw.n_chunks, nr, counts);
+               0, main_st, chunk_counts, Lw.n_base, nr, counts);
     if (!L.end("route_scan", main_st)) return L.status;
   }
   // 4. offsets + m-tile prefix, stable permutation, 16-byte row copies (with a
   //    seat limit, only each expert's first `capacity` pairs get rows)
-  const int64_t seats = capacity_seats(p, T);
-  const int seat_limit = seats > 0 && seats < INT_MAX ? static_cast<int>(seats) : INT_MAX;
   {
     const size_t smem = size_t(moe::kMaxRouted + nr) * 4 + size_t(2) * Lw.tpc * k * 4;
     // split the row copy into column slices of at least 32 vectors so that
@@ -720,17 +913,15 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     if (slices < 1) slices = 1;
     L.begin("route_scatter", main_st);
     launch_pdl(moe::route_scatter_kernel, dim3(Lw.n_chunks, slices), dim3(moe::kRouteThreads), smem,
-               main_st, (const int*)idx, (const int*)chunk_counts, (const int*)counts,
+               main_st, (const int*)idx, (const int*)chunk_counts, (const int*)sub_base,
+               Lw.n_chunks / Lw.n_base, (const int*)counts,
                static_cast<int>(T), k, nr, Lw.tpc, Lw.n_chunks, moe::kBM, seat_limit,
                reinterpret_cast<const uint4*>(x), d / 8, reinterpret_cast<uint4*>(xperm),
-               perm_src, inv_pos, offsets, mtiles, mtiles2);
+               perm_src, inv_pos, offsets, mtiles, mtiles2, status);
     if (!L.end("route_scatter", main_st)) return L.status;
   }
   const int max_mtiles = static_cast<int>((A + 127) / 128 + (A < nr ? A : nr));
   const int max_mtiles2 = static_cast<int>((A + 255) / 256 + (A < nr ? A : nr));
-  // expected rows per expert against the thresholds (a division: the
-  // thresholds may be huge, and a product with N_r could overflow)
-  const long long rows_per_expert = A / nr < seat_limit ? A / nr : seat_limit;
   const bool routed_pair_swiglu = rows_per_expert >= p->pair_min_rows_swiglu;
   const bool routed_pair = rows_per_expert >= p->pair_min_rows_plain;
   const int expected_mtiles2 = static_cast<int>((A + 255) / 256);
@@ -743,7 +934,14 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   const bool merge_dn = merge_gu && !routed_pair;
   const CUtensorMap xgu[3] = {mX, mW1s, mW3s};
   const CUtensorMap xdn[3] = {mHs, mW2s, mW2s};
-  // 5. grouped gate/up GEMM with the SiLU(gate) * up epilogue
+  // the routed GEMMs leave the concurrent shared expert its SMs
+  if (shared_sms > 0) L.grid_cap = p->num_sms - shared_sms;
+  // 5. grouped gate/up GEMM with the SiLU(gate) * up epilogue. With few rows
+  //    per expert (weight streaming) the single-CTA kernel uses 64-column
+  //    tiles: twice as many, shorter tiles, so the last wave is shorter.
+  const bool narrow_gu =
+      !routed_pair_swiglu && !merge_gu &&
+      (p->swiglu_tile_cols == 64 || (p->swiglu_tile_cols == 0 && rows_per_expert < 32));
   {
     moe::GemmParams g{};
     g.group_offsets = offsets;
@@ -751,7 +949,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.num_groups = nr;
     g.K = d;
     g.N = f;
-    g.n_tiles = (f + 127) / 128;
+    g.n_tiles = narrow_gu ? (f + 63) / 64 : (f + 127) / 128;
     g.out = hidden;
     g.ldo = f;
     g.status = status;
@@ -769,12 +967,21 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
       g.x_out = hshared;
       g.x_ldo = nsf;
     }
-    if (routed_pair_swiglu ? !launch_pair_auto<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1,
-                                                         mW3, g, f, expected_mtiles2, max_mtiles2)
-                    : !launch_gemm<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1, mW3,
-                                                    g, max_mtiles * g.n_tiles,
-                                                    merge_gu ? xgu : nullptr))
+    if (narrow_gu) {
+      CUtensorMap mW1n, mW3n;
+      if (!make_map(&mW1n, W1, nr, f, d, 64) || !make_map(&mW3n, W3, nr, f, d, 64))
+        return fail(MOE_CUDA_ERROR, "cuTensorMapEncodeTiled rejected a tensor map");
+      if (!launch_gemm<moe::kEpiSwiGLU, 128>(L, main_st, "grouped_gate_up", mXp, mW1n, mW3n, g,
+                                             max_mtiles * g.n_tiles))
+        return L.status;
+    } else if (routed_pair_swiglu
+                   ? !launch_pair_auto<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1,
+                                                        mW3, g, f, expected_mtiles2, max_mtiles2)
+                   : !launch_gemm<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1, mW3,
+                                                   g, max_mtiles * g.n_tiles,
+                                                   merge_gu ? xgu : nullptr)) {
       return L.status;
+    }
   }
   // 6. grouped down GEMM
   {
@@ -806,6 +1013,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
                                                   merge_dn ? xdn : nullptr))
       return L.status;
   }
+  L.grid_cap = INT_MAX;
   // 7. the shared expert (inline, merged, or joined from the side stream), then
   //    the weighted combine + shared add with one bf16 rounding
   if (p->n_shared > 0 && !shared_forked) {
@@ -821,7 +1029,8 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     L.begin("combine", main_st);
     launch_pdl(moe::combine_kernel, grid, dim3(moe::kCombineThreads), 0, main_st,
                reinterpret_cast<const uint4*>(yrouted), (const float*)yshared,
-               (const int*)inv_pos, (const float*)gate, k, d_vec, reinterpret_cast<uint4*>(out));
+               (const int*)inv_pos, (const float*)gate, k, d_vec, reinterpret_cast<uint4*>(out),
+               Lw.fused ? reinterpret_cast<int*>(ws + Lw.ticket) : static_cast<int*>(nullptr));
     if (!L.end("combine", main_st)) return L.status;
   }
   L.finish();
@@ -885,7 +1094,7 @@ int moe_plan_device_status(moe_plan_t p) {
   }
   p->noalloc_used = false;
   if (worst != MOE_OK)
-    return fail(worst, "a kernel gave up a bounded wait (device status %d)", worst);
+    return fail(worst, "device status %d: %s", worst, moe_strerror(worst));
   return MOE_OK;
 }
 
@@ -952,6 +1161,14 @@ int moe_forward_noalloc(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_
   // keep describing the last moe_forward, whose routing is still in the
   // plan's workspace). The status word at the start of the scratch is not
   // cleared here: a bounded-wait timeout stays visible to moe_plan_device_status.
+  // The router's ticket must start at zero; every call clears it, so that two
+  // calls that overlapped (which race) cannot leave it disturbed for the next.
+  if (T > 0) {
+    const Layout Ln = make_layout(p, T);
+    cudaError_t e = cudaMemsetAsync(static_cast<char*>(p->noalloc_scratch) + Ln.ticket, 0,
+                                    sizeof(int), static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(MOE_CUDA_ERROR, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+  }
   char* saved_ws = p->ws;
   const size_t saved_bytes = p->ws_bytes;
   const bool saved_timing = p->timing;
@@ -993,6 +1210,7 @@ const char* moe_strerror(int s) {
     case MOE_CUDA_ERROR: return "CUDA error";
     case MOE_UNSUPPORTED: return "unsupported shape";
     case MOE_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+    case MOE_DEVICE_INCONSISTENT: return "a kernel found inconsistent routing state";
     default: return "unknown status";
   }
 }

@@ -31,6 +31,80 @@ constexpr int kRouteThreads = 256;             // 8 warps
 constexpr int kMaxTopK = 32;
 constexpr int kMaxRouted = 1024;
 
+// One token's routing, computed by one warp from its N_r router scores (lane
+// i holds the scores of experts lane + 32*j in v[j], the bias not yet added):
+// softmax over all N_r experts, the top_k experts by the biased score with
+// ties to the lower index, and the gates (raw probabilities, or renormalised
+// over the selected set). Lane j < top_k receives the j-th selected expert in
+// `my_e` and its gate in `my_g`.
+template <int NPL>
+__device__ __forceinline__ void route_token(float (&v)[NPL], const float* __restrict__ bias,
+                                            int n_routed, int top_k, int renorm,
+                                            int bias_select_only, int lane, int& my_e,
+                                            float& my_g) {
+  // The biased scores rank the experts; the gates are the softmax of the
+  // biased scores (logit bias) or of the unbiased ones (selection-only bias).
+  float m = -INFINITY;
+  float key[NPL];
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int e = lane + 32 * i;
+    const float b = (bias && e < n_routed) ? bias[e] : 0.0f;
+    key[i] = e < n_routed ? v[i] + b : -INFINITY;
+    v[i] = e < n_routed ? (bias_select_only ? v[i] : key[i]) : -INFINITY;
+    m = fmaxf(m, v[i]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float sum = 0.0f;
+#pragma unroll
+  for (int i = 0; i < NPL; ++i)
+    if (lane + 32 * i < n_routed) sum += expf(v[i] - m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+
+  // Selection keys: a NaN score (from NaN or infinite inputs) ranks as -inf,
+  // so the order stays total and every lane agrees on each winner. Each key is
+  // mapped to an unsigned integer with the same order (-0 and +0 equal), so a
+  // round of the selection is two warp reductions (redux.sync): the largest key,
+  // then the lowest expert index holding it - ties go to the lower index. An
+  // empty lane's 0 is below every real key (-inf maps to 0x007fffff).
+  uint32_t okey[NPL];
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    float kv = key[i] == key[i] ? key[i] : -INFINITY;
+    kv = kv == 0.0f ? 0.0f : kv;
+    const uint32_t b = __float_as_uint(kv);
+    okey[i] = lane + 32 * i < n_routed ? ((b & 0x80000000u) ? ~b : (b | 0x80000000u)) : 0u;
+  }
+  uint32_t taken = 0;
+  float sel_sum = 0.0f, my_p = 0.0f;
+  my_e = -1;
+  for (int j = 0; j < top_k; ++j) {
+    uint32_t lmax = 0u;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+      if (!((taken >> i) & 1u)) lmax = okey[i] > lmax ? okey[i] : lmax;
+    const uint32_t gmax = __reduce_max_sync(0xffffffffu, lmax);
+    int lidx = 0x7fffffff;
+#pragma unroll
+    for (int i = NPL - 1; i >= 0; --i)     // descending: the last match is the lowest index
+      if (!((taken >> i) & 1u) && okey[i] == gmax) lidx = lane + 32 * i;
+    const int be = static_cast<int>(__reduce_min_sync(0xffffffffu, static_cast<unsigned>(lidx)));
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    // the winner's gate score, from the lane that holds it
+    float gw = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+      if (i == (be >> 5)) gw = v[i];
+    gw = __shfl_sync(0xffffffffu, gw, be & 31);
+    const float p = expf(gw - m) / sum;
+    sel_sum += p;
+    if (lane == j) { my_p = p; my_e = be; }
+  }
+  my_g = renorm ? my_p / sel_sum : my_p;
+}
+
 // One warp per token; block = one chunk of `tpc` consecutive tokens.
 // NPL = router scores held per lane (N_r <= 32 * NPL). The scores arrive as
 // `splits` (<= MAXS) fp32 partial sums (split-K of the router GEMM),
@@ -72,67 +146,13 @@ __global__ void __launch_bounds__(kRouteThreads)
       for (int sp = 1; sp < MAXS; ++sp) a += part[sp][i];
       v[i] = a;
     }
-    // The biased scores rank the experts; the gates are the softmax of the
-    // biased scores (logit bias) or of the unbiased ones (selection-only bias).
-    float m = -INFINITY;
-    float key[NPL];
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      const int e = lane + 32 * i;
-      const float b = (bias && e < n_routed) ? bias[e] : 0.0f;
-      key[i] = e < n_routed ? v[i] + b : -INFINITY;
-      v[i] = e < n_routed ? (bias_select_only ? v[i] : key[i]) : -INFINITY;
-      m = fmaxf(m, v[i]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float sum = 0.0f;
-#pragma unroll
-    for (int i = 0; i < NPL; ++i)
-      if (lane + 32 * i < n_routed) sum += expf(v[i] - m);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-
-    // Selection keys: a NaN score (from NaN or infinite inputs) ranks as -inf,
-    // so the order stays total and every lane agrees on each winner; the
-    // sentinel index of an empty lane loses every tie against a real expert.
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) key[i] = key[i] == key[i] ? key[i] : -INFINITY;
-    uint32_t taken = 0;
-    float sel_sum = 0.0f, my_p = 0.0f;
-    int my_e = -1;
-    for (int j = 0; j < top_k; ++j) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < NPL; ++i) {
-        const int e = lane + 32 * i;     // ascending within the lane: '>' keeps the lower index
-        if (e < n_routed && !((taken >> i) & 1u) && (key[i] > bv || be == 0x7fffffff)) {
-          bv = key[i];
-          be = e;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-      }
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      // the winner's gate score, from the lane that holds it
-      float gw = 0.0f;
-#pragma unroll
-      for (int i = 0; i < NPL; ++i)
-        if (i == (be >> 5)) gw = v[i];
-      gw = __shfl_sync(0xffffffffu, gw, be & 31);
-      const float p = expf(gw - m) / sum;
-      sel_sum += p;
-      if (lane == j) { my_p = p; my_e = be; }
-    }
+    int my_e;
+    float my_g;
+    route_token<NPL>(v, bias, n_routed, top_k, renorm, bias_select_only, lane, my_e, my_g);
     if (lane < top_k) {
       const long long o = static_cast<long long>(t) * top_k + lane;
       idx[o] = my_e;
-      gate[o] = renorm ? my_p / sel_sum : my_p;
+      gate[o] = my_g;
       atomicAdd(&s_hist[my_e], 1);
     }
   }
@@ -150,11 +170,38 @@ __device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
   return v;
 }
 
-// One warp per expert (8 experts per block). chunk_counts [N_r][n_chunks]
-// becomes, in place, the exclusive prefix over chunks of each expert; the
-// warp's loads for up to 32*kScanPrefetch chunks are issued before any scan.
+// One warp scans one expert's row of chunk_counts [N_r][n_chunks]: the row
+// becomes, in place, the exclusive prefix over chunks; returns the expert's
+// total to every lane. The warp's loads for up to 32*kScanPrefetch chunks are
+// issued before any scan. kL2 reads through L2 only (rows another block of the
+// same grid wrote, made visible by a fence).
 constexpr int kScanPrefetch = 16;
 
+template <bool kL2>
+__device__ __forceinline__ int scan_expert_chunks(int* row, int n_chunks, int lane) {
+  int running = 0;
+  for (int c0 = 0; c0 < n_chunks; c0 += 32 * kScanPrefetch) {
+    int v[kScanPrefetch];
+#pragma unroll
+    for (int b = 0; b < kScanPrefetch; ++b) {
+      const int c = c0 + b * 32 + lane;
+      v[b] = c < n_chunks ? (kL2 ? __ldcg(row + c) : row[c]) : 0;
+    }
+    const int nb = min(kScanPrefetch, (n_chunks - c0 + 31) / 32);   // warp-uniform
+#pragma unroll
+    for (int b = 0; b < kScanPrefetch; ++b) {
+      if (b >= nb) break;
+      const int c = c0 + b * 32 + lane;
+      const int incl = warp_inclusive_scan(v[b], lane);
+      if (c < n_chunks) row[c] = running + incl - v[b];
+      running += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+  return running;
+}
+
+// One warp per expert (8 experts per block): exclusive prefix over chunks of
+// each expert's counts, in place, and the expert's total.
 __global__ void __launch_bounds__(kRouteThreads)
     route_scan_kernel(int* __restrict__ chunk_counts, int n_chunks, int n_routed,
                       int* __restrict__ counts) {
@@ -163,24 +210,9 @@ __global__ void __launch_bounds__(kRouteThreads)
   const int lane = threadIdx.x & 31;
   const int e = blockIdx.x * (kRouteThreads / 32) + (threadIdx.x >> 5);
   if (e >= n_routed) return;
-  int* row = chunk_counts + static_cast<long long>(e) * n_chunks;
-  int running = 0;
-  for (int c0 = 0; c0 < n_chunks; c0 += 32 * kScanPrefetch) {
-    int v[kScanPrefetch];
-#pragma unroll
-    for (int b = 0; b < kScanPrefetch; ++b) {
-      const int c = c0 + b * 32 + lane;
-      v[b] = c < n_chunks ? row[c] : 0;
-    }
-#pragma unroll
-    for (int b = 0; b < kScanPrefetch; ++b) {
-      const int c = c0 + b * 32 + lane;
-      const int incl = warp_inclusive_scan(v[b], lane);
-      if (c < n_chunks) row[c] = running + incl - v[b];
-      running += __shfl_sync(0xffffffffu, incl, 31);
-    }
-  }
-  if (lane == 0) counts[e] = running;
+  const int total =
+      scan_expert_chunks<false>(chunk_counts + static_cast<long long>(e) * n_chunks, n_chunks, lane);
+  if (lane == 0) counts[e] = total;
 }
 
 // Exclusive scan of n (<= kMaxRouted) ints in shared memory by a 256-thread
@@ -216,8 +248,24 @@ __device__ __forceinline__ int block_exclusive_scan(int* s, int n, int* tmp) {
   return total;
 }
 
-// Block = one chunk. The chunk's expert ids and their per-chunk bases are
-// staged in shared memory by all threads; warp 0 then ranks the (token, slot)
+// Sum of one int per thread over a 256-thread block; every thread gets it.
+// `tmp` holds 8 ints; the block must be converged.
+__device__ __forceinline__ int block_sum(int v, int* tmp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) tmp[warp] = v;
+  __syncthreads();
+  int total = 0;
+#pragma unroll
+  for (int w = 0; w < kRouteThreads / 32; ++w) total += tmp[w];
+  __syncthreads();
+  return total;
+}
+
+// Block = one chunk. The chunk's expert ids and their bases inside each
+// expert's group are staged in shared memory by all threads; warp 0 then ranks the (token, slot)
 // entries in order with match-any, so rows inside an expert group follow
 // ascending (t, j); every warp then copies token rows (d_vec 16-byte vectors
 // each) to their k rows, four vectors in flight per lane. With a seat limit
@@ -230,12 +278,14 @@ constexpr int kCopyUnroll = 4;
 
 __global__ void __launch_bounds__(kRouteThreads)
     route_scatter_kernel(const int* __restrict__ idx, const int* __restrict__ chunk_base,
+                         const int* __restrict__ sub_base, int chunks_per_base,
                          const int* __restrict__ counts, int T, int top_k, int n_routed,
                          int tpc, int n_chunks, int tile_rows, int capacity,
                          const uint4* __restrict__ x,
                          int d_vec, uint4* __restrict__ xperm, int* __restrict__ perm_src,
                          int* __restrict__ inv_pos, int* __restrict__ offsets_out,
-                         int* __restrict__ mtiles_out, int* __restrict__ mtiles2_out) {
+                         int* __restrict__ mtiles_out, int* __restrict__ mtiles2_out,
+                         int* __restrict__ status) {
   extern __shared__ int smem_i[];
   int* s_off = smem_i;                        // [kMaxRouted] expert offsets
   int* s_run = smem_i + kMaxRouted;           // [n_routed]
@@ -246,22 +296,46 @@ __global__ void __launch_bounds__(kRouteThreads)
   pdl_wait();
   const int chunk = blockIdx.x;
   const int t0 = chunk * tpc;
-  const int ntok = min(tpc, T - t0);
+  const int ntok = max(0, min(tpc, T - t0));   // the last tile's chunks may hold no token
   const int n_ent = ntok * top_k;
   const long long ebase = static_cast<long long>(t0) * top_k;
+  // the chunk's base inside each expert's group: one level (chunk_base
+  // [N_r][n_chunks]) or two (chunk_base [N_r][n_chunks / chunks_per_base] per
+  // group of chunks, plus sub_base [N_r][n_chunks] inside the group)
+  const int n_base = n_chunks / chunks_per_base;
   for (int i = threadIdx.x; i < n_ent; i += blockDim.x) {
     const int e = idx[ebase + i];
     s_e[i] = e;
-    s_pos[i] = chunk_base[static_cast<long long>(e) * n_chunks + chunk];
+    int b = chunk_base[static_cast<long long>(e) * n_base + chunk / chunks_per_base];
+    if (sub_base) b += sub_base[static_cast<long long>(e) * n_chunks + chunk];
+    s_pos[i] = b;
   }
   // an expert keeps at most `capacity` rows: its first pairs in (token, slot) order
   for (int e = threadIdx.x; e < n_routed; e += blockDim.x) {
     s_off[e] = min(counts[e], capacity);
     s_run[e] = 0;
   }
+  // consistency of the routing state: the expert totals must add up to the
+  // T*top_k pairs and be non-negative. They always do unless the workspace was
+  // overwritten during a forward; then every block of the grid sees the same
+  // totals and the forward degrades to writing nothing out of range: no rows,
+  // empty expert groups, every slot dropped, and the device status reports it.
+  __syncthreads();
+  const int pairs = T * top_k;
+  int csum = 0, crange = 0;
+  for (int e = threadIdx.x; e < n_routed; e += blockDim.x) {
+    const int c = counts[e];
+    csum += c;
+    crange |= c < 0 || c > pairs;
+  }
+  const int out_of_range = __syncthreads_or(crange);
+  const bool bad = out_of_range || block_sum(csum, s_tmp) != pairs;
+  if (bad)
+    for (int e = threadIdx.x; e < n_routed; e += blockDim.x) s_off[e] = 0;
   __syncthreads();
   const int total = block_exclusive_scan(s_off, n_routed, s_tmp);
   if (blockIdx.x == 0 && blockIdx.y == 0) {
+    if (bad && threadIdx.x == 0) atomicExch(status, 7 /* MOE_DEVICE_INCONSISTENT */);
     // publish offsets and the m-tile prefix for the grouped GEMMs
     for (int e = threadIdx.x; e < n_routed; e += blockDim.x) offsets_out[e] = s_off[e];
     if (threadIdx.x == 0) offsets_out[n_routed] = total;
@@ -271,7 +345,7 @@ __global__ void __launch_bounds__(kRouteThreads)
       int* dst = pass ? mtiles2_out : mtiles_out;
       __syncthreads();
       for (int e = threadIdx.x; e < n_routed; e += blockDim.x)
-        s_run[e] = (min(counts[e], capacity) + rows - 1) / rows;
+        s_run[e] = bad ? 0 : (min(counts[e], capacity) + rows - 1) / rows;
       __syncthreads();
       const int total_mt = block_exclusive_scan(s_run, n_routed, s_tmp);
       for (int e = threadIdx.x; e < n_routed; e += blockDim.x) {
@@ -293,7 +367,9 @@ __global__ void __launch_bounds__(kRouteThreads)
       const int rank = __popc(same & ((1u << lane) - 1u));
       if (valid) {
         const int r = s_pos[i] + s_run[e] + rank;   // place among the expert's pairs
-        s_pos[i] = r < capacity ? s_off[e] + r : -1;  // -1: dropped, no seat left
+        const bool ok = !bad && r >= 0 && r < counts[e];
+        if (!ok && !bad) atomicExch(status, 7 /* MOE_DEVICE_INCONSISTENT */);
+        s_pos[i] = ok && r < capacity ? s_off[e] + r : -1;  // -1: dropped, no seat left
       }
       __syncwarp();
       if (valid && lane == 31 - __clz(same)) s_run[e] += __popc(same);
@@ -360,11 +436,14 @@ constexpr int kCombineCols = kCombineThreads * kCombineVec;
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const uint4* __restrict__ Y, const float* __restrict__ shared,
                    const int* __restrict__ inv_pos, const float* __restrict__ gate, int top_k,
-                   int d_vec, uint4* __restrict__ out) {
+                   int d_vec, uint4* __restrict__ out, int* __restrict__ router_ticket) {
   __shared__ int s_pos[kMaxTopK];
   __shared__ float s_w[kMaxTopK];
   pdl_launch_dependents();
   pdl_wait();
+  // the fused router leaves its ticket at zero; resetting it here as well means
+  // a ticket found corrupted in one forward cannot disturb the next
+  if (router_ticket && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *router_ticket = 0;
   const long long t = blockIdx.x;
   if (threadIdx.x < top_k) {
     s_pos[threadIdx.x] = inv_pos[t * top_k + threadIdx.x];

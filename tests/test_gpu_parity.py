@@ -43,6 +43,77 @@ def test_small_layers_all_outputs(case):
     assert res["near_ties"] <= max(2, T * k // 20)
 
 
+ROUTER_CASES = [
+    # name, T, d, f, N_r, k, N_s, renorm, bias: shapes that reach the fused router's
+    # edges (clusters of 1..8 CTAs, one or two accumulators, CTAs without K blocks,
+    # ragged token tiles and K tails, the chunk scan folded or separate)
+    ("fr_one_token_512", 1, 256, 64, 512, 10, 1, True, "zipf1.1"),      # 4 K blocks, 8 CTAs
+    ("fr_second_acc_one_expert", 129, 128, 64, 257, 9, 0, False, "none"),
+    ("fr_eight_experts", 300, 512, 64, 8, 2, 0, True, "none"),          # 16-row W_g boxes
+    ("fr_k_tail", 200, 200, 64, 100, 5, 1, True, "normal_var0.5"),     # d = 3*64 + 8
+    ("fr_two_acc_ragged", 1000, 1024, 64, 384, 6, 1, True, "zipf1.1"),
+    ("fr_scan_not_folded", 16384, 256, 64, 256, 8, 0, True, "normal_var0.5"),
+]
+
+
+@pytest.mark.parametrize("case", ROUTER_CASES, ids=[c[0] for c in ROUTER_CASES])
+def test_fused_router_edges(case):
+    name, T, d, f, n, k, ns, renorm, bias = case
+    shape = LayerShape(name, T, d, f, n, k, ns, renorm, bias)
+    inp = make_layer_inputs(shape, seed=21, device="cuda")
+    tokens = None
+    if T > 2048:
+        tokens = np.sort(np.random.default_rng(3).choice(T, size=512, replace=False))
+    res = full_parity(inp, shape, tokens=tokens)
+    names = res["layer"].plan.kernel_names()
+    assert "route_fused" in names and "router_gemm" not in names, names
+    assert ("route_scan" in names) == (name == "fr_scan_not_folded"), names
+
+
+SPLIT_ROUTER_CASES = ["one_token", "ragged_17", "k_equals_n", "wide_router", "skewed_groups"]
+
+
+@pytest.mark.parametrize("case", [c for c in SMALL if c[0] in SPLIT_ROUTER_CASES],
+                         ids=[c[0] for c in SMALL if c[0] in SPLIT_ROUTER_CASES])
+def test_split_router_kernels(case):
+    # the two-kernel router (split-K scores GEMM, then softmax + top-k), which
+    # layers with more than 512 experts use, forced on shapes the fused one covers
+    name, T, d, f, n, k, ns, renorm, bias = case
+    shape = LayerShape(name, T, d, f, n, k, ns, renorm, bias)
+    inp = make_layer_inputs(shape, seed=1, device="cuda")
+    res = full_parity(inp, shape, fused_router=0)
+    names = res["layer"].plan.kernel_names()
+    assert "router_gemm" in names and "route_fused" not in names, names
+
+
+NARROW_CASES = [
+    # name, T, d, f, N_r, k, N_s, renorm, bias: the 64-column SwiGLU tiles (N=128
+    # accumulators, four in TMEM) against the 128-column ones
+    LayerShape("narrow_decode_like", 128, 2048, 512, 512, 10, 1, True, "zipf1.1"),
+    LayerShape("narrow_ragged", 600, 384, 328, 6, 2, 1, True, "none"),      # f tail of 8
+    LayerShape("narrow_k_tail", 77, 136, 72, 9, 3, 0, True, "none"),
+]
+
+
+@pytest.mark.parametrize("shape", NARROW_CASES, ids=[c.name for c in NARROW_CASES])
+def test_narrow_swiglu_tiles(shape):
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    inp = make_layer_inputs(shape, seed=8, device="cuda")
+    res = full_parity(inp, shape)        # default tile choice, against the oracle
+    outs = {}
+    for cols in (64, 128):
+        layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
+                         shape.renorm, inp, bias=inp["bias"], device="cuda",
+                         swiglu_tile_cols=cols)
+        outs[cols] = layer(inp["x"]).clone()
+        names = layer.plan.kernel_names()
+        assert ("grouped_gate_up[n64]" in names) == (cols == 64), names
+    torch.cuda.synchronize()
+    # every output element is the same sum in the same k order on both tile shapes
+    assert torch.equal(outs[64], outs[128])
+    del res
+
+
 PAIR_CASES = ["three_tokens", "ragged_17", "two_shared_raw", "ragged_tiles", "k_tail_not_64",
               "skewed_groups"]
 
@@ -113,6 +184,31 @@ def test_merged_and_separate_shared_expert_agree_bitwise(case):
         outs.append(layer(inp["x"]).clone())
         torch.cuda.synchronize()
         assert layer.device_status() == 0
+    assert torch.equal(outs[0], outs[1])
+
+
+CONCURRENT_CASES = [
+    # a shared expert too large for the routing phase, beside weight-streaming
+    # routed GEMMs (fewer than 192 rows per expert): forked onto a few SMs
+    LayerShape("concurrent_prefill_like", 2048, 512, 256, 64, 4, 1, True, "normal_var0.5"),
+    LayerShape("concurrent_two_shared", 1500, 384, 192, 48, 6, 2, False, "none"),
+]
+
+
+@pytest.mark.parametrize("shape", CONCURRENT_CASES, ids=[c.name for c in CONCURRENT_CASES])
+def test_shared_expert_beside_the_routed_gemms(shape):
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    inp = make_layer_inputs(shape, seed=9, device="cuda")
+    full_parity(inp, shape)                     # default policy, against the oracle
+    outs = []
+    for conc in (0, 1):
+        layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
+                         shape.renorm, inp, bias=inp["bias"], device="cuda",
+                         shared_concurrent=conc)
+        outs.append(layer(inp["x"]).clone())
+        torch.cuda.synchronize()
+        assert layer.device_status() == 0
+    # the same kernels on other SMs and streams: the same bits
     assert torch.equal(outs[0], outs[1])
 
 
