@@ -128,12 +128,22 @@ int moe_last_status(void);
  *   expected rows per expert (T*top_k/N_r) are below 32 - the weight-streaming
  *   decode regime, where twice as many, shorter tiles leave a shorter last
  *   wave - and 128 otherwise; 64 or 128 force it.
+ * MOE_OPTION_TILE_ROWS: rows of one tile of the routed GEMMs when they run
+ *   one CTA per tile: 0 (default) chooses 64 when the expected rows per expert
+ *   are below 32 (M=64 MMAs and 64-row boxes of the grouped rows: smaller
+ *   pipeline stages, so more of them and more weight bytes in flight per SM),
+ *   and 128 otherwise; 64 or 128 force it.
+ * MOE_OPTION_INTERLEAVE: order of the tiles of the routed GEMMs when they run
+ *   one CTA per 128-row tile. 1: the tiles of experts with at least two
+ *   m-blocks (tensor-heavy, their weight tiles reused through L2) are spread
+ *   evenly among the other experts' tiles (weight streaming), so that tensor
+ *   and HBM work overlap; 0: expert order; -1 (default): 1 when the expected
+ *   rows per expert are below 192.
  * MOE_OPTION_SHARED_CONCURRENT: where a shared expert too large for the
- *   routing phase runs. -1 (default): beside the routed GEMMs, on a second
- *   stream and a few SMs (the routed GEMMs keep the rest), when those stream
- *   weights (fewer than 192 expected rows per expert); else after them on the
- *   caller's stream. 1: always beside them; 0: never. Small shared experts
- *   always run beside the routing kernels.
+ *   routing phase runs. 1: beside the routed GEMMs, on a second stream and a
+ *   few SMs (the routed GEMMs keep the rest); -1 (default) and 0: after them on
+ *   the caller's stream (measured faster on B200 for the DeepSeek-V3 layer
+ *   shape). Small shared experts always run beside the routing kernels.
  * MOE_OPTION_TEST_WAIT_TIMEOUT: test hook for the failure path, not for normal
  *   use. Value 1 arms it for the next forward only: if that forward runs the
  *   routed gate/up GEMM on the one-CTA-per-tile kernel, one CTA withholds the
@@ -151,6 +161,8 @@ enum {
   MOE_OPTION_FUSED_ROUTER = 7,
   MOE_OPTION_SWIGLU_TILE_COLS = 8,
   MOE_OPTION_SHARED_CONCURRENT = 9,
+  MOE_OPTION_TILE_ROWS = 10,
+  MOE_OPTION_INTERLEAVE = 11,
   MOE_OPTION_TEST_WAIT_TIMEOUT = 100
 };
 int moe_plan_set_option(moe_plan_t plan, int option, int64_t value);

@@ -31,6 +31,8 @@ MOE_OPTION_CAPACITY_FACTOR_PERMILLE = 6
 MOE_OPTION_FUSED_ROUTER = 7
 MOE_OPTION_SWIGLU_TILE_COLS = 8
 MOE_OPTION_SHARED_CONCURRENT = 9
+MOE_OPTION_TILE_ROWS = 10
+MOE_OPTION_INTERLEAVE = 11
 MOE_OPTION_TEST_WAIT_TIMEOUT = 100
 
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_INVALID_CONFIG", 2: "MOE_INVALID_ARG",

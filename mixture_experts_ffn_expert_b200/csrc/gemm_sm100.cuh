@@ -64,7 +64,12 @@ __host__ __device__ constexpr int tile_cols(int mode) { return mode == kEpiSwiGL
 
 struct GemmParams {
   const int* group_offsets;  // device (num_groups+1); nullptr: one dense group of dense_rows
-  const int* group_mtiles;   // device (num_groups+1) exclusive prefix of ceil(n_g / 128)
+  const int* group_mtiles;   // device (num_groups+1) exclusive prefix of ceil(n_g / tile rows)
+  // Optional second class of groups (nullptr: one class). With it, group_mtiles
+  // counts only the groups of class A (the others contribute 0) and
+  // group_mtiles_b only those of class B; the tiles of class A are spread
+  // evenly over the launch, those of class B fill the positions between them.
+  const int* group_mtiles_b;
   int num_groups;
   int dense_rows;
   int K;                     // reduction length (elements)
@@ -90,25 +95,31 @@ struct GemmParams {
   int test_withhold;
 };
 
-// Single-CTA kernel shapes: BN accumulator columns per tile (MMA N). BN = 256
-// is the default; BN = 128 (SwiGLU only: 64 gate + 64 up columns, 64 output
-// columns per tile) halves the weight bytes per tile, so that weight-streaming
-// launches with few rows per expert split into more, shorter tiles and their
-// last wave is shorter, and it keeps four accumulators in TMEM.
-template <int BN>
+// Single-CTA kernel shapes: BN accumulator columns per tile (MMA N), TM rows
+// per tile. BN = 256, TM = 128 is the default. BN = 128 (SwiGLU only: 64 gate +
+// 64 up columns, 64 output columns per tile) halves the weight bytes per tile,
+// so that weight-streaming launches with few rows per expert split into more,
+// shorter tiles, and it keeps four accumulators in TMEM. TM = 64 (M=64 MMAs,
+// 64-row boxes of the grouped rows) halves the grouped-row bytes per stage, so
+// that the same shared memory holds more stages, i.e. more weight bytes in
+// flight per SM, when the groups are small anyway.
+template <int BN, int TM = 128>
 struct SingleCfg {
-  static constexpr int kBBytes = BN * kBK * 2;                // B rows per stage
-  static constexpr int kStage = kATileBytes + kBBytes;        // 48 KB (256), 32 KB (128)
-  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kABytes = TM * kBK * 2;                // grouped rows per stage
+  static constexpr int kBBytes = BN * kBK * 2;                // weight rows per stage
+  static constexpr int kStage = kABytes + kBBytes;
+  // as many stages as 200 KB hold, at most 8: 4 x 48 KB, 6 x 32 KB, 8 x 24 KB, 5 x 40 KB
+  static constexpr int kStages = (200 * 1024) / kStage < 8 ? (200 * 1024) / kStage : 8;
   static constexpr int kAcc = 512 / BN;                       // accumulators in TMEM
   static constexpr int kHalfRows = BN / 2;                    // rows of one SwiGLU B box
 };
 
 // Dynamic shared memory the kernel needs for a given number of groups.
-template <int BN = 256>
+template <int BN = 256, int TM = 128>
 __host__ __device__ constexpr size_t gemm_smem_bytes(int num_groups) {
-  return 1024 /* alignment slack */ + size_t(SingleCfg<BN>::kStages) * SingleCfg<BN>::kStage +
-         256 /* barriers */ + size_t(2) * (num_groups + 1) * sizeof(int);
+  return 1024 /* alignment slack */ +
+         size_t(SingleCfg<BN, TM>::kStages) * SingleCfg<BN, TM>::kStage + 256 /* barriers */ +
+         size_t(3) * (num_groups + 1) * sizeof(int);
 }
 
 struct TileCoord {
@@ -142,12 +153,31 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, const int* s_off, con
   return c;
 }
 
+// Tile t of a two-class grouped launch: the H tiles of class A sit at positions
+// floor(i*(H+C)/H) of the combined list, the C tiles of class B fill the others
+// in order; inside each class the usual order (group, n-block, m-block).
+__device__ __forceinline__ TileCoord decode_tile_two(int tile, const int* s_off, const int* s_mp,
+                                                     const int* s_mp_b, int num_groups,
+                                                     int n_tiles, int tile_m) {
+  const long long H = static_cast<long long>(s_mp[num_groups]) * n_tiles;
+  const long long total = H + static_cast<long long>(s_mp_b[num_groups]) * n_tiles;
+  if (H > 0) {
+    const long long cnt = ((static_cast<long long>(tile) + 1) * H + total - 1) / total;
+    const long long i = cnt - 1;
+    if (i >= 0 && (i * total) / H == tile)
+      return decode_tile(static_cast<int>(i), s_off, s_mp, num_groups, n_tiles, tile_m);
+    return decode_tile(tile - static_cast<int>(cnt), s_off, s_mp_b, num_groups, n_tiles, tile_m);
+  }
+  return decode_tile(tile, s_off, s_mp_b, num_groups, n_tiles, tile_m);
+}
+
 // Tile t of a launch that may carry an extra dense problem: the X extra tiles
 // sit at positions floor(i*total/X) of the combined list (so they are spread
 // evenly over time and over SMs), the grouped tiles fill the others in order.
 __device__ __forceinline__ TileCoord decode_tile_mixed(int tile, const int* s_off, const int* s_mp,
-                                                       int num_groups, const GemmParams& P,
-                                                       int grouped_tiles, bool& extra) {
+                                                       const int* s_mp_b, int num_groups,
+                                                       const GemmParams& P, int grouped_tiles,
+                                                       bool& extra, int tile_m = kBM) {
   if (P.x_tiles > 0) {
     const long long total = static_cast<long long>(grouped_tiles) + P.x_tiles;
     // number of extra positions <= tile
@@ -168,7 +198,8 @@ __device__ __forceinline__ TileCoord decode_tile_mixed(int tile, const int* s_of
     tile -= static_cast<int>(cnt);
   }
   extra = false;
-  return decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles);
+  if (s_mp_b) return decode_tile_two(tile, s_off, s_mp, s_mp_b, num_groups, P.n_tiles, tile_m);
+  return decode_tile(tile, s_off, s_mp, num_groups, P.n_tiles, tile_m);
 }
 
 __device__ __forceinline__ void raise_timeout(volatile int* s_abort, int* status) {
@@ -177,15 +208,17 @@ __device__ __forceinline__ void raise_timeout(volatile int* s_abort, int* status
 }
 
 
-template <int MODE, int BN = 256>
+template <int MODE, int BN = 256, int TM = 128>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmA2,
                     const __grid_constant__ CUtensorMap tmB0x, const __grid_constant__ CUtensorMap tmB1x,
                     const GemmParams P) {
   static_assert(BN == 256 || (BN == 128 && MODE == kEpiSwiGLU), "BN 128 is a SwiGLU shape");
-  using Cfg = SingleCfg<BN>;
+  static_assert(TM == 128 || TM == 64, "tiles of 128 or 64 rows");
+  using Cfg = SingleCfg<BN, TM>;
   constexpr int kStages = Cfg::kStages;
+  constexpr int kABytes = Cfg::kABytes;
   constexpr int kStageBytes = Cfg::kStage;
   constexpr int kNumAcc = Cfg::kAcc;
   constexpr int kHalfBytes = Cfg::kHalfRows * kBK * 2;       // one SwiGLU B box
@@ -203,6 +236,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   int* s_off = reinterpret_cast<int*>(smem + size_t(kStages) * kStageBytes + 256);
   const int num_groups = P.group_offsets ? P.num_groups : 1;
   int* s_mp = s_off + (num_groups + 1);
+  int* s_mp_b = P.group_mtiles_b ? s_mp + (num_groups + 1) : nullptr;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -240,19 +274,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int i = threadIdx.x; i <= num_groups; i += blockDim.x) {
       s_off[i] = P.group_offsets[i];
       s_mp[i] = P.group_mtiles[i];
+      if (s_mp_b) s_mp_b[i] = P.group_mtiles_b[i];
     }
   } else if (threadIdx.x == 0) {
     s_off[0] = 0;
     s_off[1] = P.dense_rows;
     s_mp[0] = 0;
-    s_mp[1] = (P.dense_rows + kBM - 1) / kBM;
+    s_mp[1] = (P.dense_rows + TM - 1) / TM;
   }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *s_tmem;
 
-  const int grouped_tiles = s_mp[num_groups] * P.n_tiles * P.k_splits;
+  const int grouped_tiles =
+      (s_mp[num_groups] + (s_mp_b ? s_mp_b[num_groups] : 0)) * P.n_tiles * P.k_splits;
   const int total_tiles = grouped_tiles + P.x_tiles;
   // k-block range of a tile: its split's share (split-K launches carry no extra
   // problem), else the whole reduction of the tile's problem
@@ -280,7 +316,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint64_t once = l2_evict_first_policy();
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
       bool ex;
-      const TileCoord tc = decode_tile_mixed(tile, s_off, s_mp, num_groups, P, grouped_tiles, ex);
+      const TileCoord tc = decode_tile_mixed(tile, s_off, s_mp, s_mp_b, num_groups, P, grouped_tiles, ex, TM);
       const int z = (P.group_offsets && !ex) ? tc.group : 0;
       const bool stream = grouped && !ex && tc.mtiles == 1;
       const CUtensorMap* mA = ex ? &tmA2 : &tmA;
@@ -302,7 +338,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (lane == 0) {
           const uint32_t fb = smem_u32(&full_bar[s]);
           const uint32_t a_dst = smem_u32(smem + size_t(s) * kStageBytes);
-          const uint32_t b_dst = a_dst + kATileBytes;
+          const uint32_t b_dst = a_dst + kABytes;
           const int k0 = kb * kBK;
           mbar_arrive_expect_tx(fb, kStageBytes);
           tma_load_2d(a_dst, mA, fb, k0, tc.row0);
@@ -344,7 +380,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     bool ok = true;
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
       bool ex;
-      const TileCoord tc = decode_tile_mixed(tile, s_off, s_mp, num_groups, P, grouped_tiles, ex);
+      const TileCoord tc = decode_tile_mixed(tile, s_off, s_mp, s_mp_b, num_groups, P, grouped_tiles, ex, TM);
       const uint32_t idesc = tc.rows <= 64 ? idesc64 : idesc128;
       int kb_begin, kb_end;
       kb_range(tc, ex, kb_begin, kb_end);
@@ -360,7 +396,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_after_sync();
         if (lane == 0) {
           const uint32_t a_base = smem_u32(smem + size_t(s) * kStageBytes);
-          const uint32_t b_base = a_base + kATileBytes;
+          const uint32_t b_base = a_base + kABytes;
 #pragma unroll
           for (int k = 0; k < kBK / kUK; ++k) {
             umma_bf16(d_tmem, sdesc_kmajor_sw128(a_base + k * kUK * 2),
@@ -396,7 +432,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_ph = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
       bool ex;
-      const TileCoord tc = decode_tile_mixed(tile, s_off, s_mp, num_groups, P, grouped_tiles, ex);
+      const TileCoord tc = decode_tile_mixed(tile, s_off, s_mp, s_mp_b, num_groups, P, grouped_tiles, ex, TM);
       void* const out_base = ex ? P.x_out : P.out;
       const long long ldo = ex ? P.x_ldo : P.ldo;
       const int n_valid = ex ? P.x_N : P.N;

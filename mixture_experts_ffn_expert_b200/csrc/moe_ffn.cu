@@ -43,7 +43,7 @@ constexpr int kTimingRing = 4;   // event sets: forward i records into set i % k
 
 struct Layout {
   size_t status, ticket, scores, idx, gate, chunk_counts, sub_base, counts, offsets, mtiles,
-      mtiles2, perm_src, inv_pos;
+      mtiles2, mtiles64, mt_hot, mt_cold, perm_src, inv_pos;
   size_t xperm, hidden, yrouted, hshared, yshared, total;
   int lds;            // row stride of the fp32 router scores
   int tpc;            // tokens per routing chunk (a block of route_scatter)
@@ -80,6 +80,13 @@ struct moe_plan {
   // the expected rows per expert are below 32, the weight-streaming regime,
   // else 128), 64 or 128
   int swiglu_tile_cols = 0;
+  // interleave the tiles of experts with several m-blocks among the others in
+  // single-CTA 128-row routed GEMMs: -1 automatic (when the expected rows per
+  // expert are below 192, i.e. most experts stream weights), 0 never, 1 always
+  int interleave = -1;
+  // rows of a single-CTA routed GEMM tile: 0 automatic (64 when the expected
+  // rows per expert are below 32, else 128), 64 or 128
+  int tile_rows = 0;
   // shared expert beside weight-streaming routed GEMMs: -1 automatic, 0 never, 1 always.
   // Measured on B200 (DeepSeek-V3-shaped prefill): beside the routed GEMMs on 16
   // SMs the layer took 7.09 ms per step against 6.19 ms inline (the capped
@@ -124,21 +131,17 @@ struct moe_plan {
 
 namespace {
 
-// Launch shape of the fused router for T tokens (see router_sm100.cuh): the
-// cluster size CS splits each 128-token tile's K range; CS is at least N_r/64
-// so that one CTA's scores (128/CS tokens x N_r fp32) fit in 32 KB, and grows
-// (up to 8, and up to the number of K blocks) until the grid covers about
-// three quarters of the SMs.
+// Launch shape of the fused router for T tokens (see router_sm100.cuh): a
+// cluster of CS CTAs per 128-token tile, CTA r scoring experts
+// [r*E, (r+1)*E) over the whole K range. CS is the power of two that makes the
+// slices about 64 experts (E <= 256), at most 8.
 moe::RouterParams router_shape(const moe_plan* p, int64_t T, size_t* smem) {
   moe::RouterParams r{};
   const int nr = p->n_routed;
   const int mt = static_cast<int>((T + moe::kBM - 1) / moe::kBM);
-  const int num_kb = (p->d + moe::kBK - 1) / moe::kBK;
-  int cs = nr <= 64 ? 1 : (nr <= 128 ? 2 : (nr <= 256 ? 4 : 8));
-  while (cs < moe::kRtMaxCluster && static_cast<long long>(mt) * cs < (3LL * p->num_sms) / 4 &&
-         cs < num_kb)
-    cs *= 2;
   auto up = [](int v, int m) { return (v + m - 1) / m * m; };
+  int cs = 1;
+  while (cs < moe::kRtMaxCluster && (nr + cs - 1) / cs > 64) cs *= 2;
   r.T = static_cast<int>(T);
   r.d = p->d;
   r.n_routed = nr;
@@ -146,39 +149,30 @@ moe::RouterParams router_shape(const moe_plan* p, int64_t T, size_t* smem) {
   r.renorm = p->renorm;
   r.bias_select_only = p->bias_select_only;
   r.cs = cs;
-  r.num_kb = num_kb;
-  r.kb_per = (num_kb + cs - 1) / cs;
+  r.e_per = up((nr + cs - 1) / cs, 16);
+  r.ncols = up(r.e_per, 32);
+  r.num_kb = (p->d + moe::kBK - 1) / moe::kBK;
   r.own_rows = moe::kBM / cs;
-  r.n_chunks = mt;                 // one chunk of the histogram per 128-token tile
-  r.n_acc = nr > 256 ? 2 : 1;
-  r.mma_n0 = up(nr < 256 ? nr : 256, 16);
-  r.mma_n1 = r.n_acc > 1 ? up(nr - 256, 16) : 0;
-  r.ncols0 = up(nr < 256 ? nr : 256, 32);
-  r.ncols1 = r.n_acc > 1 ? up(nr - 256, 32) : 0;
-  r.box_rows = r.mma_n0 < 128 ? r.mma_n0 : 128;
-  r.nbox0 = (r.mma_n0 + r.box_rows - 1) / r.box_rows;
-  r.nbox1 = r.n_acc > 1 ? (r.mma_n1 + r.box_rows - 1) / r.box_rows : 0;
-  const int box_bytes = r.box_rows * moe::kBK * 2;
-  r.b_acc1_off = moe::kATileBytes + r.nbox0 * box_bytes;
-  r.stage_bytes = moe::kATileBytes + (r.nbox0 + r.nbox1) * box_bytes;
-  int stages = (160 * 1024) / r.stage_bytes;
-  if (stages > r.kb_per + 1) stages = r.kb_per + 1;
+  r.n_chunks = mt;                 // one column of the histogram per 128-token tile
+  r.box_rows = r.e_per < 128 ? r.e_per : 128;
+  r.nbox = (r.e_per + r.box_rows - 1) / r.box_rows;
+  r.stage_bytes = moe::kATileBytes + r.nbox * r.box_rows * moe::kBK * 2;
+  int stages = (168 * 1024) / r.stage_bytes;
+  if (stages > r.num_kb) stages = r.num_kb;
   stages = stages < 2 ? 2 : (stages > moe::kRtMaxStages ? moe::kRtMaxStages : stages);
   r.stages = stages;
-  const int exch = moe::kBM * ((r.ncols0 > r.ncols1 ? r.ncols0 : r.ncols1) + 4) * 4;
-  const int ring = stages * r.stage_bytes;
-  r.ring_bytes = up(ring > exch ? ring : exch, 1024);
-  r.lds = up(nr, 32);
+  r.ring_bytes = up(stages * r.stage_bytes, 1024);
   int cols = 32;
-  while (cols < r.ncols0) cols *= 2;
-  r.tmem_cols = r.n_acc > 1 ? 512 : cols;
-  // fold the chunk scan into the router's last cluster while there are few
-  // chunks (one thread per expert walks them)
+  while (cols < r.ncols) cols *= 2;
+  r.tmem_cols = cols;
+  // fold the tile scan into the router's last cluster while there are few
+  // tiles (one thread per expert walks them)
   r.fold_scan = r.n_chunks <= 64 ? 1 : 0;
   // at least kRouterMinSmem so that two router CTAs never share an SM: each
-  // allocates tensor memory and waits at cluster barriers, and two clusters
-  // interleaved on two SMs could otherwise wait on each other's allocation
-  size_t bytes = moe::router_smem_bytes(r.ring_bytes, r.own_rows, r.lds, nr);
+  // allocates tensor memory and then waits at cluster barriers, and two
+  // clusters interleaved on two SMs could otherwise wait on each other
+  const size_t bytes = p->top_k <= 8 ? moe::router_smem_bytes<8>(r.ring_bytes, nr)
+                                      : moe::router_smem_bytes<16>(r.ring_bytes, nr);
   *smem = bytes < kRouterMinSmem ? kRouterMinSmem : bytes;
   return r;
 }
@@ -187,7 +181,8 @@ Layout make_layout(const moe_plan* p, int64_t T) {
   Layout L{};
   const int64_t A = T * p->top_k;
   const int nsf = p->n_shared * p->f;
-  L.fused = p->fused_router != 0 && p->n_routed <= moe::kRtMaxExperts;
+  L.fused = p->fused_router != 0 && p->n_routed <= moe::kRtMaxExperts &&
+            p->top_k <= moe::kRtMaxTopK;
   L.lds = static_cast<int>(align_up(p->n_routed, 8));
   if (L.fused) {
     // the router's histogram has one column per 128-token tile, plus each CTA's
@@ -230,6 +225,9 @@ Layout make_layout(const moe_plan* p, int64_t T) {
   L.offsets = take(size_t(p->n_routed + 1) * 4);
   L.mtiles = take(size_t(p->n_routed + 1) * 4);
   L.mtiles2 = take(size_t(p->n_routed + 1) * 4);
+  L.mtiles64 = take(size_t(p->n_routed + 1) * 4);
+  L.mt_hot = take(size_t(p->n_routed + 1) * 4);
+  L.mt_cold = take(size_t(p->n_routed + 1) * 4);
   L.perm_src = take(size_t(A) * 4);
   L.inv_pos = take(size_t(A) * 4);
   L.xperm = take(size_t(A) * p->d * 2);
@@ -387,21 +385,24 @@ bool launch_pair_auto(Launcher& L, cudaStream_t s, const char* name, const CUten
 // Single-CTA GEMM with BN accumulator columns per tile. x (optional) holds the
 // A, B0, B1 maps of the extra dense problem that prm.x_tiles describes;
 // max_tiles bounds the grouped tiles only.
-template <int MODE, int BN = 256>
+template <int MODE, int BN = 256, int TM = 128>
 bool launch_gemm(Launcher& L, cudaStream_t s, const char* name, const CUtensorMap& a,
                  const CUtensorMap& b0, const CUtensorMap& b1, const moe::GemmParams& prm,
                  int max_tiles, const CUtensorMap* x = nullptr) {
   const int num_groups = prm.group_offsets ? prm.num_groups : 1;
-  const size_t smem = moe::gemm_smem_bytes<BN>(num_groups);
+  const size_t smem = moe::gemm_smem_bytes<BN, TM>(num_groups);
   const long long tiles = static_cast<long long>(max_tiles) + (x ? prm.x_tiles : 0);
   const int sms = L.p->num_sms < L.grid_cap ? L.p->num_sms : L.grid_cap;
   int grid = tiles < sms ? static_cast<int>(tiles) : sms;
   if (grid < 1) grid = 1;
   moe::GemmParams q = prm;
   if (!x) q.x_tiles = 0;
-  L.begin(name, s, q.x_tiles > 0 ? "[+shared]" : (BN == 128 ? "[n64]" : ""));
-  launch_pdl(moe::moe_gemm_kernel<MODE, BN>, dim3(grid), dim3(moe::kGemmThreads), smem, s, a,
-             b0, b1, x ? x[0] : a, x ? x[1] : b0, x ? x[2] : b1, q);
+  const char* tag = q.x_tiles > 0 ? "[+shared]"
+                    : BN == 128 ? (TM == 64 ? "[n64,m64]" : "[n64]")
+                    : (TM == 64 ? "[m64]" : "");
+  L.begin(name, s, tag);
+  launch_pdl(moe::moe_gemm_kernel<MODE, BN, TM>, dim3(grid), dim3(moe::kGemmThreads), smem, s,
+             a, b0, b1, x ? x[0] : a, x ? x[1] : b0, x ? x[2] : b1, q);
   return L.end(name, s);
 }
 
@@ -422,11 +423,18 @@ int set_kernel_attributes() {
     if (e != cudaSuccess)
       return fail(MOE_CUDA_ERROR, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
   const size_t smem = moe::gemm_smem_bytes(moe::kMaxRouted);
-  const cudaError_t e0 = cudaFuncSetAttribute(
-      moe::moe_gemm_kernel<moe::kEpiSwiGLU, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-      int(moe::gemm_smem_bytes<128>(moe::kMaxRouted)));
-  if (e0 != cudaSuccess)
-    return fail(MOE_CUDA_ERROR, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e0));
+  const cudaError_t e0[4] = {
+      cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiSwiGLU, 128>, attr,
+                           int(moe::gemm_smem_bytes<128>(moe::kMaxRouted))),
+      cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiSwiGLU, 128, 64>, attr,
+                           int(moe::gemm_smem_bytes<128, 64>(moe::kMaxRouted))),
+      cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiSwiGLU, 256, 64>, attr,
+                           int(moe::gemm_smem_bytes<256, 64>(moe::kMaxRouted))),
+      cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiBF16, 256, 64>, attr,
+                           int(moe::gemm_smem_bytes<256, 64>(moe::kMaxRouted)))};
+  for (cudaError_t e : e0)
+    if (e != cudaSuccess)
+      return fail(MOE_CUDA_ERROR, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
   cudaError_t e1 = cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiSwiGLU>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   cudaError_t e2 = cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiBF16>,
@@ -437,10 +445,7 @@ int set_kernel_attributes() {
     return fail(MOE_CUDA_ERROR, "cudaFuncSetAttribute failed: %s",
                 cudaGetErrorString(e1 != cudaSuccess ? e1 : (e2 != cudaSuccess ? e2 : e3)));
   const int rsm = 227 * 1024;
-  const cudaError_t er[5] = {cudaFuncSetAttribute(moe::route_fused_kernel<1>, attr, rsm),
-                             cudaFuncSetAttribute(moe::route_fused_kernel<2>, attr, rsm),
-                             cudaFuncSetAttribute(moe::route_fused_kernel<4>, attr, rsm),
-                             cudaFuncSetAttribute(moe::route_fused_kernel<8>, attr, rsm),
+  const cudaError_t er[2] = {cudaFuncSetAttribute(moe::route_fused_kernel<8>, attr, rsm),
                              cudaFuncSetAttribute(moe::route_fused_kernel<16>, attr, rsm)};
   for (cudaError_t e : er)
     if (e != cudaSuccess)
@@ -466,11 +471,7 @@ cudaError_t launch_router(const Layout& Lw, const moe::RouterParams& rt, const C
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  const int npl = (rt.n_routed + 31) / 32;
-  if (npl <= 1) return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<1>, mX, mWg, rt);
-  if (npl <= 2) return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<2>, mX, mWg, rt);
-  if (npl <= 4) return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<4>, mX, mWg, rt);
-  if (npl <= 8) return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<8>, mX, mWg, rt);
+  if (rt.top_k <= 8) return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<8>, mX, mWg, rt);
   return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<16>, mX, mWg, rt);
 }
 
@@ -620,6 +621,15 @@ int moe_plan_set_option(moe_plan_t p, int option, int64_t value) {
         return fail(MOE_INVALID_ARG, "shared_concurrent must be -1, 0 or 1");
       p->shared_concurrent = static_cast<int>(value);
       return MOE_OK;
+    case MOE_OPTION_INTERLEAVE:
+      if (value < -1 || value > 1) return fail(MOE_INVALID_ARG, "interleave must be -1, 0 or 1");
+      p->interleave = static_cast<int>(value);
+      return MOE_OK;
+    case MOE_OPTION_TILE_ROWS:
+      if (value != 0 && value != 64 && value != 128)
+        return fail(MOE_INVALID_ARG, "tile rows must be 0, 64 or 128");
+      p->tile_rows = static_cast<int>(value);
+      return MOE_OK;
     case MOE_OPTION_SWIGLU_TILE_COLS:
       if (value != 0 && value != 64 && value != 128)
         return fail(MOE_INVALID_ARG, "swiglu tile columns must be 0, 64 or 128");
@@ -718,6 +728,9 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   int* offsets = reinterpret_cast<int*>(ws + Lw.offsets);
   int* mtiles = reinterpret_cast<int*>(ws + Lw.mtiles);
   int* mtiles2 = reinterpret_cast<int*>(ws + Lw.mtiles2);
+  int* mtiles64 = reinterpret_cast<int*>(ws + Lw.mtiles64);
+  int* mt_hot = reinterpret_cast<int*>(ws + Lw.mt_hot);
+  int* mt_cold = reinterpret_cast<int*>(ws + Lw.mt_cold);
   int* perm_src = reinterpret_cast<int*>(ws + Lw.perm_src);
   int* inv_pos = reinterpret_cast<int*>(ws + Lw.inv_pos);
   void* xperm = ws + Lw.xperm;
@@ -917,7 +930,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
                Lw.n_chunks / Lw.n_base, (const int*)counts,
                static_cast<int>(T), k, nr, Lw.tpc, Lw.n_chunks, moe::kBM, seat_limit,
                reinterpret_cast<const uint4*>(x), d / 8, reinterpret_cast<uint4*>(xperm),
-               perm_src, inv_pos, offsets, mtiles, mtiles2, status);
+               perm_src, inv_pos, offsets, mtiles, mtiles2, mtiles64, mt_hot, mt_cold, status);
     if (!L.end("route_scatter", main_st)) return L.status;
   }
   const int max_mtiles = static_cast<int>((A + 127) / 128 + (A < nr ? A : nr));
@@ -938,14 +951,30 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   if (shared_sms > 0) L.grid_cap = p->num_sms - shared_sms;
   // 5. grouped gate/up GEMM with the SiLU(gate) * up epilogue. With few rows
   //    per expert (weight streaming) the single-CTA kernel uses 64-column
-  //    tiles: twice as many, shorter tiles, so the last wave is shorter.
+  //    tiles (twice as many, shorter tiles, so the last wave is shorter) of 64
+  //    rows (more stages, so more weight bytes in flight per SM).
   const bool narrow_gu =
       !routed_pair_swiglu && !merge_gu &&
       (p->swiglu_tile_cols == 64 || (p->swiglu_tile_cols == 0 && rows_per_expert < 32));
+  const bool short_gu = !routed_pair_swiglu && !merge_gu &&
+                        (p->tile_rows == 64 || (p->tile_rows == 0 && rows_per_expert < 32));
+  const bool short_dn = !routed_pair && !merge_dn &&
+                        (p->tile_rows == 64 || (p->tile_rows == 0 && rows_per_expert < 32));
+  const int max_mtiles64 = static_cast<int>((A + 63) / 64 + (A < nr ? A : nr));
+  // 128-row single-CTA routed GEMMs in the weight-streaming regime run the
+  // tiles of experts with several m-blocks (tensor-heavy: each weight tile is
+  // reused through L2) spread evenly among the weight-streaming experts' tiles,
+  // so that tensor and HBM work overlap instead of alternating
+  const bool interleave =
+      p->interleave == 1 || (p->interleave == -1 && rows_per_expert < 192);
+  CUtensorMap mXp64, mH64;
+  if ((short_gu && !make_map(&mXp64, xperm, 0, A, d, 64)) ||
+      (short_dn && !make_map(&mH64, hidden, 0, A, f, 64)))
+    return fail(MOE_CUDA_ERROR, "cuTensorMapEncodeTiled rejected a tensor map");
   {
     moe::GemmParams g{};
     g.group_offsets = offsets;
-    g.group_mtiles = routed_pair_swiglu ? mtiles2 : mtiles;
+    g.group_mtiles = routed_pair_swiglu ? mtiles2 : (short_gu ? mtiles64 : mtiles);
     g.num_groups = nr;
     g.K = d;
     g.N = f;
@@ -967,27 +996,38 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
       g.x_out = hshared;
       g.x_ldo = nsf;
     }
+    const int mtmax = short_gu ? max_mtiles64 : max_mtiles;
+    bool launched;
     if (narrow_gu) {
       CUtensorMap mW1n, mW3n;
       if (!make_map(&mW1n, W1, nr, f, d, 64) || !make_map(&mW3n, W3, nr, f, d, 64))
         return fail(MOE_CUDA_ERROR, "cuTensorMapEncodeTiled rejected a tensor map");
-      if (!launch_gemm<moe::kEpiSwiGLU, 128>(L, main_st, "grouped_gate_up", mXp, mW1n, mW3n, g,
-                                             max_mtiles * g.n_tiles))
-        return L.status;
-    } else if (routed_pair_swiglu
-                   ? !launch_pair_auto<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1,
-                                                        mW3, g, f, expected_mtiles2, max_mtiles2)
-                   : !launch_gemm<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1, mW3,
-                                                   g, max_mtiles * g.n_tiles,
-                                                   merge_gu ? xgu : nullptr)) {
-      return L.status;
+      launched = short_gu ? launch_gemm<moe::kEpiSwiGLU, 128, 64>(L, main_st, "grouped_gate_up",
+                                                                  mXp64, mW1n, mW3n, g,
+                                                                  mtmax * g.n_tiles)
+                          : launch_gemm<moe::kEpiSwiGLU, 128>(L, main_st, "grouped_gate_up", mXp,
+                                                              mW1n, mW3n, g, mtmax * g.n_tiles);
+    } else if (routed_pair_swiglu) {
+      launched = launch_pair_auto<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1, mW3, g,
+                                                   f, expected_mtiles2, max_mtiles2);
+    } else if (short_gu) {
+      launched = launch_gemm<moe::kEpiSwiGLU, 256, 64>(L, main_st, "grouped_gate_up", mXp64, mW1,
+                                                       mW3, g, mtmax * g.n_tiles);
+    } else {
+      if (interleave && !merge_gu) {
+        g.group_mtiles = mt_hot;
+        g.group_mtiles_b = mt_cold;
+      }
+      launched = launch_gemm<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1, mW3, g,
+                                              mtmax * g.n_tiles, merge_gu ? xgu : nullptr);
     }
+    if (!launched) return L.status;
   }
   // 6. grouped down GEMM
   {
     moe::GemmParams g{};
     g.group_offsets = offsets;
-    g.group_mtiles = routed_pair ? mtiles2 : mtiles;
+    g.group_mtiles = routed_pair ? mtiles2 : (short_dn ? mtiles64 : mtiles);
     g.num_groups = nr;
     g.K = f;
     g.N = d;
@@ -1006,12 +1046,22 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
       g.x_ldo = d;
       g.x_out_f32 = 1;
     }
-    if (routed_pair ? !launch_pair_auto<moe::kEpiBF16>(L, main_st, "grouped_down", mH, mW2, mW2, g,
-                                                       d, expected_mtiles2, max_mtiles2)
-                    : !launch_gemm<moe::kEpiBF16>(L, main_st, "grouped_down", mH, mW2, mW2, g,
-                                                  max_mtiles * g.n_tiles,
-                                                  merge_dn ? xdn : nullptr))
-      return L.status;
+    bool launched;
+    if (routed_pair)
+      launched = launch_pair_auto<moe::kEpiBF16>(L, main_st, "grouped_down", mH, mW2, mW2, g, d,
+                                                 expected_mtiles2, max_mtiles2);
+    else if (short_dn)
+      launched = launch_gemm<moe::kEpiBF16, 256, 64>(L, main_st, "grouped_down", mH64, mW2, mW2,
+                                                     g, max_mtiles64 * g.n_tiles);
+    else {
+      if (interleave && !merge_dn) {
+        g.group_mtiles = mt_hot;
+        g.group_mtiles_b = mt_cold;
+      }
+      launched = launch_gemm<moe::kEpiBF16>(L, main_st, "grouped_down", mH, mW2, mW2, g,
+                                            max_mtiles * g.n_tiles, merge_dn ? xdn : nullptr);
+    }
+    if (!launched) return L.status;
   }
   L.grid_cap = INT_MAX;
   // 7. the shared expert (inline, merged, or joined from the side stream), then

@@ -65,9 +65,7 @@ __device__ __forceinline__ void route_token(float (&v)[NPL], const float* __rest
 
   // Selection keys: a NaN score (from NaN or infinite inputs) ranks as -inf,
   // so the order stays total and every lane agrees on each winner. Each key is
-  // mapped to an unsigned integer with the same order (-0 and +0 equal), so a
-  // round of the selection is two warp reductions (redux.sync): the largest key,
-  // then the lowest expert index holding it - ties go to the lower index. An
+  // mapped to an unsigned integer with the same order (-0 and +0 equal); an
   // empty lane's 0 is below every real key (-inf maps to 0x007fffff).
   uint32_t okey[NPL];
 #pragma unroll
@@ -77,31 +75,45 @@ __device__ __forceinline__ void route_token(float (&v)[NPL], const float* __rest
     const uint32_t b = __float_as_uint(kv);
     okey[i] = lane + 32 * i < n_routed ? ((b & 0x80000000u) ? ~b : (b | 0x80000000u)) : 0u;
   }
+  // Each lane keeps its best untaken expert (largest key, lowest index among
+  // equal keys) with its gate score. A round of the selection is two warp
+  // reductions (redux.sync): the largest key, then the lowest expert index
+  // holding it - ties go to the lower index; only the winning lane rescans.
   uint32_t taken = 0;
-  float sel_sum = 0.0f, my_p = 0.0f;
+  uint32_t lk = 0u;
+  int li = 0x7fffffff;
+  float lv = 0.0f;
+  auto rescan = [&]() {
+    lk = 0u;
+    li = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+      if (!((taken >> i) & 1u) && okey[i] > lk) {   // ascending i: '>' keeps the lower index
+        lk = okey[i];
+        li = lane + 32 * i;
+        lv = v[i];
+      }
+  };
+  rescan();
+  float my_gw = 0.0f;
   my_e = -1;
   for (int j = 0; j < top_k; ++j) {
-    uint32_t lmax = 0u;
-#pragma unroll
-    for (int i = 0; i < NPL; ++i)
-      if (!((taken >> i) & 1u)) lmax = okey[i] > lmax ? okey[i] : lmax;
-    const uint32_t gmax = __reduce_max_sync(0xffffffffu, lmax);
-    int lidx = 0x7fffffff;
-#pragma unroll
-    for (int i = NPL - 1; i >= 0; --i)     // descending: the last match is the lowest index
-      if (!((taken >> i) & 1u) && okey[i] == gmax) lidx = lane + 32 * i;
-    const int be = static_cast<int>(__reduce_min_sync(0xffffffffu, static_cast<unsigned>(lidx)));
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    // the winner's gate score, from the lane that holds it
-    float gw = 0.0f;
-#pragma unroll
-    for (int i = 0; i < NPL; ++i)
-      if (i == (be >> 5)) gw = v[i];
-    gw = __shfl_sync(0xffffffffu, gw, be & 31);
-    const float p = expf(gw - m) / sum;
-    sel_sum += p;
-    if (lane == j) { my_p = p; my_e = be; }
+    const uint32_t gmax = __reduce_max_sync(0xffffffffu, lk);
+    const int be = static_cast<int>(
+        __reduce_min_sync(0xffffffffu, static_cast<unsigned>(lk == gmax ? li : 0x7fffffff)));
+    const float gw = __shfl_sync(0xffffffffu, lv, be & 31);   // the winner's gate score
+    if (lane == j) { my_gw = gw; my_e = be; }
+    if ((be & 31) == lane) {
+      taken |= 1u << (be >> 5);
+      rescan();
+    }
   }
+  // lane j < top_k: the probability of the j-th selected expert; the sum over
+  // the selected ones for the renormalisation
+  const float my_p = lane < top_k ? expf(my_gw - m) / sum : 0.0f;
+  float sel_sum = my_p;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sel_sum += __shfl_xor_sync(0xffffffffu, sel_sum, o);
   my_g = renorm ? my_p / sel_sum : my_p;
 }
 
@@ -285,7 +297,8 @@ __global__ void __launch_bounds__(kRouteThreads)
                          int d_vec, uint4* __restrict__ xperm, int* __restrict__ perm_src,
                          int* __restrict__ inv_pos, int* __restrict__ offsets_out,
                          int* __restrict__ mtiles_out, int* __restrict__ mtiles2_out,
-                         int* __restrict__ status) {
+                         int* __restrict__ mtiles4_out, int* __restrict__ mt_hot_out,
+                         int* __restrict__ mt_cold_out, int* __restrict__ status) {
   extern __shared__ int smem_i[];
   int* s_off = smem_i;                        // [kMaxRouted] expert offsets
   int* s_run = smem_i + kMaxRouted;           // [n_routed]
@@ -339,13 +352,22 @@ __global__ void __launch_bounds__(kRouteThreads)
     // publish offsets and the m-tile prefix for the grouped GEMMs
     for (int e = threadIdx.x; e < n_routed; e += blockDim.x) offsets_out[e] = s_off[e];
     if (threadIdx.x == 0) offsets_out[n_routed] = total;
-    // prefixes of m-tiles of tile_rows and of 2*tile_rows rows (CTA-pair tiles)
-    for (int pass = 0; pass < 2; ++pass) {
-      const int rows = tile_rows << pass;
-      int* dst = pass ? mtiles2_out : mtiles_out;
+    // prefixes of m-tiles of tile_rows, 2*tile_rows (CTA-pair tiles) and
+    // tile_rows/2 rows (the 64-row tiles of weight-streaming launches), and the
+    // tile_rows prefix split in two classes: experts with at least two m-tiles
+    // (their tiles reuse a weight tile through L2: tensor-heavy) and the others
+    // (weight-streaming), which a launch may interleave
+    for (int pass = 0; pass < 5; ++pass) {
+      const int rows = pass == 2 ? tile_rows / 2 : (pass == 1 ? tile_rows * 2 : tile_rows);
+      int* dst = pass == 0 ? mtiles_out
+               : pass == 1 ? mtiles2_out
+               : pass == 2 ? mtiles4_out
+               : pass == 3 ? mt_hot_out : mt_cold_out;
       __syncthreads();
-      for (int e = threadIdx.x; e < n_routed; e += blockDim.x)
-        s_run[e] = bad ? 0 : (min(counts[e], capacity) + rows - 1) / rows;
+      for (int e = threadIdx.x; e < n_routed; e += blockDim.x) {
+        const int mt = bad ? 0 : (min(counts[e], capacity) + rows - 1) / rows;
+        s_run[e] = pass == 3 ? (mt >= 2 ? mt : 0) : (pass == 4 ? (mt == 1 ? 1 : 0) : mt);
+      }
       __syncthreads();
       const int total_mt = block_exclusive_scan(s_run, n_routed, s_tmp);
       for (int e = threadIdx.x; e < n_routed; e += blockDim.x) {

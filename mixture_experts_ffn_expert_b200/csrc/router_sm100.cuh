@@ -1,30 +1,31 @@
 // router_sm100.cuh - the fused router: for a tile of 128 tokens, the router
 // scores s = x W_g^T on the 5th-generation tensor core, the softmax over the N_r
-// experts, the warp-shuffle top-k with ties to the lower expert index, the gates
-// and the per-chunk expert histogram, in one launch ("What is an "expert,"
-// really?", glossary: router / gate, top-k, softmax; panel 2: a linear scorer,
-// softmax blend weights, keep the top k). With few chunks the last CTA of the
-// grid also turns the histogram into per-chunk bases and expert totals, so the
+// experts, the top-k with ties to the lower expert index, the gates and the
+// expert histogram, in one launch ("What is an "expert," really?", glossary:
+// router / gate, top-k, softmax; panel 2: a linear scorer, softmax blend
+// weights, keep the top k). With few tiles the last cluster of the grid also
+// turns the histogram into per-tile bases and expert totals, so the
 // permutation kernel can follow directly.
 //
-// Design (sm_100a, N_r <= 512):
-//  * a cluster of CS CTAs (CS <= 8) owns one 128-token tile; CTA r of the
-//    cluster reduces over its own K range (split-K) for ALL experts, so each
-//    CTA streams 1/CS of the token rows and of W_g through TMA (no multicast);
-//  * warp 0 loads A (x rows, one 128x64 box) and B (W_g rows, boxes of up to
-//    128 rows) per 64-wide K block; warp 1 issues tcgen05.mma M=128 into one
-//    or two TMEM accumulators of <= 256 columns;
-//  * the partial scores are reduced across the cluster through distributed
-//    shared memory: each CTA copies its accumulator (warps 4..7, one TMEM lane
-//    quarter each) into its own shared memory, and after a cluster barrier the
-//    CTA that routes tokens m .. m + 128/CS - 1 reads those rows from every CTA
-//    of the cluster (coalesced 16-byte loads) and adds the CS partials in rank
-//    order (deterministic), up to 256 experts per round;
-//  * every warp then routes tokens of its CTA with route_token (one warp per
-//    token, N_r/32 scores per lane), writes idx and gates, and counts experts in
-//    a shared histogram; reading the cluster's histograms, each CTA writes its
-//    experts' offsets within the tile (the pairs of lower-ranked CTAs) and the
-//    first CTA the tile's totals, one column of the tile histogram.
+// Design (sm_100a, N_r <= 512, top_k <= 16):
+//  * a cluster of CS CTAs (CS <= 8) owns one 128-token tile; CTA r computes the
+//    scores of its slice of E = N_r/CS experts over the whole K range (one
+//    TMEM accumulator of <= 256 columns), so no partial sums are exchanged;
+//  * warp 0 loads A (x rows, one 128x64 box) and B (the slice's W_g rows, boxes
+//    of up to 128 rows) per 64-wide K block through TMA (no multicast); warp 1
+//    issues tcgen05.mma M=128, N=E;
+//  * warps 4..7 read the accumulator, one thread per token (its TMEM lane): the
+//    slice's softmax statistics (its largest gate score and the sum of
+//    exp(score - largest)) and its top-k candidates (selection key, expert, gate
+//    score), kept sorted in registers - all 128 tokens of the tile at once;
+//  * after a cluster barrier, one warp per token of this CTA's 128/CS tokens
+//    gathers the CS slices' candidates and statistics through distributed
+//    shared memory and selects the top k among them with warp reductions
+//    (largest key, then lowest index: ties to the lower expert index); the
+//    softmax over all N_r experts follows from the statistics;
+//  * a shared histogram per CTA; reading the cluster's histograms, each CTA
+//    writes its experts' offsets inside the tile and the first CTA the tile's
+//    totals, one column of the tile histogram.
 #pragma once
 
 #include "gemm_sm100.cuh"
@@ -32,31 +33,28 @@
 
 namespace moe {
 
-constexpr int kRtThreads = 256;
+constexpr int kRtThreads = 512;   // 16 warps: 16 tokens merged at once per CTA
 constexpr int kRtMaxCluster = 8;
 constexpr int kRtMaxStages = 8;
 constexpr int kRtMaxExperts = 512;
+constexpr int kRtMaxTopK = 16;
 
 struct RouterParams {
   int T, d, n_routed, top_k, renorm, bias_select_only;
   const float* bias;     // device (N_r) or null
-  int cs;                // CTAs per cluster = K splits of one token tile
-  int kb_per;            // 64-wide K blocks per CTA
-  int num_kb;            // K blocks of d
-  int own_rows;          // tokens each CTA routes (128 / cs)
+  int cs;                // CTAs per cluster = expert slices of one token tile
+  int e_per;             // experts per slice (multiple of 16, <= 256): MMA N
+  int ncols;             // accumulator columns read (e_per rounded up to 32)
+  int num_kb;            // 64-wide K blocks of d
+  int own_rows;          // tokens each CTA merges (128 / cs)
   int n_chunks;          // ceil(T / 128): columns of tile_counts
-  int n_acc;             // accumulators (1, or 2 when N_r > 256)
-  int mma_n0, mma_n1;    // MMA N of each accumulator (multiples of 16)
-  int ncols0, ncols1;    // exchanged columns of each accumulator (multiples of 32)
   int box_rows;          // rows of one W_g TMA box
-  int nbox0, nbox1;      // W_g boxes per accumulator per stage
+  int nbox;              // W_g boxes per stage
   int stages;
   int stage_bytes;       // A box + B boxes of one stage
-  int b_acc1_off;        // offset of accumulator 1's B rows inside a stage
-  int ring_bytes;        // the stage ring, reused as the exchange buffer
-  int lds;               // row stride (floats) of the CTA's score buffer
+  int ring_bytes;
   int tmem_cols;
-  int fold_scan;         // 1: the grid's last cluster scans the chunk histogram
+  int fold_scan;         // 1: the grid's last cluster scans the tile histogram
   int* idx;              // (T, top_k)
   float* gate;           // (T, top_k)
   int* tile_counts;      // [N_r][n_chunks] pairs per expert and tile (scanned in place)
@@ -66,37 +64,50 @@ struct RouterParams {
   int* status;           // device status word
 };
 
-// Dynamic shared memory of a launch: ring, scores, histogram, barriers.
-__host__ __device__ constexpr size_t router_smem_bytes(int ring_bytes, int own_rows, int lds,
-                                                       int n_routed) {
-  return 1024 + size_t(ring_bytes) + size_t(own_rows) * lds * 4 +
+// Shared memory of the candidates: KMAX per token of the tile (top_k <= KMAX)
+// as (key, expert, gate score), plus the token's (max, sum) statistics.
+template <int KMAX>
+__host__ __device__ constexpr size_t router_cand_bytes() {
+  return size_t(kBM) * KMAX * 12 + size_t(kBM) * 8;
+}
+
+// Dynamic shared memory of a launch: ring, candidates, histogram, barriers.
+template <int KMAX>
+__host__ __device__ constexpr size_t router_smem_bytes(int ring_bytes, int n_routed) {
+  return 1024 + size_t(ring_bytes) + router_cand_bytes<KMAX>() +
          size_t((n_routed + 3) / 4 * 4) * 4 + 256;
 }
 
-__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
   return v;
 }
 
-__device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
-  int v;
-  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
+// Order-preserving map of a selection key to an unsigned integer: NaN ranks
+// as -inf, -0 equals +0, and -inf maps to 0x007fffff, above the 0 that marks
+// an empty candidate.
+__device__ __forceinline__ uint32_t order_key(float k) {
+  k = k == k ? k : -INFINITY;
+  k = k == 0.0f ? 0.0f : k;
+  const uint32_t b = __float_as_uint(k);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-template <int NPL>
+template <int KMAX>
 __global__ void __launch_bounds__(kRtThreads, 1)
     route_fused_kernel(const __grid_constant__ CUtensorMap tmX,
                        const __grid_constant__ CUtensorMap tmWg, const RouterParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  float* s_scores = reinterpret_cast<float*>(ring + P.ring_bytes);
-  int* s_hist = reinterpret_cast<int*>(s_scores + size_t(P.own_rows) * P.lds);
+  // candidates of the 128 tokens of the tile from this CTA's slice, [token][slot]
+  uint32_t* c_key = reinterpret_cast<uint32_t*>(ring + P.ring_bytes);
+  int* c_idx = reinterpret_cast<int*>(c_key + kBM * KMAX);
+  float* c_val = reinterpret_cast<float*>(c_idx + kBM * KMAX);
+  float* c_max = c_val + kBM * KMAX;               // [token] largest gate score of the slice
+  float* c_sum = c_max + kBM;                      // [token] sum of exp(score - largest)
+  int* s_hist = reinterpret_cast<int*>(c_sum + kBM);
   uint64_t* bars = reinterpret_cast<uint64_t*>(s_hist + (P.n_routed + 3) / 4 * 4);
   uint64_t* full_bar = bars;                        // [stages] TMA -> MMA
   uint64_t* empty_bar = bars + kRtMaxStages;        // [stages] MMA -> TMA
@@ -111,9 +122,10 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const int tile = blockIdx.x / P.cs;
   const int row0 = tile * kBM;
-  const int kb0 = static_cast<int>(rank) * P.kb_per;
-  const int kb1 = min(P.num_kb, kb0 + P.kb_per);
-  const int nkb = kb1 > kb0 ? kb1 - kb0 : 0;
+  const int e0 = static_cast<int>(rank) * P.e_per;           // first expert of the slice
+  const int n_valid = max(0, min(P.e_per, P.n_routed - e0)); // experts of the slice
+  const int nkb = n_valid > 0 ? P.num_kb : 0;
+  const int k = P.top_k;
 
   pdl_launch_dependents();
   if (threadIdx.x == 0) {
@@ -158,13 +170,11 @@ __global__ void __launch_bounds__(kRtThreads, 1)
       if (lane == 0) {
         const uint32_t fb = smem_u32(&full_bar[s]);
         const uint32_t a_dst = smem_u32(ring + size_t(s) * P.stage_bytes);
-        const int k0 = (kb0 + it) * kBK;
+        const int k0 = it * kBK;
         mbar_arrive_expect_tx(fb, P.stage_bytes);
         tma_load_2d(a_dst, &tmX, fb, k0, row0);
-        for (int j = 0; j < P.nbox0; ++j)
-          tma_load_2d(a_dst + kATileBytes + j * box_bytes, &tmWg, fb, k0, j * P.box_rows);
-        for (int j = 0; j < P.nbox1; ++j)
-          tma_load_2d(a_dst + P.b_acc1_off + j * box_bytes, &tmWg, fb, k0, 256 + j * P.box_rows);
+        for (int j = 0; j < P.nbox; ++j)
+          tma_load_2d(a_dst + kATileBytes + j * box_bytes, &tmWg, fb, k0, e0 + j * P.box_rows);
       }
       __syncwarp();
       issued_mask |= 1u << s;
@@ -172,7 +182,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     }
     if (!ok && lane == 0) {
       // give the copies already issued a bounded chance to land before the
-      // ring is reused or the CTA exits
+      // CTA exits
       for (int i = 0; i < P.stages; ++i)
         if (issued_mask & (1u << i)) {
           int never = 0;
@@ -181,8 +191,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    const uint32_t idesc0 = idesc_bf16_f32(kBM, P.mma_n0);
-    const uint32_t idesc1 = idesc_bf16_f32(kBM, P.n_acc > 1 ? P.mma_n1 : 16);
+    const uint32_t idesc = idesc_bf16_f32(kBM, P.e_per);
     bool ok = true;
     for (int it = 0; it < nkb; ++it) {
       const int s = it % P.stages;
@@ -193,19 +202,12 @@ __global__ void __launch_bounds__(kRtThreads, 1)
       tc_fence_after_sync();
       if (lane == 0) {
         const uint32_t a_base = smem_u32(ring + size_t(s) * P.stage_bytes);
-        const uint32_t b0 = a_base + kATileBytes;
-        const uint32_t b1 = a_base + P.b_acc1_off;
+        const uint32_t b_base = a_base + kATileBytes;
 #pragma unroll
-        for (int k = 0; k < kBK / kUK; ++k)
-          umma_bf16(tmem_base, sdesc_kmajor_sw128(a_base + k * kUK * 2),
-                    sdesc_kmajor_sw128(b0 + k * kUK * 2), idesc0, (it > 0 || k > 0) ? 1u : 0u);
-        if (P.n_acc > 1) {
-#pragma unroll
-          for (int k = 0; k < kBK / kUK; ++k)
-            umma_bf16(tmem_base + 256, sdesc_kmajor_sw128(a_base + k * kUK * 2),
-                      sdesc_kmajor_sw128(b1 + k * kUK * 2), idesc1,
-                      (it > 0 || k > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < kBK / kUK; ++kk)
+          umma_bf16(tmem_base, sdesc_kmajor_sw128(a_base + kk * kUK * 2),
+                    sdesc_kmajor_sw128(b_base + kk * kUK * 2), idesc,
+                    (it > 0 || kk > 0) ? 1u : 0u);
         umma_commit(smem_u32(&empty_bar[s]));   // frees the stage when these MMAs finish
       }
       __syncwarp();
@@ -217,106 +219,192 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         int never = 0;
         mbar_wait(smem_u32(drain_bar), 0, &never);
       } else if (nkb > 0) {
-        umma_commit(smem_u32(tfull_bar));        // accumulators complete
+        umma_commit(smem_u32(tfull_bar));        // accumulator complete
       } else {
-        mbar_arrive(smem_u32(tfull_bar));        // no K blocks: nothing to wait for
+        mbar_arrive(smem_u32(tfull_bar));        // empty slice: nothing to wait for
       }
     }
     __syncwarp();
-  }
-  if (warp >= 4) {
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ slice statistics
+    // one thread per token of the tile (its TMEM lane): the slice's largest
+    // gate score, the sum of exp(score - largest), and its top-k candidates
     bool ok = mbar_wait(smem_u32(tfull_bar), 0, s_abort);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok && lane == 0) raise_timeout(s_abort, P.status);
     tc_fence_after_sync();
-  }
-
-  // ---------------------------------------------------------------- reduce
-  // Round a exchanges accumulator a (experts 256a .. 256a + ncols - 1). Each
-  // CTA first copies its 128 partial rows into its own exchange buffer (the
-  // stage ring, free once every MMA of this CTA has completed: the first barrier
-  // of round 0 follows the TMEM readers' wait; in round 1 it follows every
-  // CTA's reads of round 0), then every CTA reads its own tokens' rows from all
-  // CS buffers of the cluster and adds them in rank order.
-  const int own = P.own_rows;
-  for (int a = 0; a < P.n_acc; ++a) {
-    const int ncols = a ? P.ncols1 : P.ncols0;
-    const int xld = ncols + 4;      // row stride: 4 banks apart, conflict-free v4 stores
-    tc_fence_before_sync();
-    cluster_sync();
-    tc_fence_after_sync();
-    if (warp >= 4) {
-      const int q = warp & 3;
-      const int row = q * 32 + lane;                 // token row of the tile = TMEM lane
-      float* dst = reinterpret_cast<float*>(ring) + row * xld;
-      const bool have = nkb > 0 && *s_abort == 0;    // uniform over the CTA
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                             static_cast<uint32_t>(a * 256);
-      for (int c = 0; c < ncols; c += 32) {
-        uint32_t v[32];
-        if (have) {
-          tmem_ld_32cols(taddr + c, v);
-          tmem_ld_wait();
-        } else {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    const bool have = nkb > 0 && *s_abort == 0;    // uniform over the CTA
+    uint32_t ck[KMAX];
+    int ci[KMAX];
+    float cv[KMAX];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0u;
+    for (int j = 0; j < KMAX; ++j) {
+      ck[j] = 0u;
+      ci[j] = 0x7fffffff;
+      cv[j] = 0.0f;
+    }
+    uint32_t kth = 0u;   // key of the current k-th candidate (0 while fewer than k)
+    float lmax = -INFINITY;
+    // pass 1: the largest gate score
+    for (int c = 0; have && c < P.ncols; c += 32) {
+      uint32_t a[32];
+      tmem_ld_32cols(taddr + c, a);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (c + i < n_valid) {
+          const float raw = __uint_as_float(a[i]);
+          const float g = (P.bias && !P.bias_select_only) ? raw + __ldg(P.bias + e0 + c + i) : raw;
+          lmax = fmaxf(lmax, g);
         }
+    }
+    // pass 2: the sum of exponentials and the candidates, in ascending expert
+    // order (a later expert displaces a candidate only with a larger key, so
+    // equal keys keep the lower expert first)
+    float lsum = 0.0f;
+    for (int c = 0; have && c < P.ncols; c += 32) {
+      uint32_t a[32];
+      tmem_ld_32cols(taddr + c, a);
+      tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          *reinterpret_cast<uint4*>(dst + c + 4 * i) =
-              make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      for (int i = 0; i < 32; ++i) {
+        if (c + i >= n_valid) continue;
+        const int e = e0 + c + i;
+        const float raw = __uint_as_float(a[i]);
+        const float key = P.bias ? raw + __ldg(P.bias + e) : raw;
+        const float g = P.bias_select_only ? raw : key;
+        lsum += expf(g - lmax);
+        const uint32_t ok_ = order_key(key);
+        if (ok_ > kth) {
+          int pos = k - 1;
+#pragma unroll
+          for (int j = KMAX - 1; j >= 1; --j)
+            if (j <= k - 1 && ok_ > ck[j - 1]) {
+              ck[j] = ck[j - 1];
+              ci[j] = ci[j - 1];
+              cv[j] = cv[j - 1];
+              pos = j - 1;
+            }
+#pragma unroll
+          for (int j = 0; j < KMAX; ++j) {
+            if (j == pos) {
+              ck[j] = ok_;
+              ci[j] = e;
+              cv[j] = g;
+            }
+            if (j == k - 1) kth = ck[j];
+          }
+        }
       }
     }
-    cluster_sync();
-    // this CTA's tokens: the same rows of every CTA's buffer, added in rank order
-    const uint32_t xbase = smem_u32(ring);
-    const int n4 = ncols / 4;
-    for (int i = threadIdx.x; i < own * n4; i += kRtThreads) {
-      const int r = i / n4;
-      const int c = (i - r * n4) * 4;
-      const uint32_t off =
-          static_cast<uint32_t>(((static_cast<int>(rank) * own + r) * xld + c) * 4);
-      float4 part[kRtMaxCluster];
 #pragma unroll
-      for (int s = 0; s < kRtMaxCluster; ++s)
-        if (s < P.cs) part[s] = ld_cluster_f4(mapa_shared(xbase + off, static_cast<uint32_t>(s)));
-      float4 sum = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll
-      for (int s = 0; s < kRtMaxCluster; ++s)
-        if (s < P.cs) {
-          sum.x += part[s].x;
-          sum.y += part[s].y;
-          sum.z += part[s].z;
-          sum.w += part[s].w;
-        }
-      *reinterpret_cast<float4*>(s_scores + r * P.lds + a * 256 + c) = sum;
-    }
+    for (int j = 0; j < KMAX; ++j)
+      if (j < k) {
+        c_key[row * KMAX + j] = ck[j];
+        c_idx[row * KMAX + j] = ci[j];
+        c_val[row * KMAX + j] = cv[j];
+      }
+    c_max[row] = lmax;
+    c_sum[row] = lsum;
   }
-  // every CTA has read the cluster's buffers: the ring may be reused, and no
-  // CTA leaves while another can still read its shared memory
-  cluster_sync();
 
-  // ---------------------------------------------------------------- route
+  // ---------------------------------------------------------------- merge
+  // every CTA's candidates are written; one warp per token of this CTA gathers
+  // the CS slices' candidates (k each, sorted) and statistics
+  tc_fence_before_sync();
+  cluster_sync();
+  tc_fence_after_sync();
+  const int own = P.own_rows;
   const int tok0 = row0 + static_cast<int>(rank) * own;
   const int ntok = min(own, P.T - tok0);
+  const int n_cand = P.cs * k;                     // <= 8 * 16 = 128: <= 4 per lane
   for (int tl = warp; tl < ntok; tl += kRtThreads / 32) {
-    float v[NPL];
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      const int e = lane + 32 * i;
-      v[i] = e < P.n_routed ? s_scores[tl * P.lds + e] : 0.0f;
+    const int row = static_cast<int>(rank) * own + tl;   // row of the tile
+    // slice statistics: M = the largest gate score, S = the sum over all
+    // experts of exp(score - M), from each slice's (max, sum)
+    float sm = -INFINITY, ss = 0.0f;
+    if (lane < P.cs) {
+      sm = __uint_as_float(ld_cluster_u32(
+          mapa_shared(smem_u32(c_max + row), static_cast<uint32_t>(lane))));
+      ss = __uint_as_float(ld_cluster_u32(
+          mapa_shared(smem_u32(c_sum + row), static_cast<uint32_t>(lane))));
     }
-    int my_e;
-    float my_g;
-    route_token<NPL>(v, P.bias, P.n_routed, P.top_k, P.renorm, P.bias_select_only, lane, my_e,
-                     my_g);
-    if (lane < P.top_k) {
-      const long long o = static_cast<long long>(tok0 + tl) * P.top_k + lane;
+    float M = sm;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float S = lane < P.cs ? ss * expf(sm - M) : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+    // candidates: lane holds entries lane + 32*i of the (slice, slot) list
+    uint32_t okey[4];
+    int oidx[4];
+    float oval[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = lane + 32 * i;
+      okey[i] = 0u;
+      oidx[i] = 0x7fffffff;
+      oval[i] = 0.0f;
+      if (c < n_cand) {
+        const int src = c / k, slot = c - src * k;
+        const uint32_t off = static_cast<uint32_t>((row * KMAX + slot) * 4);
+        okey[i] = ld_cluster_u32(mapa_shared(smem_u32(c_key) + off, static_cast<uint32_t>(src)));
+        oidx[i] = static_cast<int>(
+            ld_cluster_u32(mapa_shared(smem_u32(c_idx) + off, static_cast<uint32_t>(src))));
+        oval[i] = __uint_as_float(
+            ld_cluster_u32(mapa_shared(smem_u32(c_val) + off, static_cast<uint32_t>(src))));
+      }
+    }
+    // k rounds of warp reductions: the largest key, then the lowest expert
+    // index holding it; each lane keeps its best untaken candidate
+    uint32_t taken = 0, lk = 0u;
+    int li = 0x7fffffff;
+    float lv = 0.0f;
+    auto rescan = [&]() {
+      lk = 0u;
+      li = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (!((taken >> i) & 1u) && (okey[i] > lk || (okey[i] == lk && oidx[i] < li))) {
+          lk = okey[i];
+          li = oidx[i];
+          lv = oval[i];
+        }
+    };
+    rescan();
+    float my_gw = 0.0f;
+    int my_e = -1;
+    for (int j = 0; j < k; ++j) {
+      const uint32_t gmax = __reduce_max_sync(0xffffffffu, lk);
+      const int be = static_cast<int>(
+          __reduce_min_sync(0xffffffffu, static_cast<unsigned>(lk == gmax ? li : 0x7fffffff)));
+      // the one lane holding the winner takes it and rescans
+      const unsigned holder = __ballot_sync(0xffffffffu, lk == gmax && li == be);
+      const int hl = __ffs(holder) - 1;
+      const float gw = __shfl_sync(0xffffffffu, lv, hl);
+      if (lane == j) { my_gw = gw; my_e = be; }
+      if (lane == hl) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (oidx[i] == be && !((taken >> i) & 1u)) taken |= 1u << i;
+        rescan();
+      }
+    }
+    const float my_p = lane < k ? expf(my_gw - M) / S : 0.0f;
+    float sel_sum = my_p;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sel_sum += __shfl_xor_sync(0xffffffffu, sel_sum, o);
+    if (lane < k) {
+      const long long o = static_cast<long long>(tok0 + tl) * k + lane;
       P.idx[o] = my_e;
-      P.gate[o] = my_g;
+      P.gate[o] = P.renorm ? my_p / sel_sum : my_p;
       atomicAdd(&s_hist[my_e], 1);
     }
   }
+
   // histograms: from the cluster's per-CTA counts, every CTA writes each
   // expert's pairs in lower-ranked CTAs of the tile (its offset inside the
   // tile) and the first CTA the tile's totals
@@ -329,8 +417,8 @@ __global__ void __launch_bounds__(kRtThreads, 1)
       for (int s2 = 0; s2 < P.cs; ++s2) {
         const int h = s2 == static_cast<int>(rank)
                           ? s_hist[e]
-                          : ld_cluster_s32(mapa_shared(hbase + static_cast<uint32_t>(e * 4),
-                                                       static_cast<uint32_t>(s2)));
+                          : static_cast<int>(ld_cluster_u32(mapa_shared(
+                                hbase + static_cast<uint32_t>(e * 4), static_cast<uint32_t>(s2))));
         pre += s2 < static_cast<int>(rank) ? h : 0;
         tot += h;
       }
@@ -338,7 +426,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
       if (rank == 0) P.tile_counts[static_cast<long long>(e) * P.n_chunks + tile] = tot;
     }
   }
-  // no CTA leaves while another can still read its histogram
+  // no CTA leaves while another can still read its shared memory
   cluster_sync();
 
   if (P.fold_scan && rank == 0) {
@@ -353,19 +441,19 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     if (*s_last) {
       __threadfence();
       for (int e = threadIdx.x; e < P.n_routed; e += kRtThreads) {
-        int* row = P.tile_counts + static_cast<long long>(e) * P.n_chunks;
+        int* rowp = P.tile_counts + static_cast<long long>(e) * P.n_chunks;
+        // all of the expert's tile counts are loaded before the first store
+        // (at most 64 tiles when the scan is folded)
+        int v[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) v[c] = c < P.n_chunks ? __ldcg(rowp + c) : 0;
         int run = 0;
-        for (int c0 = 0; c0 < P.n_chunks; c0 += 8) {
-          int v[8];
 #pragma unroll
-          for (int b = 0; b < 8; ++b) v[b] = c0 + b < P.n_chunks ? __ldcg(row + c0 + b) : 0;
-#pragma unroll
-          for (int b = 0; b < 8; ++b)
-            if (c0 + b < P.n_chunks) {
-              row[c0 + b] = run;
-              run += v[b];
-            }
-        }
+        for (int c = 0; c < 64; ++c)
+          if (c < P.n_chunks) {
+            rowp[c] = run;
+            run += v[c];
+          }
         P.counts[e] = run;
       }
       if (threadIdx.x == 0) *P.ticket = 0;

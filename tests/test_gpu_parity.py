@@ -97,21 +97,51 @@ NARROW_CASES = [
 
 @pytest.mark.parametrize("shape", NARROW_CASES, ids=[c.name for c in NARROW_CASES])
 def test_narrow_swiglu_tiles(shape):
+    # 64- or 128-column gate/up tiles, 64- or 128-row tiles of both routed GEMMs
     from mixture_experts_ffn_expert_b200.layer import MoELayer
     inp = make_layer_inputs(shape, seed=8, device="cuda")
     res = full_parity(inp, shape)        # default tile choice, against the oracle
     outs = {}
     for cols in (64, 128):
-        layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
-                         shape.renorm, inp, bias=inp["bias"], device="cuda",
-                         swiglu_tile_cols=cols)
-        outs[cols] = layer(inp["x"]).clone()
-        names = layer.plan.kernel_names()
-        assert ("grouped_gate_up[n64]" in names) == (cols == 64), names
+        for rows in (64, 128):
+            layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
+                             shape.renorm, inp, bias=inp["bias"], device="cuda",
+                             swiglu_tile_cols=cols, tile_rows=rows)
+            outs[cols, rows] = layer(inp["x"]).clone()
+            names = layer.plan.kernel_names()
+            gu = [n for n in names if n.startswith("grouped_gate_up")][0]
+            dn = [n for n in names if n.startswith("grouped_down")][0]
+            assert ("n64" in gu) == (cols == 64), names
+            assert ("m64" in gu) == (rows == 64) and ("m64" in dn) == (rows == 64), names
     torch.cuda.synchronize()
-    # every output element is the same sum in the same k order on both tile shapes
-    assert torch.equal(outs[64], outs[128])
+    # every output element is the same sum in the same k order on every tile shape
+    for key, out in outs.items():
+        assert torch.equal(out, outs[128, 128]), key
     del res
+
+
+INTERLEAVE_CASES = [
+    # skewed loads: a few experts with several 128-row m-blocks among many with one
+    LayerShape("interleave_zipf", 3000, 512, 256, 64, 6, 1, True, "zipf1.1"),
+    LayerShape("interleave_normal_bias", 2048, 256, 192, 32, 4, 0, False, "normal_var0.5"),
+]
+
+
+@pytest.mark.parametrize("shape", INTERLEAVE_CASES, ids=[c.name for c in INTERLEAVE_CASES])
+def test_interleaved_tile_order(shape):
+    # the same tiles in another order: the same bits, and parity with the oracle
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    inp = make_layer_inputs(shape, seed=17, device="cuda")
+    full_parity(inp, shape)
+    outs = []
+    for il in (0, 1):
+        layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
+                         shape.renorm, inp, bias=inp["bias"], device="cuda", interleave=il,
+                         tile_rows=128)
+        outs.append(layer(inp["x"]).clone())
+        torch.cuda.synchronize()
+        assert layer.device_status() == 0
+    assert torch.equal(outs[0], outs[1])
 
 
 PAIR_CASES = ["three_tokens", "ragged_17", "two_shared_raw", "ragged_tiles", "k_tail_not_64",
@@ -546,6 +576,34 @@ def test_bounded_wait_timeout_sets_status_and_context_recovers():
     assert layer.device_status() == 0          # reading clears it
     assert 1.5 < waited < 30.0, waited         # one bounded wait, not a hang
     again = layer(inp["x"])                    # the hook was one-shot
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    assert torch.equal(again, ref)
+
+
+def test_inconsistent_routing_state_is_reported_not_written_out_of_range():
+    # a workspace overwritten during a forward: the fused router's ticket (byte 64
+    # of the workspace, zero between forwards) is set to a value no forward
+    # reaches, so no cluster scans the tile histogram; the permutation kernel
+    # must find the totals inconsistent, drop every routed slot (the output is
+    # the shared expert alone), report MOE_DEVICE_INCONSISTENT, and the next
+    # forward must be clean again
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    shape = LayerShape("one_tile", 100, 256, 128, 24, 4, 1, True, "none")
+    inp = make_layer_inputs(shape, seed=31, device="cuda")
+    layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
+                     shape.renorm, inp, device="cuda")
+    ref = layer(inp["x"]).clone()
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    layer.workspace[64:68].view(torch.int32).fill_(1 << 20)
+    out = layer(inp["x"]).clone()
+    torch.cuda.synchronize()
+    assert layer.device_status() == 7               # MOE_DEVICE_INCONSISTENT
+    assert torch.isfinite(out).all()
+    shared_only = oracle_out(inp, shape, None, capacity=0)     # every routed slot dropped
+    check_output(to64(out), shared_only)
+    again = layer(inp["x"])
     torch.cuda.synchronize()
     assert layer.device_status() == 0
     assert torch.equal(again, ref)
