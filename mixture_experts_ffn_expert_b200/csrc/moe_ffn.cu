@@ -46,9 +46,11 @@ struct Layout {
       mtiles2, mtiles64, mt_hot, mt_cold, perm_src, inv_pos;
   size_t xperm, hidden, yrouted, hshared, yshared, total;
   int lds;            // row stride of the fp32 router scores
-  int tpc;            // tokens per routing chunk (a block of route_scatter)
-  int n_chunks;
-  int n_base;         // columns of chunk_counts: n_chunks, or the fused router's tiles
+  int tpc;            // tokens per block of route_scatter
+  int n_chunks;       // blocks of route_scatter
+  int sub_tokens;     // tokens per sub-chunk of the histogram (a multiple of tpc)
+  int n_base;         // columns of chunk_counts: one per group of subs_per_base sub-chunks
+  int subs_per_base;
   int router_splits;  // split-K factor of the router GEMM (partials summed by route_topk)
   int router_kb_per;  // k-blocks per split
   bool fused;         // router scores + softmax + top-k in one kernel (route_fused)
@@ -161,12 +163,15 @@ moe::RouterParams router_shape(const moe_plan* p, int64_t T, size_t* smem) {
   if (stages > r.num_kb) stages = r.num_kb;
   stages = stages < 2 ? 2 : (stages > moe::kRtMaxStages ? moe::kRtMaxStages : stages);
   r.stages = stages;
-  r.ring_bytes = up(stages * r.stage_bytes, 1024);
+  // the ring also holds the statistics phase's scratch once the scores are done
+  const int scratch = static_cast<int>(moe::router_scratch_bytes());
+  const int ring = stages * r.stage_bytes;
+  r.ring_bytes = up(ring > scratch ? ring : scratch, 1024);
   int cols = 32;
   while (cols < r.ncols) cols *= 2;
   r.tmem_cols = cols;
   // fold the tile scan into the router's last cluster while there are few
-  // tiles (one thread per expert walks them)
+  // tiles (one warp per expert walks them)
   r.fold_scan = r.n_chunks <= 64 ? 1 : 0;
   // at least kRouterMinSmem so that two router CTAs never share an SM: each
   // allocates tensor memory and then waits at cluster barriers, and two
@@ -186,11 +191,16 @@ Layout make_layout(const moe_plan* p, int64_t T) {
   L.lds = static_cast<int>(align_up(p->n_routed, 8));
   if (L.fused) {
     // the router's histogram has one column per 128-token tile, plus each CTA's
-    // offsets inside its tile: route_scatter's chunks are the CTAs' token ranges
+    // offsets inside its tile (sub-chunks of 128/CS tokens); route_scatter's
+    // blocks take 8..128/CS tokens, about two blocks per SM
     L.rt = router_shape(p, T, &L.rt_smem);
-    L.tpc = L.rt.own_rows;
-    L.n_chunks = L.rt.n_chunks * L.rt.cs;
+    L.sub_tokens = L.rt.own_rows;
+    L.subs_per_base = L.rt.cs;
     L.n_base = L.rt.n_chunks;
+    int tpc = 8;
+    while (tpc < L.sub_tokens && static_cast<int64_t>(tpc) * 2 * p->num_sms < T) tpc *= 2;
+    L.tpc = tpc;
+    L.n_chunks = static_cast<int>((T + tpc - 1) / tpc);
     L.router_splits = 0;
     L.router_kb_per = 0;
   } else {
@@ -199,6 +209,8 @@ Layout make_layout(const moe_plan* p, int64_t T) {
     tpc = tpc < 8 ? 8 : (tpc > 128 ? 128 : tpc);
     L.tpc = static_cast<int>(tpc);
     L.n_chunks = static_cast<int>((T + tpc - 1) / tpc);
+    L.sub_tokens = L.tpc;
+    L.subs_per_base = 1;
     L.n_base = L.n_chunks;
     // split-K of the router GEMM so that it occupies most SMs even for few tokens
     const int64_t tiles = ((T + moe::kBM - 1) / moe::kBM) * ((p->n_routed + moe::kBN - 1) / moe::kBN);
@@ -220,7 +232,8 @@ Layout make_layout(const moe_plan* p, int64_t T) {
   L.idx = take(size_t(A) * 4);
   L.gate = take(size_t(A) * 4);
   L.chunk_counts = take(size_t(p->n_routed) * (L.n_base > 0 ? L.n_base : 1) * 4);
-  L.sub_base = take(L.fused ? size_t(p->n_routed) * (L.n_chunks > 0 ? L.n_chunks : 1) * 4 : 0);
+  L.sub_base = take(L.fused ? size_t(p->n_routed) * (L.n_base > 0 ? L.n_base : 1) * L.subs_per_base * 4
+                            : 0);
   L.counts = take(size_t(p->n_routed) * 4);
   L.offsets = take(size_t(p->n_routed + 1) * 4);
   L.mtiles = take(size_t(p->n_routed + 1) * 4);
@@ -926,8 +939,8 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     if (slices < 1) slices = 1;
     L.begin("route_scatter", main_st);
     launch_pdl(moe::route_scatter_kernel, dim3(Lw.n_chunks, slices), dim3(moe::kRouteThreads), smem,
-               main_st, (const int*)idx, (const int*)chunk_counts, (const int*)sub_base,
-               Lw.n_chunks / Lw.n_base, (const int*)counts,
+               main_st, (const int*)idx, (const int*)chunk_counts, Lw.n_base,
+               (const int*)sub_base, Lw.subs_per_base, Lw.sub_tokens, (const int*)counts,
                static_cast<int>(T), k, nr, Lw.tpc, Lw.n_chunks, moe::kBM, seat_limit,
                reinterpret_cast<const uint4*>(x), d / 8, reinterpret_cast<uint4*>(xperm),
                perm_src, inv_pos, offsets, mtiles, mtiles2, mtiles64, mt_hot, mt_cold, status);

@@ -290,9 +290,9 @@ constexpr int kCopyUnroll = 4;
 
 __global__ void __launch_bounds__(kRouteThreads)
     route_scatter_kernel(const int* __restrict__ idx, const int* __restrict__ chunk_base,
-                         const int* __restrict__ sub_base, int chunks_per_base,
-                         const int* __restrict__ counts, int T, int top_k, int n_routed,
-                         int tpc, int n_chunks, int tile_rows, int capacity,
+                         int n_base, const int* __restrict__ sub_base, int subs_per_base,
+                         int sub_tokens, const int* __restrict__ counts, int T, int top_k,
+                         int n_routed, int tpc, int n_chunks, int tile_rows, int capacity,
                          const uint4* __restrict__ x,
                          int d_vec, uint4* __restrict__ xperm, int* __restrict__ perm_src,
                          int* __restrict__ inv_pos, int* __restrict__ offsets_out,
@@ -312,15 +312,26 @@ __global__ void __launch_bounds__(kRouteThreads)
   const int ntok = max(0, min(tpc, T - t0));   // the last tile's chunks may hold no token
   const int n_ent = ntok * top_k;
   const long long ebase = static_cast<long long>(t0) * top_k;
-  // the chunk's base inside each expert's group: one level (chunk_base
-  // [N_r][n_chunks]) or two (chunk_base [N_r][n_chunks / chunks_per_base] per
-  // group of chunks, plus sub_base [N_r][n_chunks] inside the group)
-  const int n_base = n_chunks / chunks_per_base;
+  // The block's base inside each expert's group. The histogram it comes from
+  // counts pairs per sub-chunk of sub_tokens tokens (a multiple of tpc):
+  // chunk_base [N_r][n_base] holds the prefix at each group of subs_per_base
+  // sub-chunks and, with two levels, sub_base [N_r][n_base * subs_per_base]
+  // the pairs of the sub-chunks before it in its group; the pairs of the
+  // sub-chunk's own tokens before this block are counted here.
+  const int sub = t0 / sub_tokens;
+  const int grp = sub / subs_per_base;
+  const int pre_tokens = t0 - sub * sub_tokens;
+  // (an expert index out of range - a router that gave up - gets a negative
+  // place, so the entry is reported and dropped below)
   for (int i = threadIdx.x; i < n_ent; i += blockDim.x) {
     const int e = idx[ebase + i];
-    s_e[i] = e;
-    int b = chunk_base[static_cast<long long>(e) * n_base + chunk / chunks_per_base];
-    if (sub_base) b += sub_base[static_cast<long long>(e) * n_chunks + chunk];
+    const bool in_range = static_cast<unsigned>(e) < static_cast<unsigned>(n_routed);
+    s_e[i] = in_range ? e : 0;
+    int b = -(1 << 30);
+    if (in_range) {
+      b = chunk_base[static_cast<long long>(e) * n_base + grp];
+      if (sub_base) b += sub_base[static_cast<long long>(e) * (n_base * subs_per_base) + sub];
+    }
     s_pos[i] = b;
   }
   // an expert keeps at most `capacity` rows: its first pairs in (token, slot) order
@@ -378,6 +389,21 @@ __global__ void __launch_bounds__(kRouteThreads)
     }
     __syncthreads();
   }
+
+  if (pre_tokens > 0 && !bad) {
+    // pairs of this sub-chunk routed before this block's tokens, per expert
+    const long long pbase = static_cast<long long>(t0 - pre_tokens) * top_k;
+    __syncthreads();
+    for (int i = threadIdx.x; i < pre_tokens * top_k; i += blockDim.x) {
+      const int e = idx[pbase + i];
+      if (static_cast<unsigned>(e) < static_cast<unsigned>(n_routed)) atomicAdd(&s_run[e], 1);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < n_ent; i += blockDim.x) s_pos[i] += s_run[s_e[i]];
+    __syncthreads();
+    for (int e = threadIdx.x; e < n_routed; e += blockDim.x) s_run[e] = 0;
+  }
+  __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0) {

@@ -9,20 +9,27 @@
 //
 // Design (sm_100a, N_r <= 512, top_k <= 16):
 //  * a cluster of CS CTAs (CS <= 8) owns one 128-token tile; CTA r computes the
-//    scores of its slice of E = N_r/CS experts over the whole K range (one
-//    TMEM accumulator of <= 256 columns), so no partial sums are exchanged;
+//    scores of its slice of E = N_r/CS <= 64 experts over the whole K range
+//    (one TMEM accumulator), so no partial sums are exchanged;
 //  * warp 0 loads A (x rows, one 128x64 box) and B (the slice's W_g rows, boxes
 //    of up to 128 rows) per 64-wide K block through TMA (no multicast); warp 1
 //    issues tcgen05.mma M=128, N=E;
-//  * warps 4..7 read the accumulator, one thread per token (its TMEM lane): the
-//    slice's softmax statistics (its largest gate score and the sum of
-//    exp(score - largest)) and its top-k candidates (selection key, expert, gate
-//    score), kept sorted in registers - all 128 tokens of the tile at once;
-//  * after a cluster barrier, one warp per token of this CTA's 128/CS tokens
-//    gathers the CS slices' candidates and statistics through distributed
-//    shared memory and selects the top k among them with warp reductions
-//    (largest key, then lowest index: ties to the lower expert index); the
-//    softmax over all N_r experts follows from the statistics;
+//  * all 16 warps copy the accumulator to shared memory; then one warp per
+//    token (lanes over the slice's experts) takes the slice's softmax
+//    statistics (the largest gate score and the sum of exp(score - largest))
+//    and its top-k candidates (selection key, expert, gate score) in k rounds
+//    of two warp reductions;
+//  * with one slice (CS = 1) these are the token's top k and softmax and the
+//    warp writes the gates itself; otherwise lane j stores candidate j, and
+//    lane 0 the statistics, into the shared memory of the CTA that routes the
+//    token (CTA m / (128/CS) for token m of the tile) through distributed
+//    shared memory, and after a cluster barrier one warp per token of this
+//    CTA's 128/CS tokens selects the top k of the CS * k candidates (largest
+//    key, ties to the lower expert index); the softmax over all N_r experts
+//    follows from the slices' statistics;
+//  * every loop over tokens or columns stays rolled: each CTA runs the code
+//    about once, so its length (instruction fetch), not its arithmetic, sets
+//    the time;
 //  * a shared histogram per CTA; reading the cluster's histograms, each CTA
 //    writes its experts' offsets inside the tile and the first CTA the tile's
 //    totals, one column of the tile histogram.
@@ -64,11 +71,20 @@ struct RouterParams {
   int* status;           // device status word
 };
 
-// Shared memory of the candidates: KMAX per token of the tile (top_k <= KMAX)
-// as (key, expert, gate score), plus the token's (max, sum) statistics.
+// Shared memory of the candidates a CTA receives: for each of the CS slices and
+// each of its 128/CS tokens (128 rows in all), KMAX candidates (top_k <= KMAX)
+// as (key, expert, gate score), plus the slice's (max, sum) statistics.
 template <int KMAX>
 __host__ __device__ constexpr size_t router_cand_bytes() {
   return size_t(kBM) * KMAX * 12 + size_t(kBM) * 8;
+}
+
+constexpr int kRtMaxSliceCols = 64;   // accumulator columns of one slice
+
+// Scratch laid over the ring once the scores are complete: the slice's scores
+// [token][ncols + 1] in fp32.
+__host__ __device__ constexpr size_t router_scratch_bytes() {
+  return size_t(kBM) * (kRtMaxSliceCols + 1) * 4;
 }
 
 // Dynamic shared memory of a launch: ring, candidates, histogram, barriers.
@@ -76,6 +92,10 @@ template <int KMAX>
 __host__ __device__ constexpr size_t router_smem_bytes(int ring_bytes, int n_routed) {
   return 1024 + size_t(ring_bytes) + router_cand_bytes<KMAX>() +
          size_t((n_routed + 3) / 4 * 4) * 4 + 256;
+}
+
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
@@ -94,6 +114,101 @@ __device__ __forceinline__ uint32_t order_key(float k) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// k rounds of selection over the warp's candidates (lane l holds key[i],
+// expert[i], gate score[i] for i < N; key 0 marks an empty one): each round
+// takes the largest key and, among equal keys, the lowest expert (two warp
+// reductions); only the winning lane rescans its own. Lane j < k receives the
+// j-th winner's key, expert and gate score.
+template <int N>
+__device__ __forceinline__ void select_rounds(const uint32_t (&key)[N], const int (&ex)[N],
+                                              const float (&val)[N], int k, int lane,
+                                              uint32_t& my_k, int& my_e, float& my_g) {
+  uint32_t taken = 0;
+  uint32_t lk = 0u;
+  int li = 0x7fffffff, slot = 0;
+  auto rescan = [&]() {
+    lk = 0u;
+    li = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if (!((taken >> i) & 1u) && (key[i] > lk || (key[i] == lk && key[i] != 0u && ex[i] < li))) {
+        lk = key[i];
+        li = ex[i];
+        slot = i;
+      }
+  };
+  rescan();
+  my_k = 0u;
+  my_e = 0x7fffffff;
+  my_g = 0.0f;
+#pragma unroll 1
+  for (int j = 0; j < k; ++j) {
+    const uint32_t gmax = __reduce_max_sync(0xffffffffu, lk);
+    const unsigned be =
+        __reduce_min_sync(0xffffffffu, static_cast<unsigned>(lk == gmax ? li : 0x7fffffff));
+    const bool win = lk == gmax && static_cast<unsigned>(li) == be;
+    const unsigned wmask = __ballot_sync(0xffffffffu, win);
+    const int wl = wmask ? __ffs(wmask) - 1 : 0;   // one lane holds the winner
+    float wv = 0.0f;
+#pragma unroll
+    for (int i = 0; i < N; ++i) wv = i == slot ? val[i] : wv;
+    wv = __shfl_sync(0xffffffffu, wv, wl);
+    if (lane == j) {
+      my_k = gmax;
+      my_e = static_cast<int>(be);
+      my_g = wv;
+    }
+    if (lane == wl && wmask) {
+      taken |= 1u << slot;
+      rescan();
+    }
+  }
+}
+
+// One warp, one token, one slice: lane l holds the slice's experts e0 + l and
+// e0 + l + 32 (n_valid of them are experts). Returns to every lane the slice's
+// largest gate score m and sum of exp(score - m) (0 for an empty slice), and
+// to lane j < k the j-th candidate by selection key (ties to the lower expert)
+// as (key, expert, gate score); key 0 where the slice has fewer than k experts.
+__device__ __forceinline__ void slice_select(const float* srow, int n_valid, int e0,
+                                             const float* __restrict__ bias, int bias_select_only,
+                                             int k, int lane, float& m, float& sum,
+                                             uint32_t& my_key, int& my_e, float& my_g) {
+  uint32_t key[2];
+  int ex[2];
+  float g[2];
+  m = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int c = lane + 32 * i;
+    const bool v = c < n_valid;
+    const float raw = v ? srow[c] : 0.0f;
+    const float kv = (v && bias) ? raw + __ldg(bias + e0 + c) : raw;
+    g[i] = bias_select_only ? raw : kv;
+    key[i] = v ? order_key(kv) : 0u;
+    ex[i] = v ? e0 + c : 0x7fffffff;
+    if (v) m = fmaxf(m, g[i]);
+  }
+  m = warp_max(m);
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    if (lane + 32 * i < n_valid) s += expf(g[i] - m);
+  sum = warp_sum(s);
+  select_rounds<2>(key, ex, g, k, lane, my_key, my_e, my_g);
+}
+
 template <int KMAX>
 __global__ void __launch_bounds__(kRtThreads, 1)
     route_fused_kernel(const __grid_constant__ CUtensorMap tmX,
@@ -101,12 +216,12 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  // candidates of the 128 tokens of the tile from this CTA's slice, [token][slot]
+  // candidates received for this CTA's tokens, [slice * own + token][slot]
   uint32_t* c_key = reinterpret_cast<uint32_t*>(ring + P.ring_bytes);
   int* c_idx = reinterpret_cast<int*>(c_key + kBM * KMAX);
   float* c_val = reinterpret_cast<float*>(c_idx + kBM * KMAX);
-  float* c_max = c_val + kBM * KMAX;               // [token] largest gate score of the slice
-  float* c_sum = c_max + kBM;                      // [token] sum of exp(score - largest)
+  float* c_max = c_val + kBM * KMAX;               // [slice * own + token] largest gate score
+  float* c_sum = c_max + kBM;                      // [slice * own + token] sum of exp(score - largest)
   int* s_hist = reinterpret_cast<int*>(c_sum + kBM);
   uint64_t* bars = reinterpret_cast<uint64_t*>(s_hist + (P.n_routed + 3) / 4 * 4);
   uint64_t* full_bar = bars;                        // [stages] TMA -> MMA
@@ -225,189 +340,136 @@ __global__ void __launch_bounds__(kRtThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ slice statistics
-    // one thread per token of the tile (its TMEM lane): the slice's largest
-    // gate score, the sum of exp(score - largest), and its top-k candidates
+  }
+
+  // ---------------------------------------------------------------- scores to shared memory
+  // every warp copies a quarter of the slice's columns of one TMEM lane
+  // quarter (warps w, w+4, w+8, w+12 share lanes 32*(w%4)..) into the score
+  // rows [token][ncols + 1] laid over the ring (every MMA has completed, so
+  // every stage has been read)
+  float* s_score = reinterpret_cast<float*>(ring);
+  const int lds = P.ncols + 1;   // odd stride: the 32 rows of a warp's stores hit 32 banks
+  {
     bool ok = mbar_wait(smem_u32(tfull_bar), 0, s_abort);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok && lane == 0) raise_timeout(s_abort, P.status);
     tc_fence_after_sync();
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    const int cpp = P.ncols / 4;                  // a multiple of 8
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    const bool have = nkb > 0 && *s_abort == 0;    // uniform over the CTA
-    uint32_t ck[KMAX];
-    int ci[KMAX];
-    float cv[KMAX];
+    if (nkb > 0 && ok) {
+#pragma unroll 1
+      for (int c = (warp >> 2) * cpp; c < ((warp >> 2) + 1) * cpp; c += 8) {
+        uint32_t a[8];
+        tmem_ld_8cols(taddr + c, a);
+        tmem_ld_wait();
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      ck[j] = 0u;
-      ci[j] = 0x7fffffff;
-      cv[j] = 0.0f;
+        for (int i = 0; i < 8; ++i) s_score[row * lds + c + i] = __uint_as_float(a[i]);
+      }
     }
-    uint32_t kth = 0u;   // key of the current k-th candidate (0 while fewer than k)
-    float lmax = -INFINITY;
-    // pass 1: the largest gate score
-    for (int c = 0; have && c < P.ncols; c += 32) {
-      uint32_t a[32];
-      tmem_ld_32cols(taddr + c, a);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (c + i < n_valid) {
-          const float raw = __uint_as_float(a[i]);
-          const float g = (P.bias && !P.bias_select_only) ? raw + __ldg(P.bias + e0 + c + i) : raw;
-          lmax = fmaxf(lmax, g);
+  }
+  __syncthreads();
+
+  // ---------------------------------------------------------------- slice top-k
+  // one warp per token (lane l holds the slice's experts l and l + 32): the
+  // slice's largest gate score and sum of exp(score - largest), and its top-k
+  // by selection key with ties to the lower expert; lane j ends with the j-th
+  {
+    const bool have = nkb > 0 && *s_abort == 0;
+    const int own_r = P.own_rows;
+#pragma unroll 1
+    for (int row = warp; row < kBM; row += kRtThreads / 32) {
+      float m, sum;
+      uint32_t my_key;
+      int my_e;
+      float my_g;
+      slice_select(s_score + row * lds, have ? n_valid : 0, e0, P.bias, P.bias_select_only,
+                   k, lane, m, sum, my_key, my_e, my_g);
+      if (P.cs == 1) {
+        // one slice holds every expert: the token's softmax and top k
+        const int t = row0 + row;
+        const float my_p = lane < k ? expf(my_g - m) / sum : 0.0f;
+        const float sel = warp_sum(my_p);
+        if (t < P.T && lane < k) {
+          const long long o = static_cast<long long>(t) * k + lane;
+          P.idx[o] = my_e;
+          P.gate[o] = P.renorm ? my_p / sel : my_p;
+          if (static_cast<unsigned>(my_e) < static_cast<unsigned>(P.n_routed))
+            atomicAdd(&s_hist[my_e], 1);
         }
-    }
-    // pass 2: the sum of exponentials and the candidates, in ascending expert
-    // order (a later expert displaces a candidate only with a larger key, so
-    // equal keys keep the lower expert first)
-    float lsum = 0.0f;
-    for (int c = 0; have && c < P.ncols; c += 32) {
-      uint32_t a[32];
-      tmem_ld_32cols(taddr + c, a);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        if (c + i >= n_valid) continue;
-        const int e = e0 + c + i;
-        const float raw = __uint_as_float(a[i]);
-        const float key = P.bias ? raw + __ldg(P.bias + e) : raw;
-        const float g = P.bias_select_only ? raw : key;
-        lsum += expf(g - lmax);
-        const uint32_t ok_ = order_key(key);
-        if (ok_ > kth) {
-          int pos = k - 1;
-#pragma unroll
-          for (int j = KMAX - 1; j >= 1; --j)
-            if (j <= k - 1 && ok_ > ck[j - 1]) {
-              ck[j] = ck[j - 1];
-              ci[j] = ci[j - 1];
-              cv[j] = cv[j - 1];
-              pos = j - 1;
-            }
-#pragma unroll
-          for (int j = 0; j < KMAX; ++j) {
-            if (j == pos) {
-              ck[j] = ok_;
-              ci[j] = e;
-              cv[j] = g;
-            }
-            if (j == k - 1) kth = ck[j];
-          }
+      } else {
+        // to the CTA that routes this token: slot (this slice, token) of its buffers
+        const uint32_t owner = static_cast<uint32_t>(row / own_r);
+        const int slot_row =
+            static_cast<int>(rank) * own_r + (row - static_cast<int>(owner) * own_r);
+        if (lane < k) {
+          st_cluster_u32(mapa_shared(smem_u32(c_key + slot_row * KMAX + lane), owner), my_key);
+          st_cluster_u32(mapa_shared(smem_u32(c_idx + slot_row * KMAX + lane), owner),
+                         static_cast<uint32_t>(my_e));
+          st_cluster_u32(mapa_shared(smem_u32(c_val + slot_row * KMAX + lane), owner),
+                         __float_as_uint(my_g));
+        }
+        if (lane == 0) {
+          st_cluster_u32(mapa_shared(smem_u32(c_max + slot_row), owner), __float_as_uint(m));
+          st_cluster_u32(mapa_shared(smem_u32(c_sum + slot_row), owner), __float_as_uint(sum));
         }
       }
     }
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j)
-      if (j < k) {
-        c_key[row * KMAX + j] = ck[j];
-        c_idx[row * KMAX + j] = ci[j];
-        c_val[row * KMAX + j] = cv[j];
-      }
-    c_max[row] = lmax;
-    c_sum[row] = lsum;
   }
 
   // ---------------------------------------------------------------- merge
-  // every CTA's candidates are written; one warp per token of this CTA gathers
-  // the CS slices' candidates (k each, sorted) and statistics
+  // every slice's candidates have arrived; one warp per token of this CTA
+  // selects the top k of the CS * k candidates (largest key, ties to the lower
+  // expert index); the softmax over all N_r experts follows from the slices'
+  // (max, sum)
   tc_fence_before_sync();
+  __syncthreads();
   cluster_sync();
   tc_fence_after_sync();
-  const int own = P.own_rows;
-  const int tok0 = row0 + static_cast<int>(rank) * own;
-  const int ntok = min(own, P.T - tok0);
-  const int n_cand = P.cs * k;                     // <= 8 * 16 = 128: <= 4 per lane
-  for (int tl = warp; tl < ntok; tl += kRtThreads / 32) {
-    const int row = static_cast<int>(rank) * own + tl;   // row of the tile
-    // slice statistics: M = the largest gate score, S = the sum over all
-    // experts of exp(score - M), from each slice's (max, sum)
-    float sm = -INFINITY, ss = 0.0f;
-    if (lane < P.cs) {
-      sm = __uint_as_float(ld_cluster_u32(
-          mapa_shared(smem_u32(c_max + row), static_cast<uint32_t>(lane))));
-      ss = __uint_as_float(ld_cluster_u32(
-          mapa_shared(smem_u32(c_sum + row), static_cast<uint32_t>(lane))));
-    }
-    float M = sm;
+  if (P.cs > 1) {
+    const int own = P.own_rows;
+    const int tok0 = row0 + static_cast<int>(rank) * own;
+    const int ntok = min(own, P.T - tok0);
+    const int n_c = P.cs * k;                    // candidates of a token (<= 128)
+#pragma unroll 1
+    for (int tl = warp; tl < ntok; tl += kRtThreads / 32) {
+      const float sm = lane < P.cs ? c_max[lane * own + tl] : -INFINITY;
+      const float M = warp_max(sm);
+      const float ss = lane < P.cs ? c_sum[lane * own + tl] : 0.0f;
+      const float S = warp_sum(ss > 0.0f ? ss * expf(sm - M) : 0.0f);
+      uint32_t ck[4];
+      int ci[4];
+      float cv[4];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float S = lane < P.cs ? ss * expf(sm - M) : 0.0f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
-    // candidates: lane holds entries lane + 32*i of the (slice, slot) list
-    uint32_t okey[4];
-    int oidx[4];
-    float oval[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int c = lane + 32 * i;
-      okey[i] = 0u;
-      oidx[i] = 0x7fffffff;
-      oval[i] = 0.0f;
-      if (c < n_cand) {
-        const int src = c / k, slot = c - src * k;
-        const uint32_t off = static_cast<uint32_t>((row * KMAX + slot) * 4);
-        okey[i] = ld_cluster_u32(mapa_shared(smem_u32(c_key) + off, static_cast<uint32_t>(src)));
-        oidx[i] = static_cast<int>(
-            ld_cluster_u32(mapa_shared(smem_u32(c_idx) + off, static_cast<uint32_t>(src))));
-        oval[i] = __uint_as_float(
-            ld_cluster_u32(mapa_shared(smem_u32(c_val) + off, static_cast<uint32_t>(src))));
+      for (int i = 0; i < 4; ++i) {
+        const int qq = lane + 32 * i;             // candidate (slice qq / k, slot qq % k)
+        const int sl = qq / k;
+        const int at = (sl * own + tl) * KMAX + (qq - sl * k);
+        ck[i] = qq < n_c ? c_key[at] : 0u;
+        ci[i] = qq < n_c ? c_idx[at] : 0x7fffffff;
+        cv[i] = qq < n_c ? c_val[at] : 0.0f;
       }
-    }
-    // k rounds of warp reductions: the largest key, then the lowest expert
-    // index holding it; each lane keeps its best untaken candidate
-    uint32_t taken = 0, lk = 0u;
-    int li = 0x7fffffff;
-    float lv = 0.0f;
-    auto rescan = [&]() {
-      lk = 0u;
-      li = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (!((taken >> i) & 1u) && (okey[i] > lk || (okey[i] == lk && oidx[i] < li))) {
-          lk = okey[i];
-          li = oidx[i];
-          lv = oval[i];
-        }
-    };
-    rescan();
-    float my_gw = 0.0f;
-    int my_e = -1;
-    for (int j = 0; j < k; ++j) {
-      const uint32_t gmax = __reduce_max_sync(0xffffffffu, lk);
-      const int be = static_cast<int>(
-          __reduce_min_sync(0xffffffffu, static_cast<unsigned>(lk == gmax ? li : 0x7fffffff)));
-      // the one lane holding the winner takes it and rescans
-      const unsigned holder = __ballot_sync(0xffffffffu, lk == gmax && li == be);
-      const int hl = __ffs(holder) - 1;
-      const float gw = __shfl_sync(0xffffffffu, lv, hl);
-      if (lane == j) { my_gw = gw; my_e = be; }
-      if (lane == hl) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (oidx[i] == be && !((taken >> i) & 1u)) taken |= 1u << i;
-        rescan();
+      uint32_t my_k;
+      int my_e;
+      float my_g;
+      select_rounds<4>(ck, ci, cv, k, lane, my_k, my_e, my_g);
+      const float my_p = lane < k ? expf(my_g - M) / S : 0.0f;
+      const float sel = warp_sum(my_p);
+      if (lane < k) {
+        const long long o = static_cast<long long>(tok0 + tl) * k + lane;
+        P.idx[o] = my_e;
+        P.gate[o] = P.renorm ? my_p / sel : my_p;
+        if (static_cast<unsigned>(my_e) < static_cast<unsigned>(P.n_routed))
+          atomicAdd(&s_hist[my_e], 1);
       }
-    }
-    const float my_p = lane < k ? expf(my_gw - M) / S : 0.0f;
-    float sel_sum = my_p;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sel_sum += __shfl_xor_sync(0xffffffffu, sel_sum, o);
-    if (lane < k) {
-      const long long o = static_cast<long long>(tok0 + tl) * k + lane;
-      P.idx[o] = my_e;
-      P.gate[o] = P.renorm ? my_p / sel_sum : my_p;
-      atomicAdd(&s_hist[my_e], 1);
     }
   }
 
   // histograms: from the cluster's per-CTA counts, every CTA writes each
   // expert's pairs in lower-ranked CTAs of the tile (its offset inside the
   // tile) and the first CTA the tile's totals
+  __syncthreads();
   cluster_sync();
   {
     const uint32_t hbase = smem_u32(s_hist);
@@ -440,21 +502,12 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     __syncthreads();
     if (*s_last) {
       __threadfence();
-      for (int e = threadIdx.x; e < P.n_routed; e += kRtThreads) {
-        int* rowp = P.tile_counts + static_cast<long long>(e) * P.n_chunks;
-        // all of the expert's tile counts are loaded before the first store
-        // (at most 64 tiles when the scan is folded)
-        int v[64];
-#pragma unroll
-        for (int c = 0; c < 64; ++c) v[c] = c < P.n_chunks ? __ldcg(rowp + c) : 0;
-        int run = 0;
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c < P.n_chunks) {
-            rowp[c] = run;
-            run += v[c];
-          }
-        P.counts[e] = run;
+      // one warp per expert (other clusters' counts: read through L2)
+#pragma unroll 1
+      for (int e = warp; e < P.n_routed; e += kRtThreads / 32) {
+        const int tot = scan_expert_chunks<true>(
+            P.tile_counts + static_cast<long long>(e) * P.n_chunks, P.n_chunks, lane);
+        if (lane == 0) P.counts[e] = tot;
       }
       if (threadIdx.x == 0) *P.ticket = 0;
     }
