@@ -124,10 +124,14 @@ int moe_last_status(void);
  *   softmax + top-k); 0 always uses the two-kernel router; 1 is the same as -1.
  *   Both give the same selection up to fp32 rounding of the scores.
  * MOE_OPTION_SWIGLU_TILE_COLS: output columns of one tile of the routed
- *   gate/up GEMM when it runs one CTA per tile: 0 (default) chooses 64 when the
+ *   gate/up GEMM when it runs one CTA per tile: 0 (default) chooses, when the
  *   expected rows per expert (T*top_k/N_r) are below 32 - the weight-streaming
- *   decode regime, where twice as many, shorter tiles leave a shorter last
- *   wave - and 128 otherwise; 64 or 128 force it.
+ *   decode regime, where more, shorter tiles leave a shorter last wave - 32
+ *   with two CTAs per SM and 64 with one, and 128 otherwise; 32, 64 or 128
+ *   force it.
+ * MOE_OPTION_DOWN_TILE_COLS: output columns of one tile of the routed down
+ *   GEMM when it runs one CTA per tile: 0 (default) chooses 128 in the
+ *   weight-streaming regime with two CTAs per SM, else 256; 128 or 256 force it.
  * MOE_OPTION_TILE_ROWS: rows of one tile of the routed GEMMs when they run
  *   one CTA per tile: 0 (default) chooses 64 when the expected rows per expert
  *   are below 32 (M=64 MMAs and 64-row boxes of the grouped rows: smaller
@@ -144,6 +148,12 @@ int moe_last_status(void);
  *   few SMs (the routed GEMMs keep the rest); -1 (default) and 0: after them on
  *   the caller's stream (measured faster on B200 for the DeepSeek-V3 layer
  *   shape). Small shared experts always run beside the routing kernels.
+ * MOE_OPTION_CTAS_PER_SM: CTAs per SM of the routed GEMMs when they run one
+ *   CTA per tile. 2: two resident CTAs per SM, each with half the pipeline
+ *   ring and half the tensor memory (two independent load pipelines per SM,
+ *   which stream weights faster); 1: one CTA per SM with the whole ring;
+ *   0 (default): 2 when the expected rows per expert are below 32 (weight
+ *   streaming), else 1.
  * MOE_OPTION_TEST_WAIT_TIMEOUT: test hook for the failure path, not for normal
  *   use. Value 1 arms it for the next forward only: if that forward runs the
  *   routed gate/up GEMM on the one-CTA-per-tile kernel, one CTA withholds the
@@ -163,6 +173,8 @@ enum {
   MOE_OPTION_SHARED_CONCURRENT = 9,
   MOE_OPTION_TILE_ROWS = 10,
   MOE_OPTION_INTERLEAVE = 11,
+  MOE_OPTION_CTAS_PER_SM = 12,
+  MOE_OPTION_DOWN_TILE_COLS = 13,
   MOE_OPTION_TEST_WAIT_TIMEOUT = 100
 };
 int moe_plan_set_option(moe_plan_t plan, int option, int64_t value);

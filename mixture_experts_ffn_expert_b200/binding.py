@@ -33,6 +33,8 @@ MOE_OPTION_SWIGLU_TILE_COLS = 8
 MOE_OPTION_SHARED_CONCURRENT = 9
 MOE_OPTION_TILE_ROWS = 10
 MOE_OPTION_INTERLEAVE = 11
+MOE_OPTION_CTAS_PER_SM = 12
+MOE_OPTION_DOWN_TILE_COLS = 13
 MOE_OPTION_TEST_WAIT_TIMEOUT = 100
 
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_INVALID_CONFIG", 2: "MOE_INVALID_ARG",

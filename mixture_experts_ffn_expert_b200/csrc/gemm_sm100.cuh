@@ -96,30 +96,45 @@ struct GemmParams {
 };
 
 // Single-CTA kernel shapes: BN accumulator columns per tile (MMA N), TM rows
-// per tile. BN = 256, TM = 128 is the default. BN = 128 (SwiGLU only: 64 gate +
-// 64 up columns, 64 output columns per tile) halves the weight bytes per tile,
-// so that weight-streaming launches with few rows per expert split into more,
-// shorter tiles, and it keeps four accumulators in TMEM. TM = 64 (M=64 MMAs,
+// per tile. BN = 256, TM = 128 is the default. Narrower tiles - SwiGLU BN = 128
+// (64 gate + 64 up columns, 64 output columns) or BN = 64 (32 output columns),
+// plain BN = 128 - carry fewer weight bytes per tile, so that weight-streaming
+// launches with few rows per expert split into more, shorter tiles and the
+// last wave of the grid is less empty. TM = 64 (M=64 MMAs,
 // 64-row boxes of the grouped rows) halves the grouped-row bytes per stage, so
 // that the same shared memory holds more stages, i.e. more weight bytes in
 // flight per SM, when the groups are small anyway.
-template <int BN, int TM = 128>
+// OCC = 2 CTAs resident per SM, each with half the ring and half the TMEM: a
+// streaming launch then runs two independent load -> MMA pipelines per SM. One
+// pipeline (one chain of stage barriers) moves about 25-30 GB/s whatever its
+// depth, so on 148 SMs one pipeline per SM stops near 4.4 TB/s of TMA traffic
+// while two reach about 6 TB/s (a load-only streaming measurement on B200).
+template <int BN, int TM = 128, int OCC = 1>
 struct SingleCfg {
   static constexpr int kABytes = TM * kBK * 2;                // grouped rows per stage
   static constexpr int kBBytes = BN * kBK * 2;                // weight rows per stage
   static constexpr int kStage = kABytes + kBBytes;
-  // as many stages as 200 KB hold, at most 8: 4 x 48 KB, 6 x 32 KB, 8 x 24 KB, 5 x 40 KB
-  static constexpr int kStages = (200 * 1024) / kStage < 8 ? (200 * 1024) / kStage : 8;
-  static constexpr int kAcc = 512 / BN;                       // accumulators in TMEM
+  // as many stages as the ring budget holds, at most 8: with 200 KB 4 x 48 KB,
+  // 6 x 32 KB, 8 x 24 KB, 5 x 40 KB; with 96 KB (two CTAs per SM) 2 x 48 KB,
+  // 3 x 32 KB, 4 x 24 KB, 2 x 40 KB
+  static constexpr int kBudget = OCC == 1 ? 200 * 1024 : 96 * 1024;
+  static constexpr int kStages = kBudget / kStage < 8 ? kBudget / kStage : 8;
+  static constexpr int kTmemCols = 512 / OCC;                 // this CTA's TMEM columns
+  static constexpr int kAcc = kTmemCols / BN;                 // accumulators in TMEM
   static constexpr int kHalfRows = BN / 2;                    // rows of one SwiGLU B box
+  // barrier area after the ring: full/empty per stage, tfull/tempty per
+  // accumulator, the drain barrier, the TMEM address and the abort flag
+  static constexpr int kBarBytes = ((2 * kStages + 2 * kAcc + 1) * 8 + 8 + 127) / 128 * 128;
+  static_assert(OCC == 1 || OCC == 2, "one or two CTAs per SM");
+  static_assert(kStages >= 2 && kAcc >= 1, "ring and accumulator fit");
 };
 
 // Dynamic shared memory the kernel needs for a given number of groups.
-template <int BN = 256, int TM = 128>
+template <int BN = 256, int TM = 128, int OCC = 1>
 __host__ __device__ constexpr size_t gemm_smem_bytes(int num_groups) {
   return 1024 /* alignment slack */ +
-         size_t(SingleCfg<BN, TM>::kStages) * SingleCfg<BN, TM>::kStage + 256 /* barriers */ +
-         size_t(3) * (num_groups + 1) * sizeof(int);
+         size_t(SingleCfg<BN, TM, OCC>::kStages) * SingleCfg<BN, TM, OCC>::kStage +
+         SingleCfg<BN, TM, OCC>::kBarBytes + size_t(3) * (num_groups + 1) * sizeof(int);
 }
 
 struct TileCoord {
@@ -208,15 +223,16 @@ __device__ __forceinline__ void raise_timeout(volatile int* s_abort, int* status
 }
 
 
-template <int MODE, int BN = 256, int TM = 128>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+template <int MODE, int BN = 256, int TM = 128, int OCC = 1>
+__global__ void __launch_bounds__(kGemmThreads, OCC)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmA2,
                     const __grid_constant__ CUtensorMap tmB0x, const __grid_constant__ CUtensorMap tmB1x,
                     const GemmParams P) {
-  static_assert(BN == 256 || (BN == 128 && MODE == kEpiSwiGLU), "BN 128 is a SwiGLU shape");
+  static_assert(BN == 256 || BN == 128 || (BN == 64 && MODE == kEpiSwiGLU),
+                "tiles of 256 or 128 accumulator columns, or 64 for SwiGLU");
   static_assert(TM == 128 || TM == 64, "tiles of 128 or 64 rows");
-  using Cfg = SingleCfg<BN, TM>;
+  using Cfg = SingleCfg<BN, TM, OCC>;
   constexpr int kStages = Cfg::kStages;
   constexpr int kABytes = Cfg::kABytes;
   constexpr int kStageBytes = Cfg::kStage;
@@ -233,7 +249,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain_bar = tempty_bar + kNumAcc;      // MMA drain on abort
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
-  int* s_off = reinterpret_cast<int*>(smem + size_t(kStages) * kStageBytes + 256);
+  int* s_off = reinterpret_cast<int*>(smem + size_t(kStages) * kStageBytes + Cfg::kBarBytes);
   const int num_groups = P.group_offsets ? P.num_groups : 1;
   int* s_mp = s_off + (num_groups + 1);
   int* s_mp_b = P.group_mtiles_b ? s_mp + (num_groups + 1) : nullptr;
@@ -264,7 +280,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(s_tmem), kTmemCols);
+    tmem_alloc(smem_u32(s_tmem), Cfg::kTmemCols);
     tmem_relinquish();
   }
   // everything above overlaps the previous kernel; the group tables and the A
@@ -342,18 +358,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int k0 = kb * kBK;
           mbar_arrive_expect_tx(fb, kStageBytes);
           tma_load_2d(a_dst, mA, fb, k0, tc.row0);
-          // SwiGLU: BN/2 rows of W1 then the same rows of W3; plain: two
-          // 128-row boxes of the one weight
+          // SwiGLU: BN/2 rows of W1 then the same rows of W3; plain: BN rows
+          // of the one weight in 128-row boxes (one or two)
           const CUtensorMap* b1 = MODE == kEpiSwiGLU ? mB1 : mB0;
-          const int n0 = MODE == kEpiSwiGLU ? tc.n_blk * (BN / 2) : tc.n_blk * 256;
+          const int n0 = MODE == kEpiSwiGLU ? tc.n_blk * (BN / 2) : tc.n_blk * BN;
           const int n1 = MODE == kEpiSwiGLU ? n0 : n0 + 128;
+          constexpr bool kTwoBoxes = MODE == kEpiSwiGLU || BN == 256;
           const uint32_t b_hi = b_dst + (MODE == kEpiSwiGLU ? kHalfBytes : kBHalfBytes);
           if (stream) {
             tma_load_3d_hint(b_dst, mB0, fb, k0, n0, z, once);
-            tma_load_3d_hint(b_hi, b1, fb, k0, n1, z, once);
+            if (kTwoBoxes) tma_load_3d_hint(b_hi, b1, fb, k0, n1, z, once);
           } else {
             tma_load_3d(b_dst, mB0, fb, k0, n0, z);
-            tma_load_3d(b_hi, b1, fb, k0, n1, z);
+            if (kTwoBoxes) tma_load_3d(b_hi, b1, fb, k0, n1, z);
           }
         }
         __syncwarp();
@@ -482,9 +499,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       } else {
-        const int col0 = tc.n_blk * 256;
+        const int col0 = tc.n_blk * BN;
 #pragma unroll 1
-        for (int c = 0; c < 256; c += 32) {
+        for (int c = 0; c < BN; c += 32) {
           if (col0 + c >= n_valid) break;              // warp-uniform
           uint32_t a[32];
           tmem_ld_32cols(tbase + c, a);
@@ -533,7 +550,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+  if (warp == 1) tmem_dealloc(tmem_base, Cfg::kTmemCols);
 }
 
 
@@ -592,6 +609,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   uint64_t* drain_bar = tempty_bar + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  static_assert((2 * kS + 2 + 2 + 1) * 8 + 8 <= 256, "pair barriers fit their 256 bytes");
   int* s_off = reinterpret_cast<int*>(smem + size_t(kS) * Cfg::kStageBytes + 256);
   const int num_groups = P.group_offsets ? P.num_groups : 1;
   int* s_mp = s_off + (num_groups + 1);

@@ -89,6 +89,12 @@ struct moe_plan {
   // rows of a single-CTA routed GEMM tile: 0 automatic (64 when the expected
   // rows per expert are below 32, else 128), 64 or 128
   int tile_rows = 0;
+  // resident CTAs per SM of single-CTA routed GEMMs: 0 automatic (2 when the
+  // expected rows per expert are below 32, else 1), 1 or 2
+  int ctas_per_sm = 0;
+  // output columns of a single-CTA routed down tile: 0 automatic (128 with two
+  // CTAs per SM when the expected rows per expert are below 32, else 256), 128 or 256
+  int down_tile_cols = 0;
   // shared expert beside weight-streaming routed GEMMs: -1 automatic, 0 never, 1 always.
   // Measured on B200 (DeepSeek-V3-shaped prefill): beside the routed GEMMs on 16
   // SMs the layer took 7.09 ms per step against 6.19 ms inline (the capped
@@ -171,7 +177,7 @@ moe::RouterParams router_shape(const moe_plan* p, int64_t T, size_t* smem) {
   while (cols < r.ncols) cols *= 2;
   r.tmem_cols = cols;
   // fold the tile scan into the router's last cluster while there are few
-  // tiles (one warp per expert walks them)
+  // tiles (one thread per expert walks them)
   r.fold_scan = r.n_chunks <= 64 ? 1 : 0;
   // at least kRouterMinSmem so that two router CTAs never share an SM: each
   // allocates tensor memory and then waits at cluster barriers, and two
@@ -398,25 +404,57 @@ bool launch_pair_auto(Launcher& L, cudaStream_t s, const char* name, const CUten
 // Single-CTA GEMM with BN accumulator columns per tile. x (optional) holds the
 // A, B0, B1 maps of the extra dense problem that prm.x_tiles describes;
 // max_tiles bounds the grouped tiles only.
-template <int MODE, int BN = 256, int TM = 128>
+template <int MODE, int BN = 256, int TM = 128, int OCC = 1>
 bool launch_gemm(Launcher& L, cudaStream_t s, const char* name, const CUtensorMap& a,
                  const CUtensorMap& b0, const CUtensorMap& b1, const moe::GemmParams& prm,
                  int max_tiles, const CUtensorMap* x = nullptr) {
   const int num_groups = prm.group_offsets ? prm.num_groups : 1;
-  const size_t smem = moe::gemm_smem_bytes<BN, TM>(num_groups);
+  const size_t smem = moe::gemm_smem_bytes<BN, TM, OCC>(num_groups);
   const long long tiles = static_cast<long long>(max_tiles) + (x ? prm.x_tiles : 0);
-  const int sms = L.p->num_sms < L.grid_cap ? L.p->num_sms : L.grid_cap;
+  const int sms = (L.p->num_sms < L.grid_cap ? L.p->num_sms : L.grid_cap) * OCC;
   int grid = tiles < sms ? static_cast<int>(tiles) : sms;
   if (grid < 1) grid = 1;
   moe::GemmParams q = prm;
   if (!x) q.x_tiles = 0;
-  const char* tag = q.x_tiles > 0 ? "[+shared]"
-                    : BN == 128 ? (TM == 64 ? "[n64,m64]" : "[n64]")
-                    : (TM == 64 ? "[m64]" : "");
+  // variant tag: output columns when not the widest tile, 64-row tiles, two
+  // CTAs per SM, or the shared expert merged in
+  char tag[32] = "";
+  const int out_cols = MODE == moe::kEpiSwiGLU ? BN / 2 : BN;
+  const bool narrow = out_cols < (MODE == moe::kEpiSwiGLU ? 128 : 256);
+  if (q.x_tiles > 0)
+    snprintf(tag, sizeof(tag), "[+shared]");
+  else if (narrow || TM == 64 || OCC == 2)
+    snprintf(tag, sizeof(tag), "[%s%s%s%s%s]",
+             narrow ? (out_cols == 32 ? "n32" : out_cols == 64 ? "n64" : "n128") : "",
+             narrow && TM == 64 ? "," : "", TM == 64 ? "m64" : "",
+             (narrow || TM == 64) && OCC == 2 ? "," : "", OCC == 2 ? "x2" : "");
   L.begin(name, s, tag);
-  launch_pdl(moe::moe_gemm_kernel<MODE, BN, TM>, dim3(grid), dim3(moe::kGemmThreads), smem, s,
-             a, b0, b1, x ? x[0] : a, x ? x[1] : b0, x ? x[2] : b1, q);
+  launch_pdl(moe::moe_gemm_kernel<MODE, BN, TM, OCC>, dim3(grid), dim3(moe::kGemmThreads), smem,
+             s, a, b0, b1, x ? x[0] : a, x ? x[1] : b0, x ? x[2] : b1, q);
   return L.end(name, s);
+}
+
+// The same launch with one or two CTAs per SM (two: the weight-streaming
+// regime, where two independent load pipelines per SM move more bytes).
+template <int MODE, int BN = 256, int TM = 128>
+bool launch_gemm_occ(bool two, Launcher& L, cudaStream_t s, const char* name,
+                     const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                     const moe::GemmParams& prm, int max_tiles, const CUtensorMap* x = nullptr) {
+  return two ? launch_gemm<MODE, BN, TM, 2>(L, s, name, a, b0, b1, prm, max_tiles, x)
+             : launch_gemm<MODE, BN, TM, 1>(L, s, name, a, b0, b1, prm, max_tiles, x);
+}
+
+// Shared-memory attributes of a two-CTAs-per-SM instantiation: its dynamic
+// shared memory, and the largest shared-memory carveout so that two fit.
+template <int MODE, int BN, int TM>
+cudaError_t set_occ2_attributes() {
+  auto* k = moe::moe_gemm_kernel<MODE, BN, TM, 2>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(moe::gemm_smem_bytes<BN, TM, 2>(moe::kMaxRouted)));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             int(cudaSharedmemCarveoutMaxShared));
+  return e;
 }
 
 typedef cudaFuncAttribute cudaAttr;
@@ -457,6 +495,31 @@ int set_kernel_attributes() {
   if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess)
     return fail(MOE_CUDA_ERROR, "cudaFuncSetAttribute failed: %s",
                 cudaGetErrorString(e1 != cudaSuccess ? e1 : (e2 != cudaSuccess ? e2 : e3)));
+  const cudaError_t en[4] = {
+      cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiSwiGLU, 64, 64>, attr,
+                           int(moe::gemm_smem_bytes<64, 64>(moe::kMaxRouted))),
+      cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiSwiGLU, 64, 128>, attr,
+                           int(moe::gemm_smem_bytes<64, 128>(moe::kMaxRouted))),
+      cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiBF16, 128, 64>, attr,
+                           int(moe::gemm_smem_bytes<128, 64>(moe::kMaxRouted))),
+      cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiBF16, 128, 128>, attr,
+                           int(moe::gemm_smem_bytes<128, 128>(moe::kMaxRouted)))};
+  for (cudaError_t e : en)
+    if (e != cudaSuccess)
+      return fail(MOE_CUDA_ERROR, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
+  const cudaError_t eo[10] = {set_occ2_attributes<moe::kEpiSwiGLU, 64, 64>(),
+                             set_occ2_attributes<moe::kEpiSwiGLU, 64, 128>(),
+                             set_occ2_attributes<moe::kEpiBF16, 128, 64>(),
+                             set_occ2_attributes<moe::kEpiBF16, 128, 128>(),
+                             set_occ2_attributes<moe::kEpiSwiGLU, 128, 64>(),
+                             set_occ2_attributes<moe::kEpiSwiGLU, 128, 128>(),
+                             set_occ2_attributes<moe::kEpiSwiGLU, 256, 64>(),
+                             set_occ2_attributes<moe::kEpiSwiGLU, 256, 128>(),
+                             set_occ2_attributes<moe::kEpiBF16, 256, 64>(),
+                             set_occ2_attributes<moe::kEpiBF16, 256, 128>()};
+  for (cudaError_t e : eo)
+    if (e != cudaSuccess)
+      return fail(MOE_CUDA_ERROR, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
   const int rsm = 227 * 1024;
   const cudaError_t er[2] = {cudaFuncSetAttribute(moe::route_fused_kernel<8>, attr, rsm),
                              cudaFuncSetAttribute(moe::route_fused_kernel<16>, attr, rsm)};
@@ -638,14 +701,23 @@ int moe_plan_set_option(moe_plan_t p, int option, int64_t value) {
       if (value < -1 || value > 1) return fail(MOE_INVALID_ARG, "interleave must be -1, 0 or 1");
       p->interleave = static_cast<int>(value);
       return MOE_OK;
+    case MOE_OPTION_CTAS_PER_SM:
+      if (value < 0 || value > 2) return fail(MOE_INVALID_ARG, "ctas per SM must be 0, 1 or 2");
+      p->ctas_per_sm = static_cast<int>(value);
+      return MOE_OK;
     case MOE_OPTION_TILE_ROWS:
       if (value != 0 && value != 64 && value != 128)
         return fail(MOE_INVALID_ARG, "tile rows must be 0, 64 or 128");
       p->tile_rows = static_cast<int>(value);
       return MOE_OK;
+    case MOE_OPTION_DOWN_TILE_COLS:
+      if (value != 0 && value != 128 && value != 256)
+        return fail(MOE_INVALID_ARG, "down tile columns must be 0, 128 or 256");
+      p->down_tile_cols = static_cast<int>(value);
+      return MOE_OK;
     case MOE_OPTION_SWIGLU_TILE_COLS:
-      if (value != 0 && value != 64 && value != 128)
-        return fail(MOE_INVALID_ARG, "swiglu tile columns must be 0, 64 or 128");
+      if (value != 0 && value != 32 && value != 64 && value != 128)
+        return fail(MOE_INVALID_ARG, "swiglu tile columns must be 0, 32, 64 or 128");
       p->swiglu_tile_cols = static_cast<int>(value);
       return MOE_OK;
     case MOE_OPTION_FUSED_ROUTER:
@@ -963,16 +1035,29 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   // the routed GEMMs leave the concurrent shared expert its SMs
   if (shared_sms > 0) L.grid_cap = p->num_sms - shared_sms;
   // 5. grouped gate/up GEMM with the SiLU(gate) * up epilogue. With few rows
-  //    per expert (weight streaming) the single-CTA kernel uses 64-column
-  //    tiles (twice as many, shorter tiles, so the last wave is shorter) of 64
-  //    rows (more stages, so more weight bytes in flight per SM).
-  const bool narrow_gu =
-      !routed_pair_swiglu && !merge_gu &&
-      (p->swiglu_tile_cols == 64 || (p->swiglu_tile_cols == 0 && rows_per_expert < 32));
-  const bool short_gu = !routed_pair_swiglu && !merge_gu &&
-                        (p->tile_rows == 64 || (p->tile_rows == 0 && rows_per_expert < 32));
-  const bool short_dn = !routed_pair && !merge_dn &&
-                        (p->tile_rows == 64 || (p->tile_rows == 0 && rows_per_expert < 32));
+  //    per expert (weight streaming) the single-CTA kernels run two CTAs per
+  //    SM (two load pipelines per SM) on narrow tiles of 64 rows: 32 output
+  //    columns (64 with one CTA per SM), so that the grid's last wave is short,
+  //    and 64-row boxes of the grouped rows, so that more stages fit.
+  const bool single_gu = !routed_pair_swiglu && !merge_gu;
+  const bool single_dn = !routed_pair && !merge_dn;
+  const bool streaming = rows_per_expert < 32;
+  const bool occ2_gu =
+      single_gu && (p->ctas_per_sm == 2 || (p->ctas_per_sm == 0 && streaming));
+  const bool occ2_dn =
+      single_dn && (p->ctas_per_sm == 2 || (p->ctas_per_sm == 0 && streaming));
+  int gu_cols = 128;   // output columns of a gate/up tile
+  if (single_gu)
+    gu_cols = p->swiglu_tile_cols != 0 ? p->swiglu_tile_cols
+                                       : (streaming ? (occ2_gu ? 32 : 64) : 128);
+  int dn_cols = 256;   // output columns of a down tile
+  if (single_dn)
+    dn_cols = p->down_tile_cols != 0 ? p->down_tile_cols : (streaming && occ2_dn ? 128 : 256);
+  const bool narrow_gu = gu_cols < 128;
+  const bool short_gu =
+      single_gu && (p->tile_rows == 64 || (p->tile_rows == 0 && streaming));
+  const bool short_dn =
+      single_dn && (p->tile_rows == 64 || (p->tile_rows == 0 && streaming));
   const int max_mtiles64 = static_cast<int>((A + 63) / 64 + (A < nr ? A : nr));
   // 128-row single-CTA routed GEMMs in the weight-streaming regime run the
   // tiles of experts with several m-blocks (tensor-heavy: each weight tile is
@@ -991,7 +1076,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.num_groups = nr;
     g.K = d;
     g.N = f;
-    g.n_tiles = narrow_gu ? (f + 63) / 64 : (f + 127) / 128;
+    g.n_tiles = (f + gu_cols - 1) / gu_cols;
     g.out = hidden;
     g.ldo = f;
     g.status = status;
@@ -1013,26 +1098,40 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     bool launched;
     if (narrow_gu) {
       CUtensorMap mW1n, mW3n;
-      if (!make_map(&mW1n, W1, nr, f, d, 64) || !make_map(&mW3n, W3, nr, f, d, 64))
+      const uint32_t box = static_cast<uint32_t>(gu_cols);
+      if (!make_map(&mW1n, W1, nr, f, d, box) || !make_map(&mW3n, W3, nr, f, d, box))
         return fail(MOE_CUDA_ERROR, "cuTensorMapEncodeTiled rejected a tensor map");
-      launched = short_gu ? launch_gemm<moe::kEpiSwiGLU, 128, 64>(L, main_st, "grouped_gate_up",
-                                                                  mXp64, mW1n, mW3n, g,
-                                                                  mtmax * g.n_tiles)
-                          : launch_gemm<moe::kEpiSwiGLU, 128>(L, main_st, "grouped_gate_up", mXp,
-                                                              mW1n, mW3n, g, mtmax * g.n_tiles);
+      if (gu_cols == 32)
+        launched = short_gu
+                       ? launch_gemm_occ<moe::kEpiSwiGLU, 64, 64>(occ2_gu, L, main_st,
+                                                                  "grouped_gate_up", mXp64, mW1n,
+                                                                  mW3n, g, mtmax * g.n_tiles)
+                       : launch_gemm_occ<moe::kEpiSwiGLU, 64>(occ2_gu, L, main_st,
+                                                              "grouped_gate_up", mXp, mW1n, mW3n,
+                                                              g, mtmax * g.n_tiles);
+      else
+        launched = short_gu
+                       ? launch_gemm_occ<moe::kEpiSwiGLU, 128, 64>(occ2_gu, L, main_st,
+                                                                   "grouped_gate_up", mXp64,
+                                                                   mW1n, mW3n, g,
+                                                                   mtmax * g.n_tiles)
+                       : launch_gemm_occ<moe::kEpiSwiGLU, 128>(occ2_gu, L, main_st,
+                                                               "grouped_gate_up", mXp, mW1n,
+                                                               mW3n, g, mtmax * g.n_tiles);
     } else if (routed_pair_swiglu) {
       launched = launch_pair_auto<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1, mW3, g,
                                                    f, expected_mtiles2, max_mtiles2);
     } else if (short_gu) {
-      launched = launch_gemm<moe::kEpiSwiGLU, 256, 64>(L, main_st, "grouped_gate_up", mXp64, mW1,
-                                                       mW3, g, mtmax * g.n_tiles);
+      launched = launch_gemm_occ<moe::kEpiSwiGLU, 256, 64>(occ2_gu, L, main_st, "grouped_gate_up",
+                                                           mXp64, mW1, mW3, g, mtmax * g.n_tiles);
     } else {
       if (interleave && !merge_gu) {
         g.group_mtiles = mt_hot;
         g.group_mtiles_b = mt_cold;
       }
-      launched = launch_gemm<moe::kEpiSwiGLU>(L, main_st, "grouped_gate_up", mXp, mW1, mW3, g,
-                                              mtmax * g.n_tiles, merge_gu ? xgu : nullptr);
+      launched = launch_gemm_occ<moe::kEpiSwiGLU>(occ2_gu, L, main_st, "grouped_gate_up", mXp, mW1,
+                                                  mW3, g, mtmax * g.n_tiles,
+                                                  merge_gu ? xgu : nullptr);
     }
     if (!launched) return L.status;
   }
@@ -1044,7 +1143,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.num_groups = nr;
     g.K = f;
     g.N = d;
-    g.n_tiles = (d + 255) / 256;
+    g.n_tiles = (d + dn_cols - 1) / dn_cols;
     g.out = yrouted;
     g.ldo = d;
     g.status = status;
@@ -1064,15 +1163,24 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
       launched = launch_pair_auto<moe::kEpiBF16>(L, main_st, "grouped_down", mH, mW2, mW2, g, d,
                                                  expected_mtiles2, max_mtiles2);
     else if (short_dn)
-      launched = launch_gemm<moe::kEpiBF16, 256, 64>(L, main_st, "grouped_down", mH64, mW2, mW2,
-                                                     g, max_mtiles64 * g.n_tiles);
+      launched = dn_cols == 128
+                     ? launch_gemm_occ<moe::kEpiBF16, 128, 64>(occ2_dn, L, main_st, "grouped_down",
+                                                               mH64, mW2, mW2, g,
+                                                               max_mtiles64 * g.n_tiles)
+                     : launch_gemm_occ<moe::kEpiBF16, 256, 64>(occ2_dn, L, main_st, "grouped_down",
+                                                               mH64, mW2, mW2, g,
+                                                               max_mtiles64 * g.n_tiles);
     else {
       if (interleave && !merge_dn) {
         g.group_mtiles = mt_hot;
         g.group_mtiles_b = mt_cold;
       }
-      launched = launch_gemm<moe::kEpiBF16>(L, main_st, "grouped_down", mH, mW2, mW2, g,
-                                            max_mtiles * g.n_tiles, merge_dn ? xdn : nullptr);
+      launched = dn_cols == 128
+                     ? launch_gemm_occ<moe::kEpiBF16, 128>(occ2_dn, L, main_st, "grouped_down",
+                                                           mH, mW2, mW2, g, max_mtiles * g.n_tiles)
+                     : launch_gemm_occ<moe::kEpiBF16>(occ2_dn, L, main_st, "grouped_down", mH,
+                                                      mW2, mW2, g, max_mtiles * g.n_tiles,
+                                                      merge_dn ? xdn : nullptr);
     }
     if (!launched) return L.status;
   }

@@ -40,7 +40,7 @@
 
 namespace moe {
 
-constexpr int kRtThreads = 512;   // 16 warps: 16 tokens merged at once per CTA
+constexpr int kRtThreads = 1024;  // 32 warps: 32 tokens selected at once per CTA
 constexpr int kRtMaxCluster = 8;
 constexpr int kRtMaxStages = 8;
 constexpr int kRtMaxExperts = 512;
@@ -177,12 +177,12 @@ __device__ __forceinline__ void select_rounds(const uint32_t (&key)[N], const in
 }
 
 // One warp, one token, one slice: lane l holds the slice's experts e0 + l and
-// e0 + l + 32 (n_valid of them are experts). Returns to every lane the slice's
+// e0 + l + 32 (n_valid of them are experts; their logit biases in bias[]). Returns to every lane the slice's
 // largest gate score m and sum of exp(score - m) (0 for an empty slice), and
 // to lane j < k the j-th candidate by selection key (ties to the lower expert)
 // as (key, expert, gate score); key 0 where the slice has fewer than k experts.
 __device__ __forceinline__ void slice_select(const float* srow, int n_valid, int e0,
-                                             const float* __restrict__ bias, int bias_select_only,
+                                             const float (&bias)[2], int bias_select_only,
                                              int k, int lane, float& m, float& sum,
                                              uint32_t& my_key, int& my_e, float& my_g) {
   uint32_t key[2];
@@ -194,7 +194,7 @@ __device__ __forceinline__ void slice_select(const float* srow, int n_valid, int
     const int c = lane + 32 * i;
     const bool v = c < n_valid;
     const float raw = v ? srow[c] : 0.0f;
-    const float kv = (v && bias) ? raw + __ldg(bias + e0 + c) : raw;
+    const float kv = raw + bias[i];   // 0 without a logit bias
     g[i] = bias_select_only ? raw : kv;
     key[i] = v ? order_key(kv) : 0u;
     ex[i] = v ? e0 + c : 0x7fffffff;
@@ -343,7 +343,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   }
 
   // ---------------------------------------------------------------- scores to shared memory
-  // every warp copies a quarter of the slice's columns of one TMEM lane
+  // warps 0..15 each copy a quarter of the slice's columns of one TMEM lane
   // quarter (warps w, w+4, w+8, w+12 share lanes 32*(w%4)..) into the score
   // rows [token][ncols + 1] laid over the ring (every MMA has completed, so
   // every stage has been read)
@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     const int row = q * 32 + lane;
     const int cpp = P.ncols / 4;                  // a multiple of 8
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    if (nkb > 0 && ok) {
+    if (nkb > 0 && ok && warp < 16) {
 #pragma unroll 1
       for (int c = (warp >> 2) * cpp; c < ((warp >> 2) + 1) * cpp; c += 8) {
         uint32_t a[8];
@@ -378,13 +378,19 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   {
     const bool have = nkb > 0 && *s_abort == 0;
     const int own_r = P.own_rows;
+    float bias[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int c = lane + 32 * i;
+      bias[i] = (P.bias && c < n_valid) ? __ldg(P.bias + e0 + c) : 0.0f;
+    }
 #pragma unroll 1
     for (int row = warp; row < kBM; row += kRtThreads / 32) {
       float m, sum;
       uint32_t my_key;
       int my_e;
       float my_g;
-      slice_select(s_score + row * lds, have ? n_valid : 0, e0, P.bias, P.bias_select_only,
+      slice_select(s_score + row * lds, have ? n_valid : 0, e0, bias, P.bias_select_only,
                    k, lane, m, sum, my_key, my_e, my_g);
       if (P.cs == 1) {
         // one slice holds every expert: the token's softmax and top k
@@ -502,12 +508,25 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     __syncthreads();
     if (*s_last) {
       __threadfence();
-      // one warp per expert (other clusters' counts: read through L2)
+      // one thread per expert (other clusters' counts: read through L2), eight
+      // tiles' counts loaded before the first of them is rewritten
 #pragma unroll 1
-      for (int e = warp; e < P.n_routed; e += kRtThreads / 32) {
-        const int tot = scan_expert_chunks<true>(
-            P.tile_counts + static_cast<long long>(e) * P.n_chunks, P.n_chunks, lane);
-        if (lane == 0) P.counts[e] = tot;
+      for (int e = threadIdx.x; e < P.n_routed; e += kRtThreads) {
+        int* rowp = P.tile_counts + static_cast<long long>(e) * P.n_chunks;
+        int run = 0;
+#pragma unroll 1
+        for (int c0 = 0; c0 < P.n_chunks; c0 += 8) {
+          int v[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[j] = c0 + j < P.n_chunks ? __ldcg(rowp + c0 + j) : 0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (c0 + j < P.n_chunks) {
+              rowp[c0 + j] = run;
+              run += v[j];
+            }
+        }
+        P.counts[e] = run;
       }
       if (threadIdx.x == 0) *P.ticket = 0;
     }

@@ -109,7 +109,7 @@ def check_output(gpu_out: np.ndarray, ref: np.ndarray):
 
 
 def run_layer(inp, shape, device="cuda", pair_min_rows=None, wide_tiles=None, merge_shared=None,
-              capacity=None, bias_selection_only=False, fused_router=None):
+              capacity=None, bias_selection_only=False, fused_router=None, **kernel_options):
     """Run the CUDA layer through the C ABI; returns (out (T,d) fp64 numpy, routing dict)."""
     from mixture_experts_ffn_expert_b200.layer import MoELayer
 
@@ -118,7 +118,8 @@ def run_layer(inp, shape, device="cuda", pair_min_rows=None, wide_tiles=None, me
                                                         "W3s", "W2s")},
                      bias=inp["bias"], device=device, pair_min_rows=pair_min_rows,
                      wide_tiles=wide_tiles, merge_shared=merge_shared, capacity=capacity,
-                     bias_selection_only=bias_selection_only, fused_router=fused_router)
+                     bias_selection_only=bias_selection_only, fused_router=fused_router,
+                     **kernel_options)
     out = layer(inp["x"])
     routing = layer.routing()
     torch.cuda.synchronize()
@@ -127,17 +128,19 @@ def run_layer(inp, shape, device="cuda", pair_min_rows=None, wide_tiles=None, me
 
 
 def full_parity(inp, shape, tokens=None, pair_min_rows=None, wide_tiles=None,
-                merge_shared=None, capacity=None, bias_selection_only=False, fused_router=None):
+                merge_shared=None, capacity=None, bias_selection_only=False, fused_router=None,
+                **kernel_options):
     """Routing on all tokens, output on `tokens` (all when None). Returns a summary dict.
     pair_min_rows forces (0) or forbids (huge) the CTA-pair GEMM kernel; wide_tiles
     forces (1) or forbids (0) its 512-column tiles; merge_shared forces (1) or
     forbids (0) the shared expert as extra tiles of the routed GEMM launches;
     capacity sets the seats per expert (token dropping); bias_selection_only keeps
-    the bias out of the gates; fused_router 0 forces the two-kernel router."""
+    the bias out of the gates; fused_router 0 forces the two-kernel router; the
+    other keyword arguments are MoELayer kernel options (tile_rows, ctas_per_sm, ...)."""
     out, routing, layer = run_layer(inp, shape, pair_min_rows=pair_min_rows,
                                     wide_tiles=wide_tiles, merge_shared=merge_shared,
                                     capacity=capacity, bias_selection_only=bias_selection_only,
-                                    fused_router=fused_router)
+                                    fused_router=fused_router, **kernel_options)
     _, idx_ref, n_near = check_routing(inp, routing, shape, capacity=capacity,
                                        bias_selection_only=bias_selection_only)
     ref = oracle_out(inp, shape, idx_ref, tokens, capacity=capacity,

@@ -144,6 +144,40 @@ def test_interleaved_tile_order(shape):
     assert torch.equal(outs[0], outs[1])
 
 
+OCC_CASES = [
+    # weight streaming: few rows per expert, 64- and 128-row tiles
+    LayerShape("occ_decode_like", 96, 256, 128, 64, 6, 1, True, "zipf1.1"),
+    # several m-blocks per expert and a ragged tail
+    LayerShape("occ_ragged", 1100, 256, 192, 8, 2, 0, False, "normal_var0.5"),
+]
+
+
+@pytest.mark.parametrize("tile_rows,cols,dcols", [(64, 32, 128), (64, 64, 256), (64, 128, 128),
+                                                   (128, 32, 256), (128, 64, 128),
+                                                   (128, 128, 256)])
+@pytest.mark.parametrize("shape", OCC_CASES, ids=[c.name for c in OCC_CASES])
+def test_two_ctas_per_sm_routed_gemms(shape, tile_rows, cols, dcols):
+    # two resident CTAs per SM run the same tiles with half the ring each, and
+    # tiles of 32..128 gate/up and 128 or 256 down output columns: the same bits
+    # as one CTA per SM, and parity with the oracle
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    inp = make_layer_inputs(shape, seed=23, device="cuda")
+    opts = dict(tile_rows=tile_rows, swiglu_tile_cols=cols, down_tile_cols=dcols,
+                pair_min_rows=1 << 40)
+    full_parity(inp, shape, ctas_per_sm=2, **opts)
+    outs = []
+    for occ in (1, 2):
+        layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
+                         shape.renorm, inp, bias=inp["bias"], device="cuda", ctas_per_sm=occ,
+                         **opts)
+        outs.append(layer(inp["x"]).clone())
+        torch.cuda.synchronize()
+        assert layer.device_status() == 0
+        names = layer.plan.kernel_names()
+        assert any(n.startswith("grouped_gate_up") and ("x2" in n) == (occ == 2) for n in names)
+    assert torch.equal(outs[0], outs[1])
+
+
 PAIR_CASES = ["three_tokens", "ragged_17", "two_shared_raw", "ragged_tiles", "k_tail_not_64",
               "skewed_groups"]
 
