@@ -43,6 +43,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling runs)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override N_r (profiling runs: a small case of the same kernels)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle timing (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
@@ -235,6 +237,8 @@ def run_reference(args, info):
     shape = WORKLOADS[args.workload]
     if args.tokens:
         shape = shape.with_tokens(args.tokens)
+    if args.experts:
+        shape = shape.with_experts(args.experts)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = host_copy_of_inputs(make_layer_inputs(shape, seed=0, device=dev))
     expert, once = oracle_experts(inp, shape)
@@ -522,6 +526,8 @@ def run_ours(args, info):
     shape = WORKLOADS[args.workload]
     if args.tokens:
         shape = shape.with_tokens(args.tokens)
+    if args.experts:
+        shape = shape.with_experts(args.experts)
 
     head = measure_workload(shape, args, info, dev, args.steps, headline=True)
     per = {}

@@ -117,32 +117,30 @@ int moe_last_status(void);
  *   load-balance bias "Shared Expert (DeepSeek-V3)" mentions for the routed
  *   centroids); the gates are the softmax of the unbiased scores over all N_r
  *   experts, renormalised over the selected ones when the plan renormalises.
- * MOE_OPTION_FUSED_ROUTER: -1 (default) computes the router in one kernel
- *   (scores on the tensor core, softmax, top-k, gates and the expert
- *   histogram of each 128-token tile, with its K range split over a cluster of
- *   up to 8 CTAs) whenever N_r <= 512, else in two (a split-K scores GEMM, then
- *   softmax + top-k); 0 always uses the two-kernel router; 1 is the same as -1.
- *   Both give the same selection up to fp32 rounding of the scores.
+ * MOE_OPTION_FUSED_ROUTER: 1 computes the router in one kernel (scores on
+ *   the tensor core, softmax, top-k, gates and the expert histogram of each
+ *   128-token tile, its experts split over a cluster of up to 8 CTAs, and with
+ *   few tiles the histogram scan) whenever N_r <= 512 and top_k <= 16; 0 and
+ *   -1 (default, measured faster on B200 for every tested shape) use the
+ *   two-kernel router (a split-K scores GEMM, then softmax + top-k, then the
+ *   histogram scan). Both give the same selection up to fp32 rounding of the
+ *   scores.
  * MOE_OPTION_SWIGLU_TILE_COLS: output columns of one tile of the routed
- *   gate/up GEMM when it runs one CTA per tile: 0 (default) chooses, when the
- *   expected rows per expert (T*top_k/N_r) are below 32 - the weight-streaming
- *   decode regime, where more, shorter tiles leave a shorter last wave - 32
- *   with two CTAs per SM and 64 with one, and 128 otherwise; 32, 64 or 128
- *   force it.
+ *   gate/up GEMM when it runs one CTA per tile: 0 (default) is 128 (N=256
+ *   MMAs: on B200 an MMA instruction costs about the same time at any size, so
+ *   the widest moves the most weight bytes, also in the weight-streaming
+ *   decode regime); 32 or 64 (more, narrower tiles) or 128 force it.
  * MOE_OPTION_DOWN_TILE_COLS: output columns of one tile of the routed down
- *   GEMM when it runs one CTA per tile: 0 (default) chooses 128 in the
- *   weight-streaming regime with two CTAs per SM, else 256; 128 or 256 force it.
+ *   GEMM when it runs one CTA per tile: 0 (default) is 256; 128 or 256.
  * MOE_OPTION_TILE_ROWS: rows of one tile of the routed GEMMs when they run
- *   one CTA per tile: 0 (default) chooses 64 when the expected rows per expert
- *   are below 32 (M=64 MMAs and 64-row boxes of the grouped rows: smaller
- *   pipeline stages, so more of them and more weight bytes in flight per SM),
- *   and 128 otherwise; 64 or 128 force it.
+ *   one CTA per tile: 0 (default) is 128; 64 (M=64 MMAs and 64-row boxes of the
+ *   grouped rows: smaller pipeline stages, so more of them) or 128 force it.
  * MOE_OPTION_INTERLEAVE: order of the tiles of the routed GEMMs when they run
  *   one CTA per 128-row tile. 1: the tiles of experts with at least two
  *   m-blocks (tensor-heavy, their weight tiles reused through L2) are spread
  *   evenly among the other experts' tiles (weight streaming), so that tensor
  *   and HBM work overlap; 0: expert order; -1 (default): 1 when the expected
- *   rows per expert are below 192.
+ *   rows per expert (T*top_k/N_r) are from 32 to 191.
  * MOE_OPTION_SHARED_CONCURRENT: where a shared expert too large for the
  *   routing phase runs. 1: beside the routed GEMMs, on a second stream and a
  *   few SMs (the routed GEMMs keep the rest); -1 (default) and 0: after them on
@@ -150,10 +148,9 @@ int moe_last_status(void);
  *   shape). Small shared experts always run beside the routing kernels.
  * MOE_OPTION_CTAS_PER_SM: CTAs per SM of the routed GEMMs when they run one
  *   CTA per tile. 2: two resident CTAs per SM, each with half the pipeline
- *   ring and half the tensor memory (two independent load pipelines per SM,
- *   which stream weights faster); 1: one CTA per SM with the whole ring;
- *   0 (default): 2 when the expected rows per expert are below 32 (weight
- *   streaming), else 1.
+ *   ring and half the tensor memory (two independent pipelines per SM; measured
+ *   no faster on B200, where the SM's MMA issue rate, shared by both, is the
+ *   limit); 1 and 0 (default): one CTA per SM with the whole ring.
  * MOE_OPTION_TEST_WAIT_TIMEOUT: test hook for the failure path, not for normal
  *   use. Value 1 arms it for the next forward only: if that forward runs the
  *   routed gate/up GEMM on the one-CTA-per-tile kernel, one CTA withholds the

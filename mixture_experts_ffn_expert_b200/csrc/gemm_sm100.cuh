@@ -104,11 +104,14 @@ struct GemmParams {
 // 64-row boxes of the grouped rows) halves the grouped-row bytes per stage, so
 // that the same shared memory holds more stages, i.e. more weight bytes in
 // flight per SM, when the groups are small anyway.
-// OCC = 2 CTAs resident per SM, each with half the ring and half the TMEM: a
-// streaming launch then runs two independent load -> MMA pipelines per SM. One
-// pipeline (one chain of stage barriers) moves about 25-30 GB/s whatever its
-// depth, so on 148 SMs one pipeline per SM stops near 4.4 TB/s of TMA traffic
-// while two reach about 6 TB/s (a load-only streaming measurement on B200).
+// OCC = 2 CTAs resident per SM, each with half the ring and half the TMEM:
+// two independent load -> MMA pipelines per SM. A load-only measurement on
+// B200 showed one pipeline of 8 KB stages stuck near 30 GB/s per SM (the
+// producer thread's issue cost per stage) and two near 6 TB/s in all; with the
+// GEMM's 24-48 KB stages one pipeline already streams 6.5 TB/s, and the routed
+// GEMMs are instead bound by the SM's MMA issue rate (about 128 cycles per
+// tcgen05.mma instruction at any size), which both CTAs share - so OCC = 2 is
+// an option, not the default.
 template <int BN, int TM = 128, int OCC = 1>
 struct SingleCfg {
   static constexpr int kABytes = TM * kBK * 2;                // grouped rows per stage

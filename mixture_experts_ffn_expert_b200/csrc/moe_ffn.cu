@@ -78,30 +78,34 @@ struct moe_plan {
   // by default: measured on B200 it ran the merged launches at a lower clock
   // under the power cap and lost 5% on the DeepSeek-V3 layer shape.
   int merge_shared = 0;
-  // output columns of a single-CTA routed SwiGLU tile: 0 automatic (64 when
-  // the expected rows per expert are below 32, the weight-streaming regime,
-  // else 128), 64 or 128
+  // output columns of a single-CTA routed SwiGLU tile: 0 automatic (128), 32,
+  // 64 or 128
   int swiglu_tile_cols = 0;
   // interleave the tiles of experts with several m-blocks among the others in
   // single-CTA 128-row routed GEMMs: -1 automatic (when the expected rows per
-  // expert are below 192, i.e. most experts stream weights), 0 never, 1 always
+  // expert are from 32 to 191, i.e. most experts stream weights but some reuse
+  // them), 0 never, 1 always
   int interleave = -1;
-  // rows of a single-CTA routed GEMM tile: 0 automatic (64 when the expected
-  // rows per expert are below 32, else 128), 64 or 128
+  // rows of a single-CTA routed GEMM tile: 0 automatic (128), 64 or 128
   int tile_rows = 0;
-  // resident CTAs per SM of single-CTA routed GEMMs: 0 automatic (2 when the
-  // expected rows per expert are below 32, else 1), 1 or 2
+  // resident CTAs per SM of single-CTA routed GEMMs: 0 automatic (1), 1 or 2
   int ctas_per_sm = 0;
-  // output columns of a single-CTA routed down tile: 0 automatic (128 with two
-  // CTAs per SM when the expected rows per expert are below 32, else 256), 128 or 256
+  // output columns of a single-CTA routed down tile: 0 automatic (256), 128 or 256
   int down_tile_cols = 0;
   // shared expert beside weight-streaming routed GEMMs: -1 automatic, 0 never, 1 always.
   // Measured on B200 (DeepSeek-V3-shaped prefill): beside the routed GEMMs on 16
   // SMs the layer took 7.09 ms per step against 6.19 ms inline (the capped
   // routed GEMMs slowed more than the shared GEMMs saved), so automatic means never.
   int shared_concurrent = -1;
-  // router: -1 automatic (the fused router whenever N_r <= 512), 0 the split
-  // router (scores GEMM, then softmax + top-k), 1 fused whenever supported
+  // router: 1 the fused router whenever supported (N_r <= 512, top_k <= 16),
+  // 0 the split router (scores GEMM, then softmax + top-k), -1 automatic = the
+  // split router. Measured on B200 (CUDA-graph steps, L2 flushed): 512-expert
+  // decode 172 us fused vs 148 us split, the 31-expert tiny layer 60 vs 43 us,
+  // DeepSeekMoE-small 2% slower fused, DeepSeek-V3 prefill within noise. The
+  // fused kernel's 128-token tile is scored by one cluster, whose CTAs each
+  // read all of x (one load pipeline each), and its per-token selection and
+  // merge run on few SMs, while the split kernels spread over the GPU and
+  // overlap their neighbours through programmatic dependent launch.
   int fused_router = -1;
   // seats per expert per forward (token dropping); 0: unlimited (dropless)
   int64_t capacity = 0;
@@ -192,7 +196,7 @@ Layout make_layout(const moe_plan* p, int64_t T) {
   Layout L{};
   const int64_t A = T * p->top_k;
   const int nsf = p->n_shared * p->f;
-  L.fused = p->fused_router != 0 && p->n_routed <= moe::kRtMaxExperts &&
+  L.fused = p->fused_router == 1 && p->n_routed <= moe::kRtMaxExperts &&
             p->top_k <= moe::kRtMaxTopK;
   L.lds = static_cast<int>(align_up(p->n_routed, 8));
   if (L.fused) {
@@ -1034,37 +1038,36 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   const CUtensorMap xdn[3] = {mHs, mW2s, mW2s};
   // the routed GEMMs leave the concurrent shared expert its SMs
   if (shared_sms > 0) L.grid_cap = p->num_sms - shared_sms;
-  // 5. grouped gate/up GEMM with the SiLU(gate) * up epilogue. With few rows
-  //    per expert (weight streaming) the single-CTA kernels run two CTAs per
-  //    SM (two load pipelines per SM) on narrow tiles of 64 rows: 32 output
-  //    columns (64 with one CTA per SM), so that the grid's last wave is short,
-  //    and 64-row boxes of the grouped rows, so that more stages fit.
+  // 5. grouped gate/up GEMM with the SiLU(gate) * up epilogue. Automatically
+  //    every single-CTA routed GEMM uses the widest tile (128 rows x 256
+  //    accumulator columns, one CTA per SM), also when the groups hold a few
+  //    rows and the GEMM streams weights: on B200 one tcgen05.mma instruction
+  //    occupies the issuing thread about 128 cycles whatever its size, so an
+  //    N=256 MMA moves twice the weight bytes per cycle of an N=128 one.
+  //    Measured on the 512-expert decode step: gate/up 64 us with these tiles,
+  //    70 us with 64x128 tiles, 72 us with 64x64 tiles at two CTAs per SM, 88
+  //    us with 64x256 tiles at two CTAs per SM. Narrower or shorter tiles and
+  //    two CTAs per SM stay available as options.
   const bool single_gu = !routed_pair_swiglu && !merge_gu;
   const bool single_dn = !routed_pair && !merge_dn;
-  const bool streaming = rows_per_expert < 32;
-  const bool occ2_gu =
-      single_gu && (p->ctas_per_sm == 2 || (p->ctas_per_sm == 0 && streaming));
-  const bool occ2_dn =
-      single_dn && (p->ctas_per_sm == 2 || (p->ctas_per_sm == 0 && streaming));
+  const bool occ2_gu = single_gu && p->ctas_per_sm == 2;
+  const bool occ2_dn = single_dn && p->ctas_per_sm == 2;
   int gu_cols = 128;   // output columns of a gate/up tile
-  if (single_gu)
-    gu_cols = p->swiglu_tile_cols != 0 ? p->swiglu_tile_cols
-                                       : (streaming ? (occ2_gu ? 32 : 64) : 128);
+  if (single_gu && p->swiglu_tile_cols != 0) gu_cols = p->swiglu_tile_cols;
   int dn_cols = 256;   // output columns of a down tile
-  if (single_dn)
-    dn_cols = p->down_tile_cols != 0 ? p->down_tile_cols : (streaming && occ2_dn ? 128 : 256);
+  if (single_dn && p->down_tile_cols != 0) dn_cols = p->down_tile_cols;
   const bool narrow_gu = gu_cols < 128;
-  const bool short_gu =
-      single_gu && (p->tile_rows == 64 || (p->tile_rows == 0 && streaming));
-  const bool short_dn =
-      single_dn && (p->tile_rows == 64 || (p->tile_rows == 0 && streaming));
+  const bool short_gu = single_gu && p->tile_rows == 64;
+  const bool short_dn = single_dn && p->tile_rows == 64;
   const int max_mtiles64 = static_cast<int>((A + 63) / 64 + (A < nr ? A : nr));
   // 128-row single-CTA routed GEMMs in the weight-streaming regime run the
   // tiles of experts with several m-blocks (tensor-heavy: each weight tile is
   // reused through L2) spread evenly among the weight-streaming experts' tiles,
   // so that tensor and HBM work overlap instead of alternating
+  // (not when every group streams: decode 161.8 vs 163.7 us without it)
   const bool interleave =
-      p->interleave == 1 || (p->interleave == -1 && rows_per_expert < 192);
+      p->interleave == 1 ||
+      (p->interleave == -1 && rows_per_expert >= 32 && rows_per_expert < 192);
   CUtensorMap mXp64, mH64;
   if ((short_gu && !make_map(&mXp64, xperm, 0, A, d, 64)) ||
       (short_dn && !make_map(&mH64, hidden, 0, A, f, 64)))

@@ -48,6 +48,10 @@ class LayerShape:
     def with_tokens(self, T: int) -> "LayerShape":
         return replace(self, T=T)
 
+    def with_experts(self, n_routed: int) -> "LayerShape":
+        """The same layer with fewer (or more) routed experts, top_k kept."""
+        return replace(self, n_routed=max(n_routed, self.top_k))
+
 
 # The layer shapes the pages describe, named by what they are.
 WORKLOADS: Dict[str, LayerShape] = {

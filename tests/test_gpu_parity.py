@@ -64,7 +64,7 @@ def test_fused_router_edges(case):
     tokens = None
     if T > 2048:
         tokens = np.sort(np.random.default_rng(3).choice(T, size=512, replace=False))
-    res = full_parity(inp, shape, tokens=tokens)
+    res = full_parity(inp, shape, tokens=tokens, fused_router=1)
     names = res["layer"].plan.kernel_names()
     assert "route_fused" in names and "router_gemm" not in names, names
     assert ("route_scan" in names) == (name == "fr_scan_not_folded"), names
@@ -76,8 +76,8 @@ SPLIT_ROUTER_CASES = ["one_token", "ragged_17", "k_equals_n", "wide_router", "sk
 @pytest.mark.parametrize("case", [c for c in SMALL if c[0] in SPLIT_ROUTER_CASES],
                          ids=[c[0] for c in SMALL if c[0] in SPLIT_ROUTER_CASES])
 def test_split_router_kernels(case):
-    # the two-kernel router (split-K scores GEMM, then softmax + top-k), which
-    # layers with more than 512 experts use, forced on shapes the fused one covers
+    # the two-kernel router (split-K scores GEMM, then softmax + top-k), the
+    # default, asked for explicitly on shapes the fused one also covers
     name, T, d, f, n, k, ns, renorm, bias = case
     shape = LayerShape(name, T, d, f, n, k, ns, renorm, bias)
     inp = make_layer_inputs(shape, seed=1, device="cuda")
@@ -626,7 +626,7 @@ def test_inconsistent_routing_state_is_reported_not_written_out_of_range():
     shape = LayerShape("one_tile", 100, 256, 128, 24, 4, 1, True, "none")
     inp = make_layer_inputs(shape, seed=31, device="cuda")
     layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
-                     shape.renorm, inp, device="cuda")
+                     shape.renorm, inp, device="cuda", fused_router=1)
     ref = layer(inp["x"]).clone()
     torch.cuda.synchronize()
     assert layer.device_status() == 0

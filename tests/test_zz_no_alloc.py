@@ -29,19 +29,21 @@ def _ptrs(inp):
             for k in ("x", "W_g", "W1", "W3", "W2", "W1s", "W3s", "W2s")]
 
 
-def _layer(shape, inp):
+def _layer(shape, inp, **options):
     return MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
-                    shape.renorm, inp, bias=inp["bias"], device="cuda")
+                    shape.renorm, inp, bias=inp["bias"], device="cuda", **options)
 
 
 # the decode shape runs its shared expert on the plan's side stream; the tiny one too,
-# with a different routing kernel configuration
+# with a different routing kernel configuration; both with the split router (the
+# default) and the fused one (whose scan ticket lives in the scratch)
+@pytest.mark.parametrize("fused", [-1, 1], ids=["split_router", "fused_router"])
 @pytest.mark.parametrize("name", ["decode_t128_d2048_f512_e512k10_s1",
                                   "tiny_t256_d128_f64_e31k7_s1"])
-def test_noalloc_forward_matches_workspace_forward_twice(name):
+def test_noalloc_forward_matches_workspace_forward_twice(name, fused):
     shape = WORKLOADS[name]
     inp = make_layer_inputs(shape, seed=0, device="cuda")
-    layer = _layer(shape, inp)
+    layer = _layer(shape, inp, fused_router=fused)
     ref = layer(inp["x"]).clone()                    # regular entry point, caller workspace
     routing_before = layer.routing()
     torch.cuda.synchronize()
