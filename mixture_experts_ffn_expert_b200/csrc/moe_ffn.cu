@@ -186,8 +186,7 @@ moe::RouterParams router_shape(const moe_plan* p, int64_t T, size_t* smem) {
   // at least kRouterMinSmem so that two router CTAs never share an SM: each
   // allocates tensor memory and then waits at cluster barriers, and two
   // clusters interleaved on two SMs could otherwise wait on each other
-  const size_t bytes = p->top_k <= 8 ? moe::router_smem_bytes<8>(r.ring_bytes, nr)
-                                      : moe::router_smem_bytes<16>(r.ring_bytes, nr);
+  const size_t bytes = moe::router_smem_bytes(r.ring_bytes, nr);
   *smem = bytes < kRouterMinSmem ? kRouterMinSmem : bytes;
   return r;
 }
@@ -525,7 +524,10 @@ int set_kernel_attributes() {
     if (e != cudaSuccess)
       return fail(MOE_CUDA_ERROR, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
   const int rsm = 227 * 1024;
-  const cudaError_t er[2] = {cudaFuncSetAttribute(moe::route_fused_kernel<8>, attr, rsm),
+  const cudaError_t er[5] = {cudaFuncSetAttribute(moe::route_fused_kernel<1>, attr, rsm),
+                             cudaFuncSetAttribute(moe::route_fused_kernel<2>, attr, rsm),
+                             cudaFuncSetAttribute(moe::route_fused_kernel<4>, attr, rsm),
+                             cudaFuncSetAttribute(moe::route_fused_kernel<8>, attr, rsm),
                              cudaFuncSetAttribute(moe::route_fused_kernel<16>, attr, rsm)};
   for (cudaError_t e : er)
     if (e != cudaSuccess)
@@ -551,7 +553,12 @@ cudaError_t launch_router(const Layout& Lw, const moe::RouterParams& rt, const C
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  if (rt.top_k <= 8) return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<8>, mX, mWg, rt);
+  // scores per lane of the selection: N_r <= 32 * NPL
+  const int npl = (rt.n_routed + 31) / 32;
+  if (npl <= 1) return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<1>, mX, mWg, rt);
+  if (npl <= 2) return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<2>, mX, mWg, rt);
+  if (npl <= 4) return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<4>, mX, mWg, rt);
+  if (npl <= 8) return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<8>, mX, mWg, rt);
   return cudaLaunchKernelEx(&cfg, moe::route_fused_kernel<16>, mX, mWg, rt);
 }
 
