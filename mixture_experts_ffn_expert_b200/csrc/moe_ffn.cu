@@ -97,15 +97,15 @@ struct moe_plan {
   // SMs the layer took 7.09 ms per step against 6.19 ms inline (the capped
   // routed GEMMs slowed more than the shared GEMMs saved), so automatic means never.
   int shared_concurrent = -1;
-  // router: 1 the fused router whenever supported (N_r <= 512, top_k <= 16),
+  // router: 1 the fused router whenever supported (N_r <= 512, top_k <= 32),
   // 0 the split router (scores GEMM, then softmax + top-k), -1 automatic = the
   // split router. Measured on B200 (CUDA-graph steps, L2 flushed): 512-expert
-  // decode 172 us fused vs 148 us split, the 31-expert tiny layer 60 vs 43 us,
-  // DeepSeekMoE-small 2% slower fused, DeepSeek-V3 prefill within noise. The
-  // fused kernel's 128-token tile is scored by one cluster, whose CTAs each
-  // read all of x (one load pipeline each), and its per-token selection and
-  // merge run on few SMs, while the split kernels spread over the GPU and
-  // overlap their neighbours through programmatic dependent launch.
+  // decode 162 us fused vs 137 us split, the 31-expert tiny layer 62 vs 43 us,
+  // DeepSeekMoE-small and coarse 3-4% slower fused, DeepSeek-V3 prefill within
+  // noise. The fused kernel takes about the split kernels' summed time, but a
+  // 128-token tile is one cluster, so small batches select on few SMs, and a
+  // cluster of large-shared-memory CTAs cannot start early beside its
+  // predecessor the way the small split kernels do.
   int fused_router = -1;
   // seats per expert per forward (token dropping); 0: unlimited (dropless)
   int64_t capacity = 0;
