@@ -71,10 +71,16 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the GEMM kernel's code (comments and blank lines removed, so that
+    a comment-only edit keeps the committed counters valid)."""
     h = hashlib.sha256()
     for name in ("gemm_sm100.cuh", "ptx_sm100.cuh"):
-        with open(os.path.join(ROOT, "mixture_experts_ffn_expert_b200", "csrc", name), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "mixture_experts_ffn_expert_b200", "csrc", name),
+                  encoding="utf-8") as fh:
+            for line in fh:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode("utf-8") + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -109,7 +109,7 @@ struct GemmParams {
 // B200 showed one pipeline of 8 KB stages stuck near 30 GB/s per SM (the
 // producer thread's issue cost per stage) and two near 6 TB/s in all; with the
 // GEMM's 24-48 KB stages one pipeline already streams 6.5 TB/s, and the routed
-// GEMMs are instead bound by the SM's MMA issue rate (about 128 cycles per
+// GEMMs are instead bound by the SM's MMA issue rate (about 95 cycles per
 // tcgen05.mma instruction at any size), which both CTAs share - so OCC = 2 is
 // an option, not the default.
 template <int BN, int TM = 128, int OCC = 1>

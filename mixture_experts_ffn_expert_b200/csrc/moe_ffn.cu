@@ -1049,7 +1049,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   //    every single-CTA routed GEMM uses the widest tile (128 rows x 256
   //    accumulator columns, one CTA per SM), also when the groups hold a few
   //    rows and the GEMM streams weights: on B200 one tcgen05.mma instruction
-  //    occupies the issuing thread about 128 cycles whatever its size, so an
+  //    occupies the issuing thread about 95 cycles whatever its size, so an
   //    N=256 MMA moves twice the weight bytes per cycle of an N=128 one.
   //    Measured on the 512-expert decode step: gate/up 64 us with these tiles,
   //    70 us with 64x128 tiles, 72 us with 64x64 tiles at two CTAs per SM, 88
