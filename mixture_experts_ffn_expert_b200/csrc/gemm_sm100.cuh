@@ -96,14 +96,14 @@ struct GemmParams {
 };
 
 // Single-CTA kernel shapes: BN accumulator columns per tile (MMA N), TM rows
-// per tile. BN = 256, TM = 128 is the default. Narrower tiles - SwiGLU BN = 128
-// (64 gate + 64 up columns, 64 output columns) or BN = 64 (32 output columns),
-// plain BN = 128 - carry fewer weight bytes per tile, so that weight-streaming
-// launches with few rows per expert split into more, shorter tiles and the
-// last wave of the grid is less empty. TM = 64 (M=64 MMAs,
-// 64-row boxes of the grouped rows) halves the grouped-row bytes per stage, so
-// that the same shared memory holds more stages, i.e. more weight bytes in
-// flight per SM, when the groups are small anyway.
+// per tile. BN = 256, TM = 128 is the default in every regime: each MMA
+// instruction then carries the most weight bytes, and on B200 an instruction
+// costs about the same issue time whatever its size. The options: narrower
+// tiles - SwiGLU BN = 128 (64 gate + 64 up columns, 64 output columns) or
+// BN = 64 (32 output columns), plain BN = 128 - split a launch into more,
+// shorter tiles; TM = 64 (M=64 MMAs, 64-row boxes of the grouped rows) halves
+// the grouped-row bytes per stage, so that the same shared memory holds more
+// stages.
 // OCC = 2 CTAs resident per SM, each with half the ring and half the TMEM:
 // two independent load -> MMA pipelines per SM. A load-only measurement on
 // B200 showed one pipeline of 8 KB stages stuck near 30 GB/s per SM (the

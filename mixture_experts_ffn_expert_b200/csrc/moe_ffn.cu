@@ -437,8 +437,7 @@ bool launch_gemm(Launcher& L, cudaStream_t s, const char* name, const CUtensorMa
   return L.end(name, s);
 }
 
-// The same launch with one or two CTAs per SM (two: the weight-streaming
-// regime, where two independent load pipelines per SM move more bytes).
+// The same launch with one or two resident CTAs per SM (MOE_OPTION_CTAS_PER_SM).
 template <int MODE, int BN = 256, int TM = 128>
 bool launch_gemm_occ(bool two, Launcher& L, cudaStream_t s, const char* name,
                      const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
