@@ -151,6 +151,11 @@ int moe_last_status(void);
  *   ring and half the tensor memory (two independent pipelines per SM; measured
  *   no faster on B200, where the SM's MMA issue rate, shared by both, is the
  *   limit); 1 and 0 (default): one CTA per SM with the whole ring.
+ * MOE_OPTION_GATHER_ROWS: 1 lets the routed gate/up GEMM, when it runs one CTA
+ *   per tile, gather its rows from x through the permutation (its producer
+ *   warps copy them into the pipeline with cp.async), so that the permutation
+ *   kernel writes no permuted row copies; 0 and -1 (default) keep the copies
+ *   and the tensor-map loads of them. The same results bit for bit.
  * MOE_OPTION_TEST_WAIT_TIMEOUT: test hook for the failure path, not for normal
  *   use. Value 1 arms it for the next forward only: if that forward runs the
  *   routed gate/up GEMM on the one-CTA-per-tile kernel, one CTA withholds the
@@ -172,6 +177,7 @@ enum {
   MOE_OPTION_INTERLEAVE = 11,
   MOE_OPTION_CTAS_PER_SM = 12,
   MOE_OPTION_DOWN_TILE_COLS = 13,
+  MOE_OPTION_GATHER_ROWS = 14,
   MOE_OPTION_TEST_WAIT_TIMEOUT = 100
 };
 int moe_plan_set_option(moe_plan_t plan, int option, int64_t value);

@@ -35,6 +35,7 @@ MOE_OPTION_TILE_ROWS = 10
 MOE_OPTION_INTERLEAVE = 11
 MOE_OPTION_CTAS_PER_SM = 12
 MOE_OPTION_DOWN_TILE_COLS = 13
+MOE_OPTION_GATHER_ROWS = 14
 MOE_OPTION_TEST_WAIT_TIMEOUT = 100
 
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_INVALID_CONFIG", 2: "MOE_INVALID_ARG",

@@ -93,7 +93,37 @@ struct GemmParams {
   // loads of its first stage, so that its MMA warp's bounded wait expires and
   // the kernel takes its timeout path (status word, drain, TMEM release).
   int test_withhold;
+  // Optional row gather for the grouped A operand (single-CTA kernel, grouped
+  // launches without an extra problem): grouped row g of the A operand is row
+  // gather_src[g] of gather_x (T rows of gather_ld_vec 16-byte vectors),
+  // copied by the producer warps with cp.async instead of a TMA box of a
+  // permuted copy; nullptr: A through its tensor map.
+  const uint4* gather_x;
+  const int* gather_src;
+  int gather_ld_vec;
+  int gather_T;              // rows of gather_x: a source row outside [0, T) reads zeros
 };
+
+// 16-byte copy global -> shared through the load/store path; src_bytes 0
+// fills the 16 bytes with zeros (rows past a group, columns past K).
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+// Arrive on `bar` once this thread's earlier cp.async copies have landed (the
+// arrival is counted in the barrier's expected count, not added to it).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+// Order this thread's view of generic-proxy shared-memory writes (cp.async)
+// before its later async-proxy operations (tcgen05.mma reading shared memory).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
 // Single-CTA kernel shapes: BN accumulator columns per tile (MMA N), TM rows
 // per tile. BN = 256, TM = 128 is the default in every regime: each MMA
@@ -263,7 +293,8 @@ __global__ void __launch_bounds__(kGemmThreads, OCC)
   pdl_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&full_bar[s]), 1);
+      // with the row gather a stage also waits for the 32 copying lanes
+      mbar_init(smem_u32(&full_bar[s]), P.gather_x ? 1 + 32 : 1);
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
     for (int b = 0; b < kNumAcc; ++b) {
@@ -343,6 +374,17 @@ __global__ void __launch_bounds__(kGemmThreads, OCC)
       const CUtensorMap* mB1 = ex ? &tmB1x : &tmB1;
       int kb_begin, kb_end;
       kb_range(tc, ex, kb_begin, kb_end);
+      // row gather: lane l copies 16-byte chunk l % 8 of the tile's rows
+      // l / 8 + 4 j; their source rows are looked up once per tile
+      // (-1: past the group, zero-filled)
+      const bool gth = MODE == kEpiSwiGLU && P.gather_x != nullptr && !ex;
+      int srow[TM / 4];
+#pragma unroll
+      for (int j = 0; j < TM / 4; ++j) {
+        const int r = (lane >> 3) + 4 * j;
+        const int src = (gth && r < tc.rows) ? __ldg(P.gather_src + tc.row0 + r) : -1;
+        srow[j] = static_cast<unsigned>(src) < static_cast<unsigned>(P.gather_T) ? src : -1;
+      }
       for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
         if ((it & 1) != pid) continue;
         if (P.test_withhold && blockIdx.x == 0 && it == 0) continue;   // test hook
@@ -359,8 +401,8 @@ __global__ void __launch_bounds__(kGemmThreads, OCC)
           const uint32_t a_dst = smem_u32(smem + size_t(s) * kStageBytes);
           const uint32_t b_dst = a_dst + kABytes;
           const int k0 = kb * kBK;
-          mbar_arrive_expect_tx(fb, kStageBytes);
-          tma_load_2d(a_dst, mA, fb, k0, tc.row0);
+          mbar_arrive_expect_tx(fb, gth ? kStageBytes - kABytes : kStageBytes);
+          if (!gth) tma_load_2d(a_dst, mA, fb, k0, tc.row0);
           // SwiGLU: BN/2 rows of W1 then the same rows of W3; plain: BN rows
           // of the one weight in 128-row boxes (one or two)
           const CUtensorMap* b1 = MODE == kEpiSwiGLU ? mB1 : mB0;
@@ -376,11 +418,32 @@ __global__ void __launch_bounds__(kGemmThreads, OCC)
             if (kTwoBoxes) tma_load_3d(b_hi, b1, fb, k0, n1, z);
           }
         }
+        if (gth) {
+          // the A box in the layout the tensor map would give it: row r at
+          // r * 128 bytes, 16-byte chunk c at (c ^ (r % 8)) * 16 (128-byte swizzle)
+          const uint32_t a_dst = smem_u32(smem + size_t(s) * kStageBytes);
+          const int c = lane & 7;
+          const int vec = kb * (kBK / 8) + c;            // 16-byte vector of the x row
+          const bool col_ok = vec < P.gather_ld_vec;
+#pragma unroll
+          for (int j = 0; j < TM / 4; ++j) {
+            const int r = (lane >> 3) + 4 * j;
+            const bool ok_r = srow[j] >= 0 && col_ok;
+            const uint4* src = ok_r ? P.gather_x + static_cast<long long>(srow[j]) * P.gather_ld_vec + vec
+                                    : P.gather_x;
+            cp_async_16(a_dst + static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4)), src,
+                        ok_r ? 16u : 0u);
+          }
+          cp_async_arrive_noinc(smem_u32(&full_bar[s]));
+        } else if (MODE == kEpiSwiGLU && P.gather_x) {
+          mbar_arrive(smem_u32(&full_bar[s]));      // A came by TMA: the lanes' arrivals
+        }
         __syncwarp();
         issued_mask |= 1u << s;
         issued_par = (issued_par & ~(1u << s)) | (ph << s);
       }
     }
+    if (P.gather_x) cp_async_wait_all();          // this lane's row copies have landed
     if (!ok && lane == 0) {
       // give the copies already issued a bounded chance to land before teardown
       for (int i = 0; i < kStages; ++i)
@@ -415,6 +478,7 @@ __global__ void __launch_bounds__(kGemmThreads, OCC)
         if (!ok) break;
         tc_fence_after_sync();
         if (lane == 0) {
+          if (P.gather_x) fence_proxy_async_smem();   // rows written by cp.async
           const uint32_t a_base = smem_u32(smem + size_t(s) * kStageBytes);
           const uint32_t b_base = a_base + kABytes;
 #pragma unroll

@@ -92,6 +92,9 @@ struct moe_plan {
   int ctas_per_sm = 0;
   // output columns of a single-CTA routed down tile: 0 automatic (256), 128 or 256
   int down_tile_cols = 0;
+  // the single-CTA routed gate/up GEMM gathers its rows from x through the
+  // permutation (no row copies): 1 on, 0 and -1 (automatic) off
+  int gather_rows = -1;
   // shared expert beside weight-streaming routed GEMMs: -1 automatic, 0 never, 1 always.
   // Measured on B200 (DeepSeek-V3-shaped prefill): beside the routed GEMMs on 16
   // SMs the layer took 7.09 ms per step against 6.19 ms inline (the capped
@@ -720,6 +723,10 @@ int moe_plan_set_option(moe_plan_t p, int option, int64_t value) {
         return fail(MOE_INVALID_ARG, "tile rows must be 0, 64 or 128");
       p->tile_rows = static_cast<int>(value);
       return MOE_OK;
+    case MOE_OPTION_GATHER_ROWS:
+      if (value < -1 || value > 1) return fail(MOE_INVALID_ARG, "gather_rows must be -1, 0 or 1");
+      p->gather_rows = static_cast<int>(value);
+      return MOE_OK;
     case MOE_OPTION_DOWN_TILE_COLS:
       if (value != 0 && value != 128 && value != 256)
         return fail(MOE_INVALID_ARG, "down tile columns must be 0, 128 or 256");
@@ -1008,26 +1015,6 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
                0, main_st, chunk_counts, Lw.n_base, nr, counts);
     if (!L.end("route_scan", main_st)) return L.status;
   }
-  // 4. offsets + m-tile prefix, stable permutation, 16-byte row copies (with a
-  //    seat limit, only each expert's first `capacity` pairs get rows)
-  {
-    const size_t smem = size_t(moe::kMaxRouted + nr) * 4 + size_t(2) * Lw.tpc * k * 4;
-    // split the row copy into column slices of at least 32 vectors so that
-    // about four blocks per SM copy (one block per chunk leaves most SMs with
-    // one or two resident blocks, too few loads in flight)
-    int slices = (4 * p->num_sms) / Lw.n_chunks;
-    const int max_slices = d / 8 / 32;
-    if (slices > max_slices) slices = max_slices;
-    if (slices < 1) slices = 1;
-    L.begin("route_scatter", main_st);
-    launch_pdl(moe::route_scatter_kernel, dim3(Lw.n_chunks, slices), dim3(moe::kRouteThreads), smem,
-               main_st, (const int*)idx, (const int*)chunk_counts, Lw.n_base,
-               (const int*)sub_base, Lw.subs_per_base, Lw.sub_tokens, (const int*)counts,
-               static_cast<int>(T), k, nr, Lw.tpc, Lw.n_chunks, moe::kBM, seat_limit,
-               reinterpret_cast<const uint4*>(x), d / 8, reinterpret_cast<uint4*>(xperm),
-               perm_src, inv_pos, offsets, mtiles, mtiles2, mtiles64, mt_hot, mt_cold, status);
-    if (!L.end("route_scatter", main_st)) return L.status;
-  }
   const int max_mtiles = static_cast<int>((A + 127) / 128 + (A < nr ? A : nr));
   const int max_mtiles2 = static_cast<int>((A + 255) / 256 + (A < nr ? A : nr));
   const bool routed_pair_swiglu = rows_per_expert >= p->pair_min_rows_swiglu;
@@ -1040,6 +1027,31 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   const bool merge_ok = p->n_shared > 0 && !shared_forked && !shared_pair && p->merge_shared == 1;
   const bool merge_gu = merge_ok && !routed_pair_swiglu;
   const bool merge_dn = merge_gu && !routed_pair;
+  // The single-CTA gate/up GEMM can gather its rows from x itself (through
+  // perm_src), so that the permutation kernel writes no row copies.
+  const bool gather_rows = p->gather_rows == 1 && !routed_pair_swiglu && !merge_gu;
+  // 4. offsets + m-tile prefix, stable permutation, 16-byte row copies (with a
+  //    seat limit, only each expert's first `capacity` pairs get rows; none
+  //    when the gate/up GEMM gathers them)
+  {
+    const size_t smem = size_t(moe::kMaxRouted + nr) * 4 + size_t(2) * Lw.tpc * k * 4;
+    // split the row copy into column slices of at least 32 vectors so that
+    // about four blocks per SM copy (one block per chunk leaves most SMs with
+    // one or two resident blocks, too few loads in flight)
+    int slices = (4 * p->num_sms) / Lw.n_chunks;
+    const int max_slices = d / 8 / 32;
+    if (slices > max_slices) slices = max_slices;
+    if (slices < 1 || gather_rows) slices = 1;
+    L.begin("route_scatter", main_st);
+    launch_pdl(moe::route_scatter_kernel, dim3(Lw.n_chunks, slices), dim3(moe::kRouteThreads), smem,
+               main_st, (const int*)idx, (const int*)chunk_counts, Lw.n_base,
+               (const int*)sub_base, Lw.subs_per_base, Lw.sub_tokens, (const int*)counts,
+               static_cast<int>(T), k, nr, Lw.tpc, Lw.n_chunks, moe::kBM, seat_limit,
+               reinterpret_cast<const uint4*>(x), d / 8,
+               gather_rows ? static_cast<uint4*>(nullptr) : reinterpret_cast<uint4*>(xperm),
+               perm_src, inv_pos, offsets, mtiles, mtiles2, mtiles64, mt_hot, mt_cold, status);
+    if (!L.end("route_scatter", main_st)) return L.status;
+  }
   const CUtensorMap xgu[3] = {mX, mW1s, mW3s};
   const CUtensorMap xdn[3] = {mHs, mW2s, mW2s};
   // the routed GEMMs leave the concurrent shared expert its SMs
@@ -1094,6 +1106,12 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     if (!routed_pair_swiglu) {
       g.test_withhold = p->test_withhold;
       p->test_withhold = 0;
+    }
+    if (gather_rows) {
+      g.gather_x = reinterpret_cast<const uint4*>(x);
+      g.gather_src = perm_src;
+      g.gather_ld_vec = d / 8;
+      g.gather_T = static_cast<int>(T);
     }
     if (merge_gu) {
       g.x_tiles = shared_mt * ((nsf + 127) / 128);

@@ -436,7 +436,8 @@ __global__ void __launch_bounds__(kRouteThreads)
   const int span = (d_vec + gridDim.y - 1) / gridDim.y;
   const int v_begin = blockIdx.y * span;
   const int v_end = min(d_vec, v_begin + span);
-  for (int tl = warp; tl < ntok; tl += kRouteThreads / 32) {
+  // (no copies when the gate/up GEMM gathers the rows itself: xperm null)
+  for (int tl = warp; xperm != nullptr && tl < ntok; tl += kRouteThreads / 32) {
     const uint4* src = x + static_cast<long long>(t0 + tl) * d_vec;
     const int* pos = s_pos + tl * top_k;
     for (int v0 = v_begin + lane; v0 < v_end; v0 += 32 * kCopyUnroll) {

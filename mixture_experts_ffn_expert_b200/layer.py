@@ -11,7 +11,7 @@ from typing import Dict, Optional
 import torch
 
 from .binding import (MOE_OPTION_BIAS_SELECTION_ONLY, MOE_OPTION_CAPACITY_FACTOR_PERMILLE,
-                      MOE_OPTION_CTAS_PER_SM, MOE_OPTION_DOWN_TILE_COLS,
+                      MOE_OPTION_CTAS_PER_SM, MOE_OPTION_DOWN_TILE_COLS, MOE_OPTION_GATHER_ROWS,
                       MOE_OPTION_EXPERT_CAPACITY, MOE_OPTION_FUSED_ROUTER,
                       MOE_OPTION_MERGE_SHARED, MOE_OPTION_PAIR_MIN_ROWS,
                       MOE_OPTION_INTERLEAVE, MOE_OPTION_SHARED_CONCURRENT,
@@ -36,8 +36,8 @@ class MoELayer:
     on token dropping; ``bias_selection_only`` makes the bias choose experts
     without entering the gates; the other options (``fused_router``,
     ``swiglu_tile_cols``, ``tile_rows``, ``interleave``, ``shared_concurrent``,
-    ``ctas_per_sm``, ``down_tile_cols`` among them) only select kernels, tile orders
-    or streams.
+    ``ctas_per_sm``, ``down_tile_cols``, ``gather_rows`` among them) only select
+    kernels, tile orders or streams.
     """
 
     def __init__(self, d: int, f: int, n_routed: int, top_k: int, n_shared: int,
@@ -50,7 +50,8 @@ class MoELayer:
                  swiglu_tile_cols: Optional[int] = None,
                  shared_concurrent: Optional[int] = None,
                  tile_rows: Optional[int] = None, interleave: Optional[int] = None,
-                 ctas_per_sm: Optional[int] = None, down_tile_cols: Optional[int] = None):
+                 ctas_per_sm: Optional[int] = None, down_tile_cols: Optional[int] = None,
+                 gather_rows: Optional[int] = None):
         dev = torch.device(device) if device is not None else torch.device("cuda")
         if dev.type == "cuda" and dev.index is None:
             dev = torch.device("cuda", torch.cuda.current_device())
@@ -79,6 +80,8 @@ class MoELayer:
             self.plan.set_option(MOE_OPTION_CTAS_PER_SM, ctas_per_sm)
         if down_tile_cols is not None:
             self.plan.set_option(MOE_OPTION_DOWN_TILE_COLS, down_tile_cols)
+        if gather_rows is not None:
+            self.plan.set_option(MOE_OPTION_GATHER_ROWS, gather_rows)
         # seats per expert per forward (token dropping); None or 0: dropless
         if capacity and capacity_factor:
             raise MoEError(2, "give either capacity or capacity_factor, not both")

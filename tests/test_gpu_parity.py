@@ -178,6 +178,40 @@ def test_two_ctas_per_sm_routed_gemms(shape, tile_rows, cols, dcols):
     assert torch.equal(outs[0], outs[1])
 
 
+GATHER_CASES = [
+    # name, T, d, f, N_r, k, N_s, renorm, bias, options
+    ("gather_default_tiles", 700, 256, 192, 8, 2, 1, True, "none", {}),
+    ("gather_k_tail", 200, 200, 64, 100, 5, 1, True, "normal_var0.5", {}),           # d = 3*64 + 8
+    ("gather_rows64", 600, 384, 328, 6, 2, 1, True, "none", {"tile_rows": 64}),     # f tail of 8
+    ("gather_cols32", 96, 256, 128, 64, 6, 1, True, "zipf1.1",
+     {"swiglu_tile_cols": 32, "tile_rows": 64}),
+    ("gather_two_ctas", 1100, 256, 192, 8, 2, 0, False, "normal_var0.5", {"ctas_per_sm": 2}),
+    ("gather_dropping", 512, 128, 64, 16, 4, 1, True, "zipf1.1", {"capacity": 40}),
+]
+
+
+@pytest.mark.parametrize("case", GATHER_CASES, ids=[c[0] for c in GATHER_CASES])
+def test_gate_up_gathers_rows_from_x(case):
+    # the gate/up GEMM's producer warps gather the grouped rows from x through
+    # the permutation (no permuted copy): the same bits as the copy path, and
+    # parity with the oracle
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    name, T, d, f, n, k, ns, renorm, bias, opts = case
+    shape = LayerShape(name, T, d, f, n, k, ns, renorm, bias)
+    inp = make_layer_inputs(shape, seed=29, device="cuda")
+    opts = dict(opts, pair_min_rows=1 << 40)
+    full_parity(inp, shape, gather_rows=1, **opts)
+    outs = []
+    for g in (0, 1):
+        layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
+                         shape.renorm, inp, bias=inp["bias"], device="cuda", gather_rows=g,
+                         **opts)
+        outs.append(layer(inp["x"]).clone())
+        torch.cuda.synchronize()
+        assert layer.device_status() == 0
+    assert torch.equal(outs[0], outs[1])
+
+
 PAIR_CASES = ["three_tokens", "ragged_17", "two_shared_raw", "ragged_tiles", "k_tail_not_64",
               "skewed_groups"]
 
