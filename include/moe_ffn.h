@@ -154,8 +154,9 @@ int moe_last_status(void);
  * MOE_OPTION_GATHER_ROWS: 1 lets the routed gate/up GEMM, when it runs one CTA
  *   per tile, gather its rows from x through the permutation (its producer
  *   warps copy them into the pipeline with cp.async), so that the permutation
- *   kernel writes no permuted row copies; 0 and -1 (default) keep the copies
- *   and the tensor-map loads of them. The same results bit for bit.
+ *   kernel writes no permuted row copies; 0 keeps the copies and the
+ *   tensor-map loads of them; -1 (default) gathers when the expected rows per
+ *   expert (T*top_k/N_r) are below 32 (decode). The same results bit for bit.
  * MOE_OPTION_TEST_WAIT_TIMEOUT: test hook for the failure path, not for normal
  *   use. Value 1 arms it for the next forward only: if that forward runs the
  *   routed gate/up GEMM on the one-CTA-per-tile kernel, one CTA withholds the
