@@ -1028,44 +1028,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   const bool merge_ok = p->n_shared > 0 && !shared_forked && !shared_pair && p->merge_shared == 1;
   const bool merge_gu = merge_ok && !routed_pair_swiglu;
   const bool merge_dn = merge_gu && !routed_pair;
-  // The single-CTA gate/up GEMM can gather its rows from x itself (through
-  // perm_src), so that the permutation kernel writes no row copies. Measured
-  // on B200: the 512-expert decode step 1-3% faster with it; the tensor-bound
-  // layers slower (the cp.async gather of a 16 KB A stage costs the producer
-  // warps far more than one TMA box: coarse +37%, DeepSeekMoE-small +8%); and
-  // DeepSeek-V3 prefill 7% slower although 16% fewer cycles, because the extra
-  // load traffic lowers the power-capped clock (1046 vs 1338 MHz). So
-  // automatically only below 32 expected rows per expert.
-  const bool gather_rows =
-      (p->gather_rows == 1 || (p->gather_rows == -1 && rows_per_expert < 32)) &&
-      !routed_pair_swiglu && !merge_gu;
-  // 4. offsets + m-tile prefix, stable permutation, 16-byte row copies (with a
-  //    seat limit, only each expert's first `capacity` pairs get rows; none
-  //    when the gate/up GEMM gathers them)
-  {
-    const size_t smem = size_t(moe::kMaxRouted + nr) * 4 + size_t(2) * Lw.tpc * k * 4;
-    // split the row copy into column slices of at least 32 vectors so that
-    // about four blocks per SM copy (one block per chunk leaves most SMs with
-    // one or two resident blocks, too few loads in flight)
-    int slices = (4 * p->num_sms) / Lw.n_chunks;
-    const int max_slices = d / 8 / 32;
-    if (slices > max_slices) slices = max_slices;
-    if (slices < 1 || gather_rows) slices = 1;
-    L.begin("route_scatter", main_st);
-    launch_pdl(moe::route_scatter_kernel, dim3(Lw.n_chunks, slices), dim3(moe::kRouteThreads), smem,
-               main_st, (const int*)idx, (const int*)chunk_counts, Lw.n_base,
-               (const int*)sub_base, Lw.subs_per_base, Lw.sub_tokens, (const int*)counts,
-               static_cast<int>(T), k, nr, Lw.tpc, Lw.n_chunks, moe::kBM, seat_limit,
-               reinterpret_cast<const uint4*>(x), d / 8,
-               gather_rows ? static_cast<uint4*>(nullptr) : reinterpret_cast<uint4*>(xperm),
-               perm_src, inv_pos, offsets, mtiles, mtiles2, mtiles64, mt_hot, mt_cold, status);
-    if (!L.end("route_scatter", main_st)) return L.status;
-  }
-  const CUtensorMap xgu[3] = {mX, mW1s, mW3s};
-  const CUtensorMap xdn[3] = {mHs, mW2s, mW2s};
-  // the routed GEMMs leave the concurrent shared expert its SMs
-  if (shared_sms > 0) L.grid_cap = p->num_sms - shared_sms;
-  // 5. grouped gate/up GEMM with the SiLU(gate) * up epilogue. Automatically
+  // Tile shapes of the routed GEMMs (step 5 and 6 below). Automatically
   //    every single-CTA routed GEMM uses the widest tile (128 rows x 256
   //    accumulator columns, one CTA per SM), also when the groups hold a few
   //    rows and the GEMM streams weights: on B200 one tcgen05.mma instruction
@@ -1095,6 +1058,49 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   const bool interleave =
       p->interleave == 1 ||
       (p->interleave == -1 && rows_per_expert >= 32 && rows_per_expert < 192);
+  // The single-CTA gate/up GEMM can gather its rows from x itself (through
+  // perm_src), so that the permutation kernel writes no row copies. Measured
+  // on B200: the 512-expert decode step 1-3% faster with it; the tensor-bound
+  // layers slower (the cp.async gather of a 16 KB A stage costs the producer
+  // warps far more than one TMA box: coarse +37%, DeepSeekMoE-small +8%); and
+  // DeepSeek-V3 prefill 7% slower although 16% fewer cycles, because the extra
+  // load traffic lowers the power-capped clock (1046 vs 1338 MHz). So
+  // automatically only below 32 expected rows per expert.
+  const bool gather_rows =
+      (p->gather_rows == 1 || (p->gather_rows == -1 && rows_per_expert < 32)) &&
+      !routed_pair_swiglu && !merge_gu;
+  // 4. offsets + m-tile prefix, stable permutation, 16-byte row copies (with a
+  //    seat limit, only each expert's first `capacity` pairs get rows; none
+  //    when the gate/up GEMM gathers them)
+  {
+    const size_t smem = size_t(moe::kMaxRouted + nr) * 4 + size_t(2) * Lw.tpc * k * 4;
+    // split the row copy into column slices of at least 32 vectors so that
+    // about four blocks per SM copy (one block per chunk leaves most SMs with
+    // one or two resident blocks, too few loads in flight)
+    int slices = (4 * p->num_sms) / Lw.n_chunks;
+    const int max_slices = d / 8 / 32;
+    if (slices > max_slices) slices = max_slices;
+    if (slices < 1 || gather_rows) slices = 1;
+    // the m-tile prefixes the routed GEMM launches below will read: 128-row
+    // tiles always, 256-row (CTA pair), 64-row and the two interleave classes
+    // only when used
+    const int pass_mask = 1 | ((routed_pair_swiglu || routed_pair) ? 2 : 0) |
+                          ((short_gu || short_dn) ? 4 : 0) | (interleave ? 8 | 16 : 0);
+    L.begin("route_scatter", main_st);
+    launch_pdl(moe::route_scatter_kernel, dim3(Lw.n_chunks, slices), dim3(moe::kRouteThreads), smem,
+               main_st, (const int*)idx, (const int*)chunk_counts, Lw.n_base,
+               (const int*)sub_base, Lw.subs_per_base, Lw.sub_tokens, (const int*)counts,
+               static_cast<int>(T), k, nr, Lw.tpc, Lw.n_chunks, moe::kBM, seat_limit,
+               reinterpret_cast<const uint4*>(x), d / 8,
+               gather_rows ? static_cast<uint4*>(nullptr) : reinterpret_cast<uint4*>(xperm),
+               perm_src, inv_pos, offsets, mtiles, mtiles2, mtiles64, mt_hot, mt_cold, pass_mask,
+               status);
+    if (!L.end("route_scatter", main_st)) return L.status;
+  }
+  const CUtensorMap xgu[3] = {mX, mW1s, mW3s};
+  const CUtensorMap xdn[3] = {mHs, mW2s, mW2s};
+  // the routed GEMMs leave the concurrent shared expert its SMs
+  if (shared_sms > 0) L.grid_cap = p->num_sms - shared_sms;
   CUtensorMap mXp64, mH64;
   if ((short_gu && !make_map(&mXp64, xperm, 0, A, d, 64)) ||
       (short_dn && !make_map(&mH64, hidden, 0, A, f, 64)))

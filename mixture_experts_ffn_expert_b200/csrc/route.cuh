@@ -298,7 +298,8 @@ __global__ void __launch_bounds__(kRouteThreads)
                          int* __restrict__ inv_pos, int* __restrict__ offsets_out,
                          int* __restrict__ mtiles_out, int* __restrict__ mtiles2_out,
                          int* __restrict__ mtiles4_out, int* __restrict__ mt_hot_out,
-                         int* __restrict__ mt_cold_out, int* __restrict__ status) {
+                         int* __restrict__ mt_cold_out, int pass_mask,
+                         int* __restrict__ status) {
   extern __shared__ int smem_i[];
   int* s_off = smem_i;                        // [kMaxRouted] expert offsets
   int* s_run = smem_i + kMaxRouted;           // [n_routed]
@@ -367,8 +368,10 @@ __global__ void __launch_bounds__(kRouteThreads)
     // tile_rows/2 rows (the 64-row tiles of weight-streaming launches), and the
     // tile_rows prefix split in two classes: experts with at least two m-tiles
     // (their tiles reuse a weight tile through L2: tensor-heavy) and the others
-    // (weight-streaming), which a launch may interleave
+    // (weight-streaming), which a launch may interleave; only the passes in
+    // pass_mask (bit i: pass i) are written
     for (int pass = 0; pass < 5; ++pass) {
+      if (!((pass_mask >> pass) & 1)) continue;        // uniform over the block
       const int rows = pass == 2 ? tile_rows / 2 : (pass == 1 ? tile_rows * 2 : tile_rows);
       int* dst = pass == 0 ? mtiles_out
                : pass == 1 ? mtiles2_out
