@@ -15,7 +15,7 @@ from parity import full_parity
 
 pytestmark = pytest.mark.gpu
 
-N_LAYERS = 12
+N_LAYERS = 40
 
 
 def _draw(seed):
