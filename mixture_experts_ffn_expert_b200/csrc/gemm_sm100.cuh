@@ -376,7 +376,7 @@ __global__ void __launch_bounds__(kGemmThreads, OCC)
       kb_range(tc, ex, kb_begin, kb_end);
       // row gather: lane l copies 16-byte chunk l % 8 of the tile's rows
       // l / 8 + 4 j; their source rows are looked up once per tile
-      // (-1: past the group, or a source row outside [0, T): not copied)
+      // (-1: past the group, or a source row outside [0, T): zero-filled)
       const bool gth = MODE == kEpiSwiGLU && P.gather_x != nullptr && !ex;
       int srow[TM / 4];
 #pragma unroll
@@ -425,19 +425,18 @@ __global__ void __launch_bounds__(kGemmThreads, OCC)
           const int c = lane & 7;
           const int vec = kb * (kBK / 8) + c;            // 16-byte vector of the x row
           const bool col_ok = vec < P.gather_ld_vec;
-          // rows past the group are left as they are: each output row depends
-          // only on its own A row, and the epilogue never stores those rows
-          // (an M=64 MMA does not even read rows 64..127); columns past K of
-          // a real row are zero-filled, as the weights' zero columns must not
-          // meet stale (possibly non-finite) values
+          // rows past the group and columns past K are zero-filled: every lane
+          // issues the same copies (measured faster on the decode step than
+          // skipping the rows past the group, whose per-lane branches cost more
+          // than the zero-fills they save)
 #pragma unroll
           for (int j = 0; j < TM / 4; ++j) {
-            if (srow[j] < 0) continue;
             const int r = (lane >> 3) + 4 * j;
-            const uint4* src = col_ok ? P.gather_x + static_cast<long long>(srow[j]) * P.gather_ld_vec + vec
-                                      : P.gather_x;
+            const bool ok_r = srow[j] >= 0 && col_ok;
+            const uint4* src = ok_r ? P.gather_x + static_cast<long long>(srow[j]) * P.gather_ld_vec + vec
+                                    : P.gather_x;
             cp_async_16(a_dst + static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4)), src,
-                        col_ok ? 16u : 0u);
+                        ok_r ? 16u : 0u);
           }
           cp_async_arrive_noinc(smem_u32(&full_bar[s]));
         } else if (MODE == kEpiSwiGLU && P.gather_x) {
