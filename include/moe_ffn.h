@@ -90,11 +90,16 @@ int moe_last_status(void);
  *   256 (fewer operand bytes per FLOP, fewer tiles). -1 (default) chooses per
  *   GEMM (wide for reductions of at least 4096 with at least 3 waves of
  *   tiles), 0 never, 1 always.
- * MOE_OPTION_MERGE_SHARED: when the shared expert runs on the main stream and a
- *   routed GEMM runs one CTA per tile, compute the matching shared GEMM as extra
- *   tiles of that same launch, spread evenly among the routed tiles (0, the
- *   default: never; 1: whenever possible). Off by default because the merged
- *   launches measured slower on B200 for the DeepSeek-style layer shapes.
+ * MOE_OPTION_MERGE_SHARED: when a routed GEMM runs one CTA per tile, compute
+ *   the matching shared GEMM as extra tiles of that same launch, spread evenly
+ *   among the routed tiles. -1 (the default): automatic - merged when the shared
+ *   expert is small (at most half the SMs' worth of 128 x 128 tiles, the decode
+ *   regime) and the routed tile options are at their defaults; a larger shared
+ *   expert runs as its own launches (merged, it measured slower on B200 for the
+ *   DeepSeek-V3 layer shape). 0: never (a small shared expert then runs on the
+ *   plan's side stream beside the routing). 1: whenever possible (a merged
+ *   launch uses the default routed tile shape). Results are the same bits
+ *   either way.
  * MOE_OPTION_EXPERT_CAPACITY: seats per expert per forward ("What is an
  *   'expert,' really?", glossary: capacity factor / token dropping, each expert
  *   has a seat limit per batch and overflow tokens are skipped). 0 (default):

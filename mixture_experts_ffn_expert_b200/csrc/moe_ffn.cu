@@ -73,11 +73,15 @@ struct moe_plan {
   long long pair_min_rows_swiglu = 1LL << 62;
   // CTA-pair tiles 512 accumulator columns wide: -1 automatic, 0 never, 1 always
   int wide_tiles = -1;
-  // shared expert as extra tiles of the routed single-CTA GEMM launches (when
-  // it is not forked onto the side stream): 0 never, 1 whenever possible. Off
-  // by default: measured on B200 it ran the merged launches at a lower clock
+  // shared expert as extra tiles of the routed single-CTA GEMM launches: -1
+  // automatic (a small shared expert, at most half the SMs' worth of tiles,
+  // when the routed launches use their default tiles), 0 never, 1 whenever
+  // possible. Measured on B200 (CUDA-graph steps, L2 flushed): the 512-expert
+  // decode step 133.1 us merged against 135.8 us with the shared expert forked
+  // onto the side stream, the 31-expert tiny layer 38.9 vs 43.6 us. A large
+  // shared expert stays separate: merged it ran the launches at a lower clock
   // under the power cap and lost 5% on the DeepSeek-V3 layer shape.
-  int merge_shared = 0;
+  int merge_shared = -1;
   // output columns of a single-CTA routed SwiGLU tile: 0 automatic (128), 32,
   // 64 or 128
   int swiglu_tile_cols = 0;
@@ -690,7 +694,8 @@ int moe_plan_set_option(moe_plan_t p, int option, int64_t value) {
       p->wide_tiles = static_cast<int>(value);
       return MOE_OK;
     case MOE_OPTION_MERGE_SHARED:
-      if (value < 0 || value > 1) return fail(MOE_INVALID_ARG, "merge_shared must be 0 or 1");
+      if (value < -1 || value > 1)
+        return fail(MOE_INVALID_ARG, "merge_shared must be -1, 0 or 1");
       p->merge_shared = static_cast<int>(value);
       return MOE_OK;
     case MOE_OPTION_TEST_WAIT_TIMEOUT:
@@ -860,10 +865,13 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   cudaStream_t main_st = L.st;
   // The shared SwiGLU (coefficient 1, outside the routing) is independent of
   // the routing. When it is small (at most half the SMs' worth of tiles, the
-  // decode regime) it runs on the plan's side stream, forked here and joined
-  // before the combine, so it hides behind the latency-bound routing kernels;
-  // a larger one would take SMs from the routing chain, so it runs inline on
-  // the main stream after the routed GEMMs instead.
+  // decode regime) it runs as extra tiles of the routed GEMM launches, which
+  // have room for them in their last wave, or else on the plan's side stream,
+  // forked here and joined before the combine, beside the latency-bound
+  // routing kernels (where it spills into the first routed GEMM wave's SMs and
+  // the join costs the combine its early launch); a larger one would take SMs
+  // from the routing chain, so it runs inline on the main stream after the
+  // routed GEMMs instead.
   const int shared_mt = static_cast<int>((T + 127) / 128);
   // seats per expert and the expected rows per expert group (a division: the
   // thresholds may be huge, and a product with N_r could overflow)
@@ -872,6 +880,15 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   const long long rows_per_expert = A / nr < seat_limit ? A / nr : seat_limit;
   const bool shared_small =
       p->n_shared > 0 && shared_mt * ((nsf + 127) / 128) <= p->num_sms / 2;
+  const bool routed_pair_swiglu = rows_per_expert >= p->pair_min_rows_swiglu;
+  const bool shared_pair = static_cast<long long>(T) >= p->pair_min_rows_swiglu;
+  // automatic merging leaves explicitly chosen routed tile shapes alone (a
+  // merged launch runs the default 128-row x 256-column tiles)
+  const bool default_tiles = (p->swiglu_tile_cols == 0 || p->swiglu_tile_cols == 128) &&
+                             p->tile_rows != 64 && p->ctas_per_sm != 2;
+  const bool merge_pref =
+      p->merge_shared == 1 || (p->merge_shared == -1 && shared_small && default_tiles);
+  const bool merge_small = shared_small && merge_pref && !routed_pair_swiglu && !shared_pair;
   // A larger shared expert runs beside the routed GEMMs when those stream
   // weights (few rows per expert: their tensor pipes idle most of the time):
   // forked at the start onto shared_sms SMs, sized so that its tensor-bound
@@ -887,9 +904,8 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     sm = sm < 8 ? 8 : (sm > p->num_sms / 4 ? p->num_sms / 4 : sm);
     shared_sms = sm;
   }
-  const bool shared_forked = shared_small || shared_sms > 0;
+  const bool shared_forked = (shared_small && !merge_small) || shared_sms > 0;
   cudaStream_t shared_st = shared_forked ? p->side : main_st;
-  const bool shared_pair = static_cast<long long>(T) >= p->pair_min_rows_swiglu;
   const int shared_mt2 = static_cast<int>((T + 255) / 256);
   auto launch_shared_gate_up = [&]() -> int {
     moe::GemmParams g{};
@@ -1018,14 +1034,13 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   }
   const int max_mtiles = static_cast<int>((A + 127) / 128 + (A < nr ? A : nr));
   const int max_mtiles2 = static_cast<int>((A + 255) / 256 + (A < nr ? A : nr));
-  const bool routed_pair_swiglu = rows_per_expert >= p->pair_min_rows_swiglu;
   const bool routed_pair = rows_per_expert >= p->pair_min_rows_plain;
   const int expected_mtiles2 = static_cast<int>((A + 255) / 256);
-  // An inline shared expert can instead run as extra dense tiles of the routed
-  // single-CTA launches, spread among the grouped tiles: tensor-bound shared
-  // tiles then overlap the weight streaming of small expert groups, and the
-  // shared GEMMs need no launches (and tails) of their own.
-  const bool merge_ok = p->n_shared > 0 && !shared_forked && !shared_pair && p->merge_shared == 1;
+  // A shared expert that is not forked can run as extra dense tiles of the
+  // routed single-CTA launches, spread among the grouped tiles: the shared
+  // GEMMs then need no launches (and tails) of their own, and a small one
+  // fills the routed launches' last waves.
+  const bool merge_ok = p->n_shared > 0 && !shared_forked && !shared_pair && merge_pref;
   const bool merge_gu = merge_ok && !routed_pair_swiglu;
   const bool merge_dn = merge_gu && !routed_pair;
   // Tile shapes of the routed GEMMs (step 5 and 6 below). Automatically
@@ -1068,7 +1083,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
   // automatically only below 32 expected rows per expert.
   const bool gather_rows =
       (p->gather_rows == 1 || (p->gather_rows == -1 && rows_per_expert < 32)) &&
-      !routed_pair_swiglu && !merge_gu;
+      !routed_pair_swiglu;
   // 4. offsets + m-tile prefix, stable permutation, 16-byte row copies (with a
   //    seat limit, only each expert's first `capacity` pairs get rows; none
   //    when the gate/up GEMM gathers them)

@@ -1,7 +1,7 @@
 """Seeded randomized GPU parity: random layer shapes, each run with the default
 kernel choices and with a random combination of the options that only change
 how the same arithmetic is scheduled (tile shapes, CTAs per SM, row gather,
-tile order, CTA-pair GEMMs). Those must give the default's bits exactly, and
+tile order, shared-expert placement, CTA-pair GEMMs). Those must give the default's bits exactly, and
 both must pass the oracle parity check; the fused router (different score
 summation order) is checked against the oracle only.
 """
@@ -42,6 +42,7 @@ def _draw(seed):
         opts["ctas_per_sm"] = 2
     opts["gather_rows"] = int(rng.choice([0, 1]))
     opts["interleave"] = int(rng.choice([-1, 0, 1]))
+    opts["merge_shared"] = int(rng.choice([-1, 0, 1]))
     pair = int(rng.choice([0, 1 << 40]))
     fused = bool(rng.integers(0, 2)) and n <= 512 and k <= 32
     return shape, opts, pair, fused

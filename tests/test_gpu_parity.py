@@ -243,8 +243,10 @@ def test_pair_and_single_kernels_agree_bitwise(pair_min_rows, wide):
 
 
 MERGE_CASES = [
-    # name, T, d, f, N_r, k, N_s, renorm, bias, expected variant names; the shared
-    # expert is too large for the side stream in all of them
+    # name, T, d, f, N_r, k, N_s, renorm, bias, expected variant names; the
+    # shared expert is too large for the side stream in the first three, small
+    # (merged by default, else forked) in the last two, whose gate/up GEMMs also
+    # gather their rows from x
     ("merged_both", 2048, 256, 640, 32, 2, 2, True, "none",
      ["grouped_gate_up[+shared]", "grouped_down[+shared]"]),
     ("merged_ragged", 2000, 320, 576, 40, 3, 3, False, "normal_var0.5",
@@ -253,6 +255,10 @@ MERGE_CASES = [
     # only the gate/up GEMM carries the shared tiles
     ("merged_gate_up_only", 2048, 256, 640, 16, 2, 2, True, "none",
      ["grouped_gate_up[+shared]", "grouped_down[pair]", "shared_down"]),
+    ("merged_small_gathered", 200, 256, 320, 96, 6, 1, True, "zipf1.1",
+     ["grouped_gate_up[+shared]", "grouped_down[+shared]"]),
+    ("merged_small_two_shared", 77, 192, 72, 40, 4, 2, False, "none",
+     ["grouped_gate_up[+shared]", "grouped_down[+shared]"]),
 ]
 
 
@@ -282,6 +288,31 @@ def test_merged_and_separate_shared_expert_agree_bitwise(case):
         outs.append(layer(inp["x"]).clone())
         torch.cuda.synchronize()
         assert layer.device_status() == 0
+    assert torch.equal(outs[0], outs[1])
+
+
+@pytest.mark.parametrize("options,merged", [({}, True), ({"merge_shared": 0}, False),
+                                            ({"swiglu_tile_cols": 64}, False),
+                                            ({"tile_rows": 64}, False)],
+                         ids=["default", "never", "narrow_tiles", "short_tiles"])
+def test_small_shared_expert_placement(options, merged):
+    # automatic placement: a small shared expert rides in the routed launches
+    # unless merging is switched off or the routed tile shape was chosen
+    # explicitly; then it runs on the side stream. Same bits either way.
+    from mixture_experts_ffn_expert_b200.layer import MoELayer
+    shape = LayerShape("small_shared", 160, 256, 256, 64, 6, 1, True, "zipf1.1")
+    inp = make_layer_inputs(shape, seed=10, device="cuda")
+    outs, names = [], []
+    for kw in ({"merge_shared": 0}, options):
+        layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
+                         shape.renorm, inp, bias=inp["bias"], device="cuda", **kw)
+        outs.append(layer(inp["x"]).clone())
+        torch.cuda.synchronize()
+        assert layer.device_status() == 0
+        names.append(layer.plan.kernel_names())
+    assert "shared_gate_up" in names[0], names[0]
+    assert ("grouped_gate_up[+shared]" in names[1]) == merged, names[1]
+    assert ("shared_gate_up" in names[1]) == (not merged), names[1]
     assert torch.equal(outs[0], outs[1])
 
 
@@ -677,15 +708,17 @@ def test_inconsistent_routing_state_is_reported_not_written_out_of_range():
     assert torch.equal(again, ref)
 
 
+@pytest.mark.parametrize("merge", [-1, 0], ids=["shared_merged", "shared_forked"])
 @pytest.mark.parametrize("name", ["decode_t128_d2048_f512_e512k10_s1", "tiny_t256_d128_f64_e31k7_s1"])
-def test_cuda_graph_replay_matches_stream_launch(name):
-    # the whole forward (including the shared expert's forked stream, when used)
-    # is captured once and replayed; replays must reproduce the plain result
+def test_cuda_graph_replay_matches_stream_launch(name, merge):
+    # the whole forward (with the small shared expert merged into the routed
+    # launches, or on its forked stream) is captured once and replayed; replays
+    # must reproduce the plain result
     from mixture_experts_ffn_expert_b200.layer import MoELayer
     shape = WORKLOADS[name]
     inp = make_layer_inputs(shape, seed=2, device="cuda")
     layer = MoELayer(shape.d, shape.f, shape.n_routed, shape.top_k, shape.n_shared,
-                     shape.renorm, inp, bias=inp["bias"], device="cuda")
+                     shape.renorm, inp, bias=inp["bias"], device="cuda", merge_shared=merge)
     x = inp["x"]
     want = layer(x).clone()
     out = torch.empty_like(x)

@@ -34,16 +34,18 @@ def _layer(shape, inp, **options):
                     shape.renorm, inp, bias=inp["bias"], device="cuda", **options)
 
 
-# the decode shape runs its shared expert on the plan's side stream; the tiny one too,
-# with a different routing kernel configuration; both with the split router (the
-# default) and the fused one (whose scan ticket lives in the scratch)
+# the decode shape and the tiny one (a different routing kernel configuration):
+# each with the split router (the default) and the fused one (whose scan ticket
+# lives in the scratch), and with its small shared expert merged into the routed
+# launches (the default) or forked onto the plan's side stream
+@pytest.mark.parametrize("merge", [-1, 0], ids=["shared_merged", "shared_forked"])
 @pytest.mark.parametrize("fused", [-1, 1], ids=["split_router", "fused_router"])
 @pytest.mark.parametrize("name", ["decode_t128_d2048_f512_e512k10_s1",
                                   "tiny_t256_d128_f64_e31k7_s1"])
-def test_noalloc_forward_matches_workspace_forward_twice(name, fused):
+def test_noalloc_forward_matches_workspace_forward_twice(name, fused, merge):
     shape = WORKLOADS[name]
     inp = make_layer_inputs(shape, seed=0, device="cuda")
-    layer = _layer(shape, inp, fused_router=fused)
+    layer = _layer(shape, inp, fused_router=fused, merge_shared=merge)
     ref = layer(inp["x"]).clone()                    # regular entry point, caller workspace
     routing_before = layer.routing()
     torch.cuda.synchronize()
