@@ -45,6 +45,7 @@ constexpr int kBHalfBytes = 128 * kBK * 2;     // 16 KB (one 128-row TMA box)
 constexpr int kBTileBytes = kBN * kBK * 2;     // 32 KB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
 constexpr int kNumAcc = 2;
+constexpr int kMaxGroups = 1024;               // expert groups a grouped launch may have
 constexpr int kTmemCols = kNumAcc * kBN;       // 512: the whole TMEM of the SM
 // Single-CTA kernel: warps 0 and 6 are TMA producers taking alternate stages,
 // warp 1 issues MMAs, warps 2..5 run the epilogue. Measured on B200 with
@@ -321,10 +322,27 @@ __global__ void __launch_bounds__(kGemmThreads, OCC)
   // operand are written by it
   pdl_wait();
   if (P.group_offsets) {
-    for (int i = threadIdx.x; i <= num_groups; i += blockDim.x) {
-      s_off[i] = P.group_offsets[i];
-      s_mp[i] = P.group_mtiles[i];
-      if (s_mp_b) s_mp_b[i] = P.group_mtiles_b[i];
+    // every load of the tables in flight at once (one L2 round trip, not one
+    // per pass of a strided loop): this sits between the dependency wait and
+    // the first operand load
+    constexpr int kPer = (kMaxGroups + 1 + kGemmThreads - 1) / kGemmThreads;
+    int o[kPer], m[kPer], mb[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = threadIdx.x + j * kGemmThreads;
+      const bool ok = i <= num_groups;
+      o[j] = ok ? P.group_offsets[i] : 0;
+      m[j] = ok ? P.group_mtiles[i] : 0;
+      mb[j] = ok && s_mp_b ? P.group_mtiles_b[i] : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = threadIdx.x + j * kGemmThreads;
+      if (i <= num_groups) {
+        s_off[i] = o[j];
+        s_mp[i] = m[j];
+        if (s_mp_b) s_mp_b[i] = mb[j];
+      }
     }
   } else if (threadIdx.x == 0) {
     s_off[0] = 0;

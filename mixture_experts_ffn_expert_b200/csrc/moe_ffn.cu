@@ -20,6 +20,9 @@
 #include "route.cuh"
 #include "router_sm100.cuh"
 
+static_assert(moe::kMaxGroups >= moe::kMaxRouted,
+              "a grouped GEMM launch holds the tables of every routed expert");
+
 namespace {
 
 thread_local std::string g_last_error;
@@ -58,6 +61,12 @@ struct Layout {
   size_t rt_smem;         // its dynamic shared memory
 };
 
+// Router score tiles are 128 columns wide: the epilogue of a tile (TMEM to
+// registers to fp32 stores, about 0.6 us per 32 columns on B200) is the
+// router GEMM's longest phase when the reduction is split K-wise over the SMs,
+// so narrower tiles on twice the CTAs halve it (512-expert decode step: the
+// epilogue took 4.9 us with 256-column tiles, 2.3 us with 128).
+constexpr int kRouterCols = 128;
 constexpr size_t kRouterMinSmem = 116 * 1024;   // one fused-router CTA per SM (see below)
 
 }  // namespace
@@ -230,11 +239,14 @@ Layout make_layout(const moe_plan* p, int64_t T) {
     L.subs_per_base = 1;
     L.n_base = L.n_chunks;
     // split-K of the router GEMM so that it occupies most SMs even for few tokens
-    const int64_t tiles = ((T + moe::kBM - 1) / moe::kBM) * ((p->n_routed + moe::kBN - 1) / moe::kBN);
+    const int64_t tiles =
+        ((T + moe::kBM - 1) / moe::kBM) * ((p->n_routed + kRouterCols - 1) / kRouterCols);
     const int num_kb = (p->d + moe::kBK - 1) / moe::kBK;
-    // at most 8 splits, and at most 128 partial scores held per lane in route_topk
+    // at most 4 splits (the partial sums cost route_topk instruction fetch and
+    // loads: on the 512-expert decode step 4 splits measured 2.2 us faster
+    // than 8), and at most 128 partial scores held per lane in route_topk
     const int npl = (p->n_routed + 31) / 32;
-    const int64_t cap = npl <= 16 ? 8 : 128 / npl;
+    const int64_t cap = npl <= 32 ? 4 : 128 / npl;
     int64_t sp = tiles > 0 ? p->num_sms / tiles : 1;
     sp = sp < 1 ? 1 : (sp > cap ? cap : sp);
     if (sp > num_kb) sp = num_kb;
@@ -427,11 +439,13 @@ bool launch_gemm(Launcher& L, cudaStream_t s, const char* name, const CUtensorMa
   if (grid < 1) grid = 1;
   moe::GemmParams q = prm;
   if (!x) q.x_tiles = 0;
-  // variant tag: output columns when not the widest tile, 64-row tiles, two
-  // CTAs per SM, or the shared expert merged in
+  // variant tag of a routed launch: output columns when not the widest tile,
+  // 64-row tiles, two CTAs per SM, or the shared expert merged in (the dense
+  // launches - router scores, shared expert - have fixed tiles)
   char tag[32] = "";
   const int out_cols = MODE == moe::kEpiSwiGLU ? BN / 2 : BN;
-  const bool narrow = out_cols < (MODE == moe::kEpiSwiGLU ? 128 : 256);
+  const bool narrow =
+      prm.group_offsets != nullptr && out_cols < (MODE == moe::kEpiSwiGLU ? 128 : 256);
   if (q.x_tiles > 0)
     snprintf(tag, sizeof(tag), "[+shared]");
   else if (narrow || TM == 64 || OCC == 2)
@@ -505,7 +519,7 @@ int set_kernel_attributes() {
   if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess)
     return fail(MOE_CUDA_ERROR, "cudaFuncSetAttribute failed: %s",
                 cudaGetErrorString(e1 != cudaSuccess ? e1 : (e2 != cudaSuccess ? e2 : e3)));
-  const cudaError_t en[4] = {
+  const cudaError_t en[5] = {
       cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiSwiGLU, 64, 64>, attr,
                            int(moe::gemm_smem_bytes<64, 64>(moe::kMaxRouted))),
       cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiSwiGLU, 64, 128>, attr,
@@ -513,6 +527,8 @@ int set_kernel_attributes() {
       cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiBF16, 128, 64>, attr,
                            int(moe::gemm_smem_bytes<128, 64>(moe::kMaxRouted))),
       cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiBF16, 128, 128>, attr,
+                           int(moe::gemm_smem_bytes<128, 128>(moe::kMaxRouted))),
+      cudaFuncSetAttribute(moe::moe_gemm_kernel<moe::kEpiF32, 128, 128>, attr,
                            int(moe::gemm_smem_bytes<128, 128>(moe::kMaxRouted)))};
   for (cudaError_t e : en)
     if (e != cudaSuccess)
@@ -983,7 +999,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.dense_rows = static_cast<int>(T);
     g.K = d;
     g.N = nr;
-    g.n_tiles = (nr + 255) / 256;
+    g.n_tiles = (nr + kRouterCols - 1) / kRouterCols;
     g.out = scores;
     g.ldo = Lw.lds;
     g.status = status;
@@ -991,7 +1007,8 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
     g.kb_per_split = Lw.router_kb_per;
     g.split_stride = static_cast<long long>(T) * Lw.lds;
     const int tiles = static_cast<int>((T + 127) / 128) * g.n_tiles * g.k_splits;
-    if (!launch_gemm<moe::kEpiF32>(L, main_st, "router_gemm", mX, mWg, mWg, g, tiles))
+    if (!launch_gemm<moe::kEpiF32, kRouterCols>(L, main_st, "router_gemm", mX, mWg, mWg, g,
+                                                 tiles))
       return L.status;
   }
   // 2. softmax + top-k + gates + per-chunk histogram
@@ -1008,8 +1025,7 @@ int moe_forward(moe_plan_t p, int64_t T, const moe_bf16_t* x, const moe_bf16_t* 
 #define MOE_TOPK_S(N)                                                                       \
   if (sp <= 1) MOE_TOPK(N, 1);                                                              \
   else if (sp <= 2) MOE_TOPK(N, 2);                                                         \
-  else if (sp <= 4) MOE_TOPK(N, 4);                                                         \
-  else MOE_TOPK(N, 8)
+  else MOE_TOPK(N, 4)
     if (npl <= 1) { MOE_TOPK_S(1); }
     else if (npl <= 2) { MOE_TOPK_S(2); }
     else if (npl <= 4) { MOE_TOPK_S(4); }

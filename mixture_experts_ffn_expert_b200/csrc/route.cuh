@@ -23,6 +23,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <climits>
+
 #include "ptx_sm100.cuh"
 
 namespace moe {
@@ -122,6 +124,15 @@ __device__ __forceinline__ void route_token(float (&v)[NPL], const float* __rest
 // `splits` (<= MAXS) fp32 partial sums (split-K of the router GEMM),
 // `split_stride` elements apart, and are added in split order; all partial
 // loads of a lane are issued before the first add.
+//
+// The kernel starts early (programmatic dependent launch) while the router
+// GEMM still runs, and each warp first runs its token body once on no data -
+// score loads and stores switched off - before the dependency wait: the
+// instructions (several KB, run once per warp) and the bias are then cached
+// when the scores arrive. After an L2 flush, or another layer's weight stream,
+// fetching them cold took longer than the selection itself (512-expert decode
+// step: the kernel ended 4.6 us earlier with the warm-up). Both passes run the
+// same code (the pass loop is not unrolled).
 template <int NPL, int MAXS>
 __global__ void __launch_bounds__(kRouteThreads)
     route_topk_kernel(const float* __restrict__ scores, int lds, int splits,
@@ -133,41 +144,54 @@ __global__ void __launch_bounds__(kRouteThreads)
   extern __shared__ int s_hist[];               // [n_routed]
   pdl_launch_dependents();
   for (int e = threadIdx.x; e < n_routed; e += blockDim.x) s_hist[e] = 0;
-  pdl_wait();                                   // scores come from the router GEMM
-  __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x;
   const int t_begin = chunk * tpc;
   const int t_end = min(T, t_begin + tpc);
-  for (int t = t_begin + warp; t < t_end; t += kRouteThreads / 32) {
-    const float* row = scores + static_cast<long long>(t) * lds;
-    float part[MAXS][NPL];
+  int warm = 0;                                 // the dry pass's (unused) selection
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    const bool dry = pass == 0;
+    if (!dry) {
+      pdl_wait();                               // scores come from the router GEMM
+      __syncthreads();
+    }
+    const int t_stop = dry ? min(t_end, t_begin + warp + 1) : t_end;   // dry: one token
+    for (int t = t_begin + warp; t < t_stop; t += kRouteThreads / 32) {
+      const float* row = scores + static_cast<long long>(t) * lds;
+      float part[MAXS][NPL];
 #pragma unroll
-    for (int sp = 0; sp < MAXS; ++sp)
+      for (int sp = 0; sp < MAXS; ++sp)
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+          const int e = lane + 32 * i;
+          part[sp][i] = (!dry && sp < splits && e < n_routed) ? row[sp * split_stride + e] : 0.0f;
+        }
+      float v[NPL];
 #pragma unroll
       for (int i = 0; i < NPL; ++i) {
-        const int e = lane + 32 * i;
-        part[sp][i] = (sp < splits && e < n_routed) ? row[sp * split_stride + e] : 0.0f;
+        float a = part[0][i];
+#pragma unroll
+        for (int sp = 1; sp < MAXS; ++sp) a += part[sp][i];
+        v[i] = a;
       }
-    float v[NPL];
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      float a = part[0][i];
-#pragma unroll
-      for (int sp = 1; sp < MAXS; ++sp) a += part[sp][i];
-      v[i] = a;
-    }
-    int my_e;
-    float my_g;
-    route_token<NPL>(v, bias, n_routed, top_k, renorm, bias_select_only, lane, my_e, my_g);
-    if (lane < top_k) {
-      const long long o = static_cast<long long>(t) * top_k + lane;
-      idx[o] = my_e;
-      gate[o] = my_g;
-      atomicAdd(&s_hist[my_e], 1);
+      int my_e;
+      float my_g;
+      route_token<NPL>(v, bias, n_routed, top_k, renorm, bias_select_only, lane, my_e, my_g);
+      if (dry) {
+        warm += my_e;
+        continue;
+      }
+      if (lane < top_k) {
+        const long long o = static_cast<long long>(t) * top_k + lane;
+        idx[o] = my_e;
+        gate[o] = my_g;
+        atomicAdd(&s_hist[my_e], 1);
+      }
     }
   }
+  if (warm == INT_MIN) atomicAdd(&s_hist[0], 0);   // keeps the dry pass (never true; adds 0)
   __syncthreads();
   for (int e = threadIdx.x; e < n_routed; e += blockDim.x)
     chunk_counts[static_cast<long long>(e) * n_chunks + chunk] = s_hist[e];
