@@ -5,6 +5,8 @@ tile order, shared-expert placement, CTA-pair GEMMs). Those must give the defaul
 both must pass the oracle parity check; the fused router (different score
 summation order) is checked against the oracle only.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -15,7 +17,7 @@ from parity import full_parity
 
 pytestmark = pytest.mark.gpu
 
-N_LAYERS = 40
+N_LAYERS = int(os.environ.get("MOE_FUZZ_LAYERS", "40"))   # more for a longer soak
 
 
 def _draw(seed):
