@@ -148,7 +148,8 @@ struct moe_plan {
   long long timed_forwards = 0;     // forwards that recorded events
   int cur_set = 0;
   bool events_made = false;
-  // the shared expert runs on a forked stream, concurrently with the routing
+  // stream and events for a shared expert forked beside the routing (a small
+  // one that is not merged) or beside the routed GEMMs (SHARED_CONCURRENT)
   cudaStream_t side = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
   // device address of the allocation-free forward's static scratch in this
