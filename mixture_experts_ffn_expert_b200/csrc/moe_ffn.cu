@@ -243,11 +243,10 @@ Layout make_layout(const moe_plan* p, int64_t T) {
     const int64_t tiles =
         ((T + moe::kBM - 1) / moe::kBM) * ((p->n_routed + kRouterCols - 1) / kRouterCols);
     const int num_kb = (p->d + moe::kBK - 1) / moe::kBK;
-    // at most 4 splits (the partial sums cost route_topk instruction fetch and
-    // loads: on the 512-expert decode step 4 splits measured 2.2 us faster
-    // than 8), and at most 128 partial scores held per lane in route_topk
-    const int npl = (p->n_routed + 31) / 32;
-    const int64_t cap = npl <= 32 ? 4 : 128 / npl;
+    // at most 4 splits: the partial sums cost route_topk instruction fetch and
+    // loads (on the 512-expert decode step 4 splits measured 2.2 us faster
+    // than 8), and 4 keeps a lane's partial scores at 4 x 32 at most (N_r <= 1024)
+    const int64_t cap = 4;
     int64_t sp = tiles > 0 ? p->num_sms / tiles : 1;
     sp = sp < 1 ? 1 : (sp > cap ? cap : sp);
     if (sp > num_kb) sp = num_kb;
